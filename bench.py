@@ -1,0 +1,493 @@
+#!/usr/bin/env python3
+"""Benchmark of the DSA layer on B200.
+
+Headline: DSA-layer decode tokens/s at 128K context — 4 sequences of 131072
+cached tokens, 64 heads, indexer 32 x 128, top_k 2048 — one step being one
+dsa_layer_forward (indexer -> top-k -> sparse attention) over the batch.  The
+JSON line also carries prefill tokens/s on one 16384-token sequence, the
+roofline fraction of the dominant kernel, an end-to-end number through host
+buffers, and the CPU oracle timed on the host as a baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+For N > 1 launch one process per GPU with torch.distributed.run; every rank
+runs an independent replica (the layer has no exchange step), timing is the
+max over ranks and `value` counts the tokens of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dsa_lightning_indexer_b200 import synth  # noqa: E402
+
+METRIC = "DSA-layer decode tokens/s at 128K ctx + prefill tokens/s; % HBM / bf16 TC peak"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ------------------------------------------------------------------ misc --
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained",
+                                                     p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML in a background thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []  # (t, sm_mhz, reasons_mask)
+        self.period = period_s
+        self.stop_flag = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id \
+                if hasattr(torch.cuda.get_device_properties(device_index), "pci_bus_id") else None
+            if bus:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            else:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                ids = [int(x) for x in vis.split(",") if x.strip().isdigit()]
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(ids[device_index] if ids else
+                                                           device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:  # noqa: BLE001
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, int(rs)))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self.stop_flag.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "sampled inside the timed region"
+        if not inside:  # very short timed region: take the samples bracketing it
+            before = [s for s in self.samples if s[0] < t0][-2:]
+            after = [s for s in self.samples if s[0] > t1][:2]
+            inside = before + after
+            note = "timed region shorter than the sampling period; bracketing samples"
+        mask = 0
+        for s in inside:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        mhz = [s[1] for s in inside]
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+# -------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is one query row of the
+    128K decode workload, computed in full (score all 131072 keys, select,
+    attend) in double precision on the host cores."""
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    wl = synth.decode_b4_128k()
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    a = (wl.q_offsets, wl.kv_offsets, wl.ctx_lens)
+
+    def step(i):
+        r = np.array([i % wl.Nq], np.int64)
+        oracle.dsa_layer(*a, wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, wl.top_k, wl.scale,
+                         sample=r)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "one query row of the 128K decode workload per step "
+                                   "(all 131072 keys scored, top-2048, 64-head attention), "
+                                   "rows cycled over the 4 sequences"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl):
+    return {"workload": wl.name, "batch": wl.B, "ctx": int(wl.ctx_lens.max()),
+            "heads": wl.H, "index_heads": synth.HI, "index_dim": synth.DI,
+            "latent_dim": synth.D, "value_dim": synth.DV, "top_k": wl.top_k,
+            "global_batch": wl.B, "seq_len": int(wl.ctx_lens.max()), "parallelism": "replicas",
+            "l2": "two rotating input copies; each step streams 134 MB of indexer keys, "
+                  "more than the 126 MB L2"}
+
+
+# ------------------------------------------------------------- our arm --
+
+def decode_bytes(wl):
+    """Algorithmic bytes of one layer step: indexer keys scanned, selected KV rows
+    gathered, per-query inputs read and outputs written."""
+    L = wl.ctx_lens.astype(np.int64)
+    nsel = np.minimum(wl.top_k, L)
+    kidx = int((L * synth.DI * 2).sum())
+    kv = int((nsel * synth.D * 2).sum())
+    per_q = wl.H * synth.D * 2 + synth.HI * synth.DI * 2 + synth.HI * 4 \
+        + wl.H * synth.DV * 4 + wl.H * 4 + wl.top_k * 4
+    return {"k_idx": kidx, "kv": kv, "query_io": per_q * wl.Nq,
+            "total": kidx + kv + per_q * wl.Nq}
+
+
+def indexer_bytes(wl):
+    L = wl.ctx_lens.astype(np.int64)
+    return int((L * synth.DI * 2).sum()) + wl.Nq * (synth.HI * synth.DI * 2 + synth.HI * 4)
+
+
+def indexer_causal_flops(wl):
+    """2 * 32 * 128 flops per (query, visible key) pair."""
+    pos = wl.positions()
+    return float(2 * synth.HI * synth.DI) * float((pos + 1).sum())
+
+
+def attn_num_splits(Nq, H, top_k, sms=148):
+    """Mirror of the library's split planning (used to count launches)."""
+    base = Nq * ((H + 63) // 64)
+    if base <= 0 or base >= sms:
+        return 1
+    max_split = (top_k + 31) // 32
+    n = min((sms + base - 1) // base, max_split)
+    if n <= 1:
+        return 1
+    per = ((top_k + n - 1) // n + 31) // 32 * 32
+    return (top_k + per - 1) // per
+
+
+def launches_per_layer(wl):
+    seqs = int((np.diff(wl.q_offsets) > 0).sum())
+    return (seqs + 63) // 64 + 1 + 1 + (1 if attn_num_splits(wl.Nq, wl.H, wl.top_k) > 1 else 0)
+
+
+def run_ours(args):
+    rank, local_rank, world = env_rank()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from dsa_lightning_indexer_b200 import binding as bd
+
+    peaks = load_peaks()
+    wl = synth.decode_b4_128k()
+    copies = [bd.DeviceWorkload(wl, dev)]
+    # a second copy of every input so consecutive steps never find their data in L2
+    c2 = bd.DeviceWorkload.__new__(bd.DeviceWorkload)
+    c2.__dict__.update(copies[0].__dict__)
+    for name in ("q_idx", "w", "k_idx", "q", "kv"):
+        setattr(c2, name, getattr(copies[0], name).clone())
+    c2.ws = torch.zeros_like(copies[0].ws)
+    copies.append(c2)
+    out, lse, idx = copies[0].new_outputs()
+
+    def step(i):
+        copies[i & 1].forward(out, lse, idx)
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    for c in copies:
+        bd.check_device_status(c.ws)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.05)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record()
+    for i in range(args.steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if dist:
+        dist.barrier()
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    for c in copies:
+        bd.check_device_status(c.ws)
+    ms_step = ms / args.steps
+    value = wl.Nq * world * args.steps / (ms / 1e3)
+
+    # --- per-kernel times: the same step as three C-ABI calls, events between them
+    ktimes = kernel_times(bd, copies, wl, args.steps, dev)
+    kb = indexer_bytes(wl)
+    k1_s = ktimes["indexer_score_us"] * 1e-6
+    achieved = kb / k1_s / 1e9
+    db = decode_bytes(wl)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_of(wl),
+        "roofline": {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": None, "peak_source": peaks["source"],
+                     "algorithmic_bytes_per_launch": kb},
+        "layer_roofline": {"algorithmic_bytes_per_step": db["total"],
+                           "achieved_gbs": db["total"] / (ms_step * 1e-3) / 1e9,
+                           "frac": db["total"] / (ms_step * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "kernel_times_us": ktimes,
+        "gpu_launches": launches_per_layer(wl) * args.steps,
+        "clocks": sampler.summary(t0, t1),
+    }
+    if not args.no_e2e:
+        line["e2e"] = e2e_decode(bd, wl, copies[0], args.steps, max(args.warmup, 3), dev, world,
+                                 dist)
+    if not args.no_prefill:
+        line["prefill"] = prefill_bench(bd, dev, peaks, args)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def kernel_times(bd, copies, wl, steps, dev):
+    """Average device time of each kernel of the step, from CUDA events on the
+    launching stream around the three C-ABI calls that make up the layer."""
+    n = max(3, min(steps, 200))
+    c0 = copies[0]
+    ld = (int(wl.ctx_lens.max()) + 3) // 4 * 4
+    scores = torch.empty(wl.Nq, ld, dtype=torch.float32, device=dev)
+    out, lse, idx = c0.new_outputs()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for i in range(n + 2):
+        c = copies[i & 1]
+        e = ev[i - 2] if i >= 2 else None
+        if e:
+            e[0].record()
+        bd.indexer_score(c.batch, c.q_idx, c.w, c.k_idx, scores, ld, c.ws)
+        if e:
+            e[1].record()
+        bd.topk(c.batch, scores, ld, c.top_k, idx, c.ws)
+        if e:
+            e[2].record()
+        bd.sparse_attn(c.batch, c.q, c.kv, idx, c.top_k, c.scale, out, lse, c.ws)
+        if e:
+            e[3].record()
+    torch.cuda.synchronize()
+    k1 = np.mean([e[0].elapsed_time(e[1]) for e in ev]) * 1e3
+    k2 = np.mean([e[1].elapsed_time(e[2]) for e in ev]) * 1e3
+    k3 = np.mean([e[2].elapsed_time(e[3]) for e in ev]) * 1e3
+    return {"indexer_score_us": float(k1), "topk_us": float(k2), "sparse_attn_us": float(k3),
+            "launches_timed": n}
+
+
+def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
+    """Decode step through host buffers: the step's new inputs (queries, indexer
+    queries and weights, and the new token's rows of both caches) are copied from
+    pinned host memory into the resident caches, the layer runs, and its output,
+    log-sum-exp and index sets are read back into pinned host memory."""
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+    h_q = pin(wl.q.view(np.int16))
+    h_qi = pin(wl.q_idx.view(np.int16))
+    h_w = pin(wl.w)
+    new_rows = [int(wl.kv_offsets[b] + wl.ctx_lens[b] - 1) for b in range(wl.B)]
+    h_krow = pin(wl.k_idx[new_rows].view(np.int16))
+    h_vrow = pin(wl.kv[new_rows].view(np.int16))
+    out, lse, idx = dw.new_outputs()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h_idx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    q16, qi16 = dw.q.view(torch.int16), dw.q_idx.view(torch.int16)
+    k16, v16 = dw.k_idx.view(torch.int16), dw.kv.view(torch.int16)
+
+    def step():
+        q16.copy_(h_q, non_blocking=True)
+        qi16.copy_(h_qi, non_blocking=True)
+        dw.w.copy_(h_w, non_blocking=True)
+        for j, r in enumerate(new_rows):
+            k16[r].copy_(h_krow[j], non_blocking=True)
+            v16[r].copy_(h_vrow[j], non_blocking=True)
+        dw.forward(out, lse, idx)
+        h_out.copy_(out, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+        h_idx.copy_(idx, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    bd.check_device_status(dw.ws)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_qi, h_w, h_krow, h_vrow))
+    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
+    return {"value": wl.Nq * world * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms / steps}
+
+
+def prefill_bench(bd, dev, peaks, args):
+    """One 16384-token causal prefill (64 heads, top_k 2048, planted indexer keys)."""
+    wl = synth.prefill_16k()
+    dw = bd.DeviceWorkload(wl, dev)
+    out, lse, idx = dw.new_outputs()
+    ld = (int(wl.ctx_lens.max()) + 3) // 4 * 4
+    scores = torch.empty(wl.Nq, ld, dtype=torch.float32, device=dev)
+    n = max(1, min(args.prefill_steps, 10))
+    for _ in range(2):
+        dw.forward(out, lse, idx)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        dw.forward(out, lse, idx)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    k1 = []
+    k2 = []
+    k3 = []
+    for _ in range(n):
+        ev[0].record()
+        bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws)
+        ev[1].record()
+        bd.topk(dw.batch, scores, ld, dw.top_k, idx, dw.ws)
+        ev[2].record()
+        bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, dw.top_k, dw.scale, out, lse, dw.ws)
+        ev[3].record()
+        torch.cuda.synchronize()
+        k1.append(ev[0].elapsed_time(ev[1]))
+        k2.append(ev[1].elapsed_time(ev[2]))
+        k3.append(ev[2].elapsed_time(ev[3]))
+    bd.check_device_status(dw.ws)
+    fl = indexer_causal_flops(wl)
+    k1s = float(np.mean(k1)) * 1e-3
+    tf = fl / k1s / 1e12
+    return {"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
+            "steps": n, "indexer_ms": k1s * 1e3, "topk_ms": float(np.mean(k2)),
+            "sparse_attn_ms": float(np.mean(k3)),
+            "indexer_roofline": {"bound": "tensor", "achieved": tf,
+                                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                 "frac": tf / peaks["bf16_tflops"], "causal_flops": fl}}
+
+
+def cpu_baseline(wl):
+    """The oracle, as it stands, on the host cores: all 4 query rows of one step."""
+    import oracle
+    oracle.build()
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    a = (wl.q_offsets, wl.kv_offsets, wl.ctx_lens)
+    t0 = time.perf_counter()
+    oracle.dsa_layer(*a, wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, wl.top_k, wl.scale)
+    dt = time.perf_counter() - t0
+    return {"value": wl.Nq / dt, "unit": UNIT, "cores": min(threads, wl.Nq), "kind": "oracle",
+            "sample": f"one full step of the workload ({wl.Nq} query rows, OpenMP over rows, "
+                      f"{dt:.1f} s)"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill-steps", type=int, default=3)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

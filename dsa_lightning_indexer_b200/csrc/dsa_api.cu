@@ -1,0 +1,363 @@
+// C ABI of the DSA layer: argument validation, workspace layout and launch
+// sequencing.  Every entry point validates everything it is given before it
+// enqueues any work, so a failing call leaves all outputs untouched.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/dsa.h"
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      return nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+namespace {
+
+// Split planning uses a fixed SM count so workspace sizes do not depend on
+// which device (or whether any device) is present.
+constexpr int kPlanSms = 148;
+
+struct BatchInfo {
+  int64_t max_len;     // longest context
+  int64_t cache_rows;  // kv_offsets[B]
+};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsa_status check_batch(const dsa_batch* b, BatchInfo* info) {
+  if (!b || b->B < 0 || b->Nq < 0) return DSA_ERR_INVALID_ARG;
+  info->max_len = 0;
+  info->cache_rows = 0;
+  if (b->B == 0) return b->Nq == 0 ? DSA_OK : DSA_ERR_INVALID_ARG;
+  if (!b->q_offsets || !b->kv_offsets || !b->ctx_lens || !b->h_q_offsets || !b->h_kv_offsets ||
+      !b->h_ctx_lens) {
+    return DSA_ERR_INVALID_ARG;
+  }
+  if (b->h_q_offsets[0] != 0 || b->h_q_offsets[b->B] != b->Nq || b->h_kv_offsets[0] < 0) {
+    return DSA_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < b->B; ++i) {
+    const int64_t nq = static_cast<int64_t>(b->h_q_offsets[i + 1]) - b->h_q_offsets[i];
+    const int64_t cap = b->h_kv_offsets[i + 1] - b->h_kv_offsets[i];
+    const int64_t L = b->h_ctx_lens[i];
+    if (nq < 0 || cap < 0 || L < 0 || nq > L || L > cap) return DSA_ERR_INVALID_ARG;
+    if (L > info->max_len) info->max_len = L;
+  }
+  info->cache_rows = b->h_kv_offsets[b->B];
+  // Row coordinates of the tensor maps are 32-bit.
+  if (info->cache_rows >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(b->Nq) * kIdxHeads >= (int64_t(1) << 31)) {
+    return DSA_ERR_UNSUPPORTED;
+  }
+  return DSA_OK;
+}
+
+dsa_status check_topk(int top_k) {
+  if (top_k < 1) return DSA_ERR_INVALID_ARG;
+  if (top_k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status check_heads(int H) {
+  if (H < 1) return DSA_ERR_INVALID_ARG;
+  if (H > kMaxHeads) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+dsa_status check_ptr(const void* p) {
+  if (!p) return DSA_ERR_INVALID_ARG;
+  return aligned16(p) ? DSA_OK : DSA_ERR_UNSUPPORTED;
+}
+
+// Workspace: [control 256 B][scores, layer forward only][attention partials].
+struct WsLayout {
+  size_t scores_off, scores_bytes, part_off, part_bytes, total;
+  int64_t ld;
+  int n_split;
+};
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bool scores,
+                 bool attn) {
+  WsLayout w;
+  w.ld = static_cast<int64_t>(round_up(static_cast<size_t>(info.max_len), 4));
+  w.scores_off = kControlBytes;
+  w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
+  w.part_off = w.scores_off + w.scores_bytes;
+  w.n_split = attn ? attn_num_splits(b->Nq, H, top_k, kPlanSms) : 1;
+  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.n_split), 256) : 0;
+  w.total = w.part_off + w.part_bytes;
+  return w;
+}
+
+dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+// The current device must be compute capability 10.0 (B200, sm_100a code).
+dsa_status check_device(int* num_sms) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_NOT_SM100;
+  }
+  static int cached_sms[64];
+  static int cached_ok[64];  // 0 unknown, 1 sm_100, 2 other
+  static std::mutex mu;
+  if (dev >= 0 && dev < 64) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached_ok[dev] == 0) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return DSA_ERR_CUDA;
+      }
+      cached_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
+      cached_sms[dev] = sms;
+    }
+    if (cached_ok[dev] != 1) return DSA_ERR_NOT_SM100;
+    *num_sms = cached_sms[dev];
+    return DSA_OK;
+  }
+  return DSA_ERR_NOT_SM100;
+}
+
+inline dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+inline unsigned* err_word(void* ws) {
+  return &reinterpret_cast<Control*>(ws)->err;
+}
+
+#define DSA_TRY(expr)                  \
+  do {                                 \
+    const dsa_status s_ = (expr);      \
+    if (s_ != DSA_OK) return s_;       \
+  } while (0)
+
+IndexerArgs indexer_args(const dsa_batch* b, const BatchInfo& info, const uint16_t* q_idx,
+                         const float* w, const uint16_t* k_idx, float* scores, int64_t ld,
+                         void* ws, int num_sms) {
+  IndexerArgs a;
+  a.B = b->B;
+  a.h_q_offsets = b->h_q_offsets;
+  a.h_kv_offsets = b->h_kv_offsets;
+  a.h_ctx_lens = b->h_ctx_lens;
+  a.Nq = b->Nq;
+  a.cache_rows = info.cache_rows;
+  a.q_idx = q_idx;
+  a.w = w;
+  a.k_idx = k_idx;
+  a.scores = scores;
+  a.ld = ld;
+  a.err = err_word(ws);
+  a.num_sms = num_sms;
+  return a;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t flags) {
+  (void)flags;
+  BatchInfo info;
+  if (check_batch(batch, &info) != DSA_OK || check_heads(H) != DSA_OK ||
+      check_topk(top_k) != DSA_OK) {
+    return 0;
+  }
+  return plan_ws(batch, info, H, top_k, true, true).total;
+}
+
+dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,
+                             const uint16_t* k_idx, float* scores, int64_t ld_scores, void* ws,
+                             size_t ws_bytes, void* stream) {
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  if (batch->Nq == 0) return DSA_OK;
+  DSA_TRY(check_ptr(q_idx));
+  DSA_TRY(check_ptr(w));
+  DSA_TRY(check_ptr(k_idx));
+  DSA_TRY(check_ptr(scores));
+  if (ld_scores < info.max_len || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kControlBytes));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  return cuda_status(launch_indexer_score(
+      indexer_args(batch, info, q_idx, w, k_idx, scores, ld_scores, ws, sms),
+      static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scores, int top_k,
+                    int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  DSA_TRY(check_topk(top_k));
+  if (batch->Nq == 0) return DSA_OK;
+  DSA_TRY(check_ptr(scores));
+  DSA_TRY(check_ptr(idx));
+  if (ld_scores < info.max_len || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
+  DSA_TRY(check_ws(ws, ws_bytes, kControlBytes));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  TopkArgs a;
+  a.B = batch->B;
+  a.Nq = batch->Nq;
+  a.q_offsets = batch->q_offsets;
+  a.ctx_lens = batch->ctx_lens;
+  a.scores = scores;
+  a.ld = ld_scores;
+  a.top_k = top_k;
+  a.idx = idx;
+  return cuda_status(launch_topk(a, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, const uint16_t* kv,
+                           const int32_t* idx, int top_k, float scale, float* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  DSA_TRY(check_heads(H));
+  DSA_TRY(check_topk(top_k));
+  if (batch->Nq == 0) return DSA_OK;
+  DSA_TRY(check_ptr(q));
+  DSA_TRY(check_ptr(kv));
+  DSA_TRY(check_ptr(idx));
+  DSA_TRY(check_ptr(out));
+  if (lse) DSA_TRY(check_ptr(lse));
+  if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  const WsLayout L = plan_ws(batch, info, H, top_k, false, true);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  AttnArgs a;
+  a.B = batch->B;
+  a.Nq = batch->Nq;
+  a.q_offsets = batch->q_offsets;
+  a.kv_offsets = batch->kv_offsets;
+  a.q = q;
+  a.H = H;
+  a.kv = kv;
+  a.idx = idx;
+  a.top_k = top_k;
+  a.scale = scale;
+  a.out = out;
+  a.lse = lse;
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
+  a.n_split = L.n_split;
+  a.num_sms = sms;
+  return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
+                             const uint16_t* q_idx, const float* w, const uint16_t* k_idx,
+                             const uint16_t* kv, int top_k, float scale, float* out, float* lse,
+                             int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags,
+                             void* stream) {
+  (void)flags;
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  DSA_TRY(check_heads(H));
+  DSA_TRY(check_topk(top_k));
+  if (batch->Nq == 0) return DSA_OK;
+  DSA_TRY(check_ptr(q));
+  DSA_TRY(check_ptr(q_idx));
+  DSA_TRY(check_ptr(w));
+  DSA_TRY(check_ptr(k_idx));
+  DSA_TRY(check_ptr(kv));
+  DSA_TRY(check_ptr(out));
+  DSA_TRY(check_ptr(idx));
+  if (lse) DSA_TRY(check_ptr(lse));
+  if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  const WsLayout L = plan_ws(batch, info, H, top_k, true, true);
+  DSA_TRY(check_ws(ws, ws_bytes, L.total));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* const scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.scores_off);
+
+  DSA_TRY(cuda_status(launch_indexer_score(
+      indexer_args(batch, info, q_idx, w, k_idx, scores, L.ld, ws, sms), st)));
+
+  TopkArgs t;
+  t.B = batch->B;
+  t.Nq = batch->Nq;
+  t.q_offsets = batch->q_offsets;
+  t.ctx_lens = batch->ctx_lens;
+  t.scores = scores;
+  t.ld = L.ld;
+  t.top_k = top_k;
+  t.idx = idx;
+  DSA_TRY(cuda_status(launch_topk(t, st)));
+
+  AttnArgs a;
+  a.B = batch->B;
+  a.Nq = batch->Nq;
+  a.q_offsets = batch->q_offsets;
+  a.kv_offsets = batch->kv_offsets;
+  a.q = q;
+  a.H = H;
+  a.kv = kv;
+  a.idx = idx;
+  a.top_k = top_k;
+  a.scale = scale;
+  a.out = out;
+  a.lse = lse;
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
+  a.n_split = L.n_split;
+  a.num_sms = sms;
+  return cuda_status(launch_sparse_attn(a, st));
+}
+
+dsa_status dsa_check_device_status(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kControlBytes) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned host_err = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemcpy(&host_err, err_word(ws), sizeof(host_err), cudaMemcpyDeviceToHost) !=
+          cudaSuccess) {
+    return DSA_ERR_CUDA;
+  }
+  if (host_err != 0) {
+    if (cudaMemset(err_word(ws), 0, sizeof(unsigned)) != cudaSuccess) return DSA_ERR_CUDA;
+    return DSA_ERR_DEVICE_TIMEOUT;
+  }
+  return DSA_OK;
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_DEVICE_TIMEOUT: return "DSA_ERR_DEVICE_TIMEOUT";
+    case DSA_ERR_NOT_SM100: return "DSA_ERR_NOT_SM100";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,179 @@
+/*
+ * dsa.h — C ABI of the B200 (sm_100a) DSA sparse-attention layer.
+ *
+ * The layer replaces full-attention MLA in 24 of the 93 layers of
+ * Kimi-K3.1-Pro (llama.cpp b12180 news: aiaulis.com paragraphs 2-3;
+ * aiunderstanding.org "What happened"; devotd.net section 1 and its
+ * configuration table).  It runs in three steps:
+ *
+ *   1. a lightning indexer of 32 heads x 128 dims, no RoPE, scores every
+ *      earlier cached token of each query:
+ *        I[q,s] = sum_h w[q,h] * ReLU( q_idx[q,h,:] . k_idx[s,:] ),  s <= p(q)
+ *      (the pages name the scorer but print no formula; this is the usual
+ *      lightning-indexer form and is an assumption of this library);
+ *   2. the top_k highest-scoring positions are kept (top_k = 2048 in the
+ *      released checkpoint), ties broken by lower position;
+ *   3. attention runs only over the kept rows of a shared key-only latent
+ *      cache: K = the whole 576-wide row, V = its first 512 entries
+ *      (devotd.net section 2: a key-only cache per DSA layer).
+ *
+ * With top_k >= p+1 for every query the result is full causal attention
+ * (aiaulis.com paragraph 7; devotd.net section 4).
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - Numbers: bf16 tensors are passed as uint16_t bit patterns; scores,
+ *    weights, outputs are IEEE fp32.  Products are exact, accumulation is
+ *    fp32, softmax runs in fp32.
+ *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller,
+ *    except the h_* fields of dsa_batch, which are HOST mirrors used to plan
+ *    the launch without a device sync.  The library allocates nothing, keeps
+ *    no state between calls and is re-entrant; calls on different streams
+ *    must use different workspaces.
+ *  - Asynchrony: all work is enqueued on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Nothing synchronises except
+ *    dsa_check_device_status.
+ *  - Errors: every call validates all arguments before it launches anything;
+ *    on any error it returns a non-OK status and writes nothing.  No C++
+ *    exception crosses this boundary.  Kernel-side failures (a bounded wait
+ *    that ran out) set an error word in the workspace, read back by
+ *    dsa_check_device_status.
+ *  - Alignment: every tensor pointer must be 16-byte aligned.
+ *  - Fixed shapes: indexer 32 heads x 128, latent row 576, value width 512,
+ *    1 <= top_k <= 2048, 1 <= H <= 128.  Other values give
+ *    DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSA_B200_H_
+#define DSA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_INDEX_HEADS 32   /* indexer heads (devotd.net configuration table) */
+#define DSA_INDEX_DIM 128    /* indexer key length (same table) */
+#define DSA_LATENT_DIM 576   /* latent key row width */
+#define DSA_VALUE_DIM 512    /* V = first 512 entries of the latent row */
+#define DSA_MAX_TOPK 2048    /* keys kept per query (same table) */
+#define DSA_MAX_HEADS 128    /* attention heads per query */
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, inconsistent batch */
+  DSA_ERR_UNSUPPORTED = 2,    /* shape outside the fixed set, misaligned pointer */
+  DSA_ERR_WORKSPACE = 3,      /* ws NULL or smaller than the call needs */
+  DSA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  DSA_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (device side) */
+  DSA_ERR_NOT_SM100 = 6       /* current device is not compute capability 10.0 */
+} dsa_status;
+
+/*
+ * A batch of sequences.  Sequence b owns
+ *   - query rows [q_offsets[b], q_offsets[b+1]) of every per-query tensor
+ *     (nq_b = q_offsets[b+1] - q_offsets[b] >= 0, q_offsets[0] = 0,
+ *     q_offsets[B] = Nq);
+ *   - cache rows [kv_offsets[b], kv_offsets[b+1]) of k_idx and kv (the two
+ *     caches share row numbering); its context is the first ctx_lens[b] of
+ *     them, so 1 <= ctx_lens[b] <= kv_offsets[b+1] - kv_offsets[b] whenever
+ *     nq_b > 0, and nq_b <= ctx_lens[b].
+ * The current tokens are already appended to the caches: the j-th query of
+ * sequence b sits at position p = ctx_lens[b] - nq_b + j and sees positions
+ * 0..p, its own included (decode: nq_b = 1, p = L-1; prefill: nq_b = L).
+ * The device arrays and their host mirrors must hold the same values.
+ */
+typedef struct {
+  int32_t B;                    /* sequences, >= 0 */
+  int32_t Nq;                   /* total query rows = q_offsets[B] */
+  const int32_t* q_offsets;     /* device, [B+1] */
+  const int64_t* kv_offsets;    /* device, [B+1] */
+  const int32_t* ctx_lens;      /* device, [B] */
+  const int32_t* h_q_offsets;   /* host mirror, [B+1] */
+  const int64_t* h_kv_offsets;  /* host mirror, [B+1] */
+  const int32_t* h_ctx_lens;    /* host mirror, [B] */
+} dsa_batch;
+
+/* Bytes of workspace that dsa_layer_forward needs for this batch; it is also
+ * enough for every other call on the same batch, H and top_k.  Returns 0 for
+ * an invalid batch.  `flags` is reserved, pass 0. */
+DSA_API size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t flags);
+
+/*
+ * Step 1, the lightning indexer (aiaulis.com paragraph 2: a light indexer
+ * scores earlier tokens; devotd.net configuration table: 32 heads, key
+ * length 128; aiunderstanding.org "What happened": no RoPE).
+ *   q_idx   [Nq, 32, 128] bf16   indexer queries (no rotary embedding applied)
+ *   w       [Nq, 32]      fp32   per-query head weights
+ *   k_idx   [rows, 128]   bf16   indexer key cache
+ *   scores  [Nq, ld_scores] fp32 out: scores[r, s] for s = 0..p(r);
+ *                                entries past p(r) are left untouched.
+ *   ld_scores >= max_b ctx_lens[b], a multiple of 4.
+ * Runs on tcgen05 tensor cores (bf16 products, fp32 accumulation).
+ */
+DSA_API dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,
+                             const uint16_t* k_idx, float* scores, int64_t ld_scores, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Step 2, top-k selection (aiaulis.com paragraphs 2-3: attention only for the
+ * highest-scored tokens, 2048 of them; devotd.net configuration table).
+ *   scores [Nq, ld_scores] fp32, read for s = 0..p(r) only.
+ *   idx    [Nq, top_k] int32 out: the n = min(top_k, p+1) positions with the
+ *          largest (score, -position), i.e. score descending with ties to the
+ *          lower position, written in ascending position order, followed by
+ *          top_k - n entries of -1.  Positions are sequence-relative.
+ *   -0.0 and +0.0 are the same score.  NaN scores are not supported.
+ */
+DSA_API dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scores, int top_k,
+                    int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 3, attention over the selected rows only (aiaulis.com paragraph 2;
+ * devotd.net section 2: the key-only cache serves as both K and V).
+ *   q    [Nq, H, 576] bf16     attention queries
+ *   kv   [rows, 576]  bf16     shared latent cache; V = first 512 entries
+ *   idx  [Nq, top_k]  int32    sequence-relative positions, -1 = unused slot;
+ *                              every other entry must satisfy 0 <= idx <= p(r)
+ *   out  [Nq, H, 512] fp32     out: softmax_s(scale * q.kv[s]) weighted sum of
+ *                              kv[s, :512] over the listed s
+ *   lse  [Nq, H] fp32 or NULL  out: natural-log log-sum-exp of the logits
+ *   A row whose idx holds no valid entry gets out = 0 and lse = -inf.
+ */
+DSA_API dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, const uint16_t* kv,
+                           const int32_t* idx, int top_k, float scale, float* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole DSA layer: dsa_indexer_score -> dsa_topk -> dsa_sparse_attn,
+ * with the scores kept in the workspace.  Arguments as above; `idx` receives
+ * the selected index sets, `out`/`lse` the attention output.  `flags` is
+ * reserved, pass 0.
+ */
+DSA_API dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
+                             const uint16_t* q_idx, const float* w, const uint16_t* k_idx,
+                             const uint16_t* kv, int top_k, float scale, float* out, float* lse,
+                             int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags,
+                             void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that the
+ * kernels of earlier calls on this workspace may have set.  Returns DSA_OK,
+ * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the stream itself reports an
+ * error. */
+DSA_API dsa_status dsa_check_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+DSA_API const char* dsa_status_string(dsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H_ */

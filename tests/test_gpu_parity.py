@@ -1,0 +1,240 @@
+"""CUDA path against the CPU oracle, through the C ABI (needs a B200).
+
+Each step is checked alone (scores; selection on the oracle's own scores;
+attention on the oracle's own index sets) and as the fused layer, on seeded
+synthetic inputs: small ragged cases spanning several tiles with ragged
+tails, the edge cases, and the specified workloads at full size (every query
+of the decode workloads; a seeded sample of rows of the 16K prefill).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dsa_lightning_indexer_b200 import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from dsa_lightning_indexer_b200 import binding as bd
+
+
+def _up4(x):
+    return (int(x) + 3) // 4 * 4
+
+
+def _args(wl):
+    return (wl.q_offsets, wl.kv_offsets, wl.ctx_lens)
+
+
+def gpu_scores(wl):
+    dw = bd.DeviceWorkload(wl)
+    ld = _up4(wl.ctx_lens.max())
+    scores = torch.full((wl.Nq, ld), float("nan"), device="cuda")
+    bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws)
+    bd.check_device_status(dw.ws)
+    return scores.cpu().numpy()
+
+
+def gpu_topk(wl, scores_np, top_k):
+    b = bd.Batch.from_workload(wl)
+    ld = scores_np.shape[1]
+    scores = torch.from_numpy(np.ascontiguousarray(scores_np, np.float32)).cuda()
+    idx = torch.full((wl.Nq, top_k), -7, dtype=torch.int32, device="cuda")
+    ws = bd.alloc_workspace(b, 1, top_k)
+    bd.topk(b, scores, ld, top_k, idx, ws)
+    bd.check_device_status(ws)
+    return idx.cpu().numpy()
+
+
+def gpu_attn(wl, idx_np):
+    dw = bd.DeviceWorkload(wl)
+    top_k = idx_np.shape[1]
+    ws = bd.alloc_workspace(dw.batch, wl.H, top_k)
+    idx = torch.from_numpy(np.ascontiguousarray(idx_np, np.int32)).cuda()
+    out = torch.full((wl.Nq, wl.H, 512), float("nan"), device="cuda")
+    lse = torch.full((wl.Nq, wl.H), float("nan"), device="cuda")
+    bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, top_k, wl.scale, out, lse, ws)
+    bd.check_device_status(ws)
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def gpu_layer(wl):
+    dw = bd.DeviceWorkload(wl)
+    out, lse, idx = dw.forward()
+    bd.check_device_status(dw.ws)
+    return out.cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+
+
+# Small shapes: several 128-key tiles, ragged tails, every queries-per-group
+# variant (1, 2, 4, 8 per sequence), unaligned cache offsets and spare rows.
+SMALL = {
+    "prefill_T1024": lambda: synth.prefill(1024, 16, 256, seed=100),
+    "ragged_mixed": lambda: synth.custom([300, 129, 1000, 1, 128, 517], [3, 1, 7, 1, 2, 517], 16,
+                                         64, seed=101, caps=[301, 140, 1000, 9, 128, 517]),
+    "decode_ragged": lambda: synth.custom([5000, 777, 128, 129, 2], [1, 1, 1, 1, 1], 64, 128,
+                                          seed=102),
+    "two_queries": lambda: synth.custom([700, 900], [2, 2], 8, 100, seed=103),
+    "four_queries": lambda: synth.custom([257, 1023], [4, 3], 8, 33, seed=104),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_indexer_scores_match_oracle(name):
+    wl = SMALL[name]()
+    got = gpu_scores(wl)
+    ref = oracle.indexer_scores(*_args(wl), wl.q_idx, wl.w, wl.k_idx, ld=got.shape[1])
+    worst = parity.check_scores(got, ref, wl)
+    # entries past each query's position are left untouched
+    pos = wl.positions()
+    for r in range(wl.Nq):
+        assert np.isnan(got[r, pos[r] + 1:]).all(), r
+    print(f"{name}: worst relative score error {worst:.2e}")
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_topk_exact_on_oracle_scores(name):
+    wl = SMALL[name]()
+    ref_scores = oracle.indexer_scores(*_args(wl), wl.q_idx, wl.w, wl.k_idx,
+                                       ld=_up4(wl.ctx_lens.max()))
+    want = oracle.topk(*_args(wl), ref_scores, wl.top_k)
+    got = gpu_topk(wl, np.nan_to_num(ref_scores, nan=0.0), wl.top_k)
+    assert np.array_equal(got, want)
+
+
+def _score_rows(lens, seed, kind):
+    """Long synthetic score rows (one query per sequence) with forced ties."""
+    lens = np.asarray(lens)
+    g = np.random.Generator(np.random.PCG64(seed))
+    ld = _up4(lens.max())
+    sc = np.zeros((lens.size, ld), np.float32)
+    for r, L in enumerate(lens):
+        if kind == "normal":
+            sc[r, :L] = g.standard_normal(L, dtype=np.float32)
+        elif kind == "coarse":            # few distinct values: ties everywhere
+            sc[r, :L] = g.integers(-3, 4, size=L).astype(np.float32) * 0.5
+        elif kind == "zeros":             # -0 and +0 mixed: one value
+            sc[r, :L] = np.where(g.random(L) < 0.5, -0.0, 0.0).astype(np.float32)
+        elif kind == "heavy":             # wide dynamic range, negatives
+            sc[r, :L] = (g.standard_normal(L) * np.exp(g.standard_normal(L) * 8)).astype(
+                np.float32)
+    return sc
+
+
+@pytest.mark.parametrize("kind", ["normal", "coarse", "zeros", "heavy"])
+def test_topk_long_rows(kind):
+    lens = [131072, 40000, 2049, 2048, 100]
+    wl = synth.Workload("rows", np.arange(len(lens) + 1, dtype=np.int32),
+                        np.concatenate([[0], np.cumsum(lens)]).astype(np.int64),
+                        np.array(lens, np.int32), None, None, None, None, None, 2048, 1.0)
+    sc = _score_rows(lens, 7, kind)
+    want = oracle.topk(*_args(wl), sc, 2048)
+    got = gpu_topk(wl, sc, 2048)
+    assert np.array_equal(got, want)
+
+
+ATTN = {
+    "prefill_h16": lambda: synth.prefill(300, 16, 64, seed=110),
+    "prefill_h20": lambda: synth.prefill(200, 20, 48, seed=111),
+    "decode_h64_split": lambda: synth.custom([3000, 2100, 64], [1, 1, 1], 64, 2048, seed=112),
+    "decode_h128": lambda: synth.custom([2500], [1], 128, 1024, seed=113),
+    "mixed_h1": lambda: synth.custom([90, 40], [5, 40], 1, 32, seed=114),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ATTN))
+def test_sparse_attention_matches_oracle(name):
+    wl = ATTN[name]()
+    _, idx, _, _ = oracle.dsa_layer(*_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, wl.top_k,
+                                    wl.scale)
+    ref_out, ref_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, idx, wl.scale)
+    out, lse = gpu_attn(wl, idx)
+    e = parity.check_attention(out, lse, ref_out, ref_lse)
+    print(f"{name}: max |out err| {e[0]:.2e}, max |lse err| {e[1]:.2e}")
+
+
+def test_sparse_attention_scattered_unused_slots():
+    wl = synth.custom([500], [3], 16, 96, seed=115)
+    g = np.random.Generator(np.random.PCG64(5))
+    idx = np.full((3, 96), -1, np.int32)
+    for r, p in enumerate(wl.positions()):
+        chosen = np.sort(g.choice(p + 1, size=60, replace=False))
+        slots = np.sort(g.choice(96, size=60, replace=False))
+        idx[r, slots] = chosen
+    idx[2, :] = -1  # a row with nothing selected: out = 0, lse = -inf
+    ref_out, ref_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, idx, wl.scale)
+    out, lse = gpu_attn(wl, idx)
+    assert (out[2] == 0).all() and np.isneginf(lse[2]).all()
+    parity.check_attention(out[:2], lse[:2], ref_out[:2], ref_lse[:2])
+
+
+def _layer_check(wl, rows=None, full_equivalence=False):
+    got_out, got_lse, got_idx = gpu_layer(wl)
+    sample = None if rows is None else rows
+    ld = _up4(wl.ctx_lens.max())
+    ref_scores, ref_idx, ref_out, ref_lse = oracle.dsa_layer(
+        *_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, wl.top_k, wl.scale, sample=sample,
+        ld=ld)
+    swaps = parity.check_selection(got_idx, ref_idx, ref_scores, wl, rows)
+    # attention checked on the GPU's own selection (equal to the oracle's up to ties)
+    att_out, att_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, got_idx, wl.scale,
+                                          sample=sample)
+    e = parity.check_attention(got_out, got_lse, att_out, att_lse, rows)
+    if swaps == 0:
+        parity.check_attention(got_out, got_lse, ref_out, ref_lse, rows)
+    if full_equivalence:
+        full_out, full_lse = oracle.full_causal_attn(*_args(wl), wl.q, wl.kv, wl.scale,
+                                                     sample=sample)
+        parity.check_attention(got_out, got_lse, full_out, full_lse, rows)
+    print(f"{wl.name}: boundary swaps {swaps}, max |out err| {e[0]:.2e}, lse {e[1]:.2e}")
+    return got_out, got_idx
+
+
+def test_layer_tiny_prefill_topk_below_context():
+    out, _ = _layer_check(synth.tiny_prefill(256))
+    # forced below the context, later queries differ from full causal attention
+    wl = synth.tiny_prefill(256)
+    full, _ = oracle.full_causal_attn(*_args(wl), wl.q, wl.kv, wl.scale,
+                                      sample=np.arange(600, 1024))
+    assert np.abs(out[600:] - full[600:]).max() > 1e-2
+
+
+def test_layer_tiny_prefill_topk_covers_context_is_full_attention():
+    _layer_check(synth.tiny_prefill(2048), full_equivalence=True)
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_layer_small_shapes(name):
+    _layer_check(SMALL[name]())
+
+
+def test_layer_edge_cases():
+    # single token contexts, top_k = 1, one head, sequences without queries
+    _layer_check(synth.custom([1, 1, 5, 9], [1, 1, 5, 0], 1, 1, seed=120))
+    _layer_check(synth.custom([1, 130, 2], [1, 130, 2], 3, 2048, seed=121))
+
+
+def test_empty_batch_launches_nothing():
+    b = bd.Batch(np.zeros(1, np.int32), np.zeros(1, np.int64), np.zeros(0, np.int32))
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    fake = 1 << 16  # never dereferenced: there is nothing to compute
+    st = bd.lib.dsa_layer_forward(b.ref, fake, 64, fake, fake, fake, fake, 2048, 0.04, fake,
+                                  None, fake, ws.data_ptr(), 256, 0, None)
+    assert st == bd.OK
+    bd.check_device_status(ws)
+
+
+def test_layer_decode_b8_32k_full():
+    _layer_check(synth.decode_b8_32k())
+
+
+def test_layer_decode_b4_128k_full():
+    _layer_check(synth.decode_b4_128k())
+
+
+def test_layer_prefill_16k_sampled_rows():
+    wl = synth.prefill_16k()
+    must = list(range(64)) + list(range(2040, 2057)) + [wl.Nq - 1]
+    rows = parity.sample_rows(wl, 160, seed=2, must=must)
+    _layer_check(wl, rows=rows)
