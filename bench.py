@@ -217,22 +217,12 @@ def indexer_causal_flops(wl):
     return float(2 * synth.HI * synth.DI) * float((pos + 1).sum())
 
 
-def attn_num_splits(Nq, H, top_k, sms=148):
-    """Mirror of the library's split planning (used to count launches)."""
-    base = Nq * ((H + 63) // 64)
-    if base <= 0 or base >= sms:
-        return 1
-    max_split = (top_k + 31) // 32
-    n = min((sms + base - 1) // base, max_split)
-    if n <= 1:
-        return 1
-    per = ((top_k + n - 1) // n + 31) // 32 * 32
-    return (top_k + per - 1) // per
-
-
 def launches_per_layer(wl):
+    """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
+    sequences with queries), the top-k selection, the sparse attention (which
+    merges its own slices)."""
     seqs = int((np.diff(wl.q_offsets) > 0).sum())
-    return (seqs + 63) // 64 + 1 + 1 + (1 if attn_num_splits(wl.Nq, wl.H, wl.top_k) > 1 else 0)
+    return (seqs + 63) // 64 + 1 + 1
 
 
 def run_ours(args):

@@ -84,11 +84,12 @@ dsa_status check_ptr(const void* p) {
   return aligned16(p) ? DSA_OK : DSA_ERR_UNSUPPORTED;
 }
 
-// Workspace: [control 256 B][scores, layer forward only][attention partials].
+// Workspace: [control 256 B][scores, layer forward only][attention partials]
+// [attention arrival tickets].
 struct WsLayout {
-  size_t scores_off, scores_bytes, part_off, part_bytes, total;
+  size_t scores_off, scores_bytes, part_off, part_bytes, ticket_off, ticket_bytes, total;
   int64_t ld;
-  int n_split;
+  AttnPlan plan;
 };
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -100,9 +101,11 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.scores_off = kControlBytes;
   w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
   w.part_off = w.scores_off + w.scores_bytes;
-  w.n_split = attn ? attn_num_splits(b->Nq, H, top_k, kPlanSms) : 1;
-  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.n_split), 256) : 0;
-  w.total = w.part_off + w.part_bytes;
+  w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
+  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
+  w.ticket_off = w.part_off + w.part_bytes;
+  w.ticket_bytes = attn ? round_up(attn_ticket_bytes(b->Nq, w.plan), 256) : 0;
+  w.total = w.ticket_off + w.ticket_bytes;
   return w;
 }
 
@@ -231,6 +234,8 @@ dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scor
   a.ld = ld_scores;
   a.top_k = top_k;
   a.idx = idx;
+  a.max_len = info.max_len;
+  a.num_sms = sms;
   return cuda_status(launch_topk(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -266,8 +271,8 @@ dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.out = out;
   a.lse = lse;
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
-  a.n_split = L.n_split;
-  a.num_sms = sms;
+  a.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.ticket_off);
+  a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -310,6 +315,8 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   t.ld = L.ld;
   t.top_k = top_k;
   t.idx = idx;
+  t.max_len = info.max_len;
+  t.num_sms = sms;
   DSA_TRY(cuda_status(launch_topk(t, st)));
 
   AttnArgs a;
@@ -326,8 +333,8 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   a.out = out;
   a.lse = lse;
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
-  a.n_split = L.n_split;
-  a.num_sms = sms;
+  a.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.ticket_off);
+  a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, st));
 }
 

@@ -35,8 +35,21 @@ struct TopkArgs {
   int64_t ld;
   int top_k;
   int32_t* idx;
+  int64_t max_len;   // longest context in the batch
+  int num_sms;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+
+// How the attention launch covers (query row, head block, slice of the set).
+struct AttnPlan {
+  int hb;           // heads per CTA: 16, 32, 48 or 64
+  int head_blocks;  // ceil(H / hb)
+  int n_split;      // slices of the selected set per (row, head block)
+  int split_len;    // index slots per slice (multiple of 32)
+};
+AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms);
+size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p);
+size_t attn_ticket_bytes(int Nq, const AttnPlan& p);
 
 struct AttnArgs {
   int B;
@@ -51,14 +64,38 @@ struct AttnArgs {
   float scale;
   float* out;
   float* lse;
-  float* part;        // split partials (workspace), may be null when n_split == 1
-  int n_split;
-  int num_sms;
+  float* part;        // split partials (workspace); unused when plan.n_split == 1
+  int* tickets;       // arrival counters (workspace, zero between calls)
+  AttnPlan plan;
 };
-// Number of key splits the attention launch uses for this shape.
-int attn_num_splits(int Nq, int H, int top_k, int num_sms);
-size_t attn_partial_bytes(int Nq, int H, int n_split);
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+
+// Launches `kernel` on `stream` as a programmatic dependent of the work before
+// it (see pdl_wait), optionally as clusters of `cluster_x` CTAs.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Driver entry point for tensor-map encoding, resolved once through the
 // runtime (no link-time dependency on libcuda).

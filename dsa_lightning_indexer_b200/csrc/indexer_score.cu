@@ -31,7 +31,6 @@ namespace dsa {
 namespace {
 
 constexpr int kKeysPerTile = 128;
-constexpr int kStages = 4;
 constexpr int kKTileBytes = kKeysPerTile * kIdxDim * 2;  // 32 KB
 constexpr int kKBoxBytes = kKTileBytes / 2;              // 128 rows x 64 dims
 constexpr int kThreads = 192;
@@ -56,6 +55,8 @@ template <int QT>
 struct Cfg {
   static constexpr int N = 32 * QT;
   static constexpr int kQBufs = QT <= 4 ? 2 : 1;
+  // K ring depth: deep for decode (HBM streaming), shallower when Q is large.
+  static constexpr int kStages = QT <= 2 ? 6 : 4;
   static constexpr int kQBoxBytes = N * 128;
   static constexpr int kQBytes = 2 * kQBoxBytes;
   static constexpr int kTmemCols = 2 * N < 32 ? 32 : 2 * N;
@@ -110,19 +111,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t k_smem = base + C::kQBufs * C::kQBytes;
   const uint32_t bars = base + C::kSmemData;
   auto full = [&](int s) { return bars + 8u * s; };
-  auto empty = [&](int s) { return bars + 8u * (kStages + s); };
-  auto qfull = [&](int i) { return bars + 8u * (2 * kStages + i); };
-  auto qempty = [&](int i) { return bars + 8u * (2 * kStages + 2 + i); };
-  auto tfull = [&](int i) { return bars + 8u * (2 * kStages + 4 + i); };
-  auto tempty = [&](int i) { return bars + 8u * (2 * kStages + 6 + i); };
+  auto empty = [&](int s) { return bars + 8u * (C::kStages + s); };
+  auto qfull = [&](int i) { return bars + 8u * (2 * C::kStages + i); };
+  auto qempty = [&](int i) { return bars + 8u * (2 * C::kStages + 2 + i); };
+  auto tfull = [&](int i) { return bars + 8u * (2 * C::kStages + 4 + i); };
+  auto tempty = [&](int i) { return bars + 8u * (2 * C::kStages + 6 + i); };
   uint32_t* const tmem_slot =
-      reinterpret_cast<uint32_t*>(base_ptr + C::kSmemData + 8 * (2 * kStages + 8));
+      reinterpret_cast<uint32_t*>(base_ptr + C::kSmemData + 8 * (2 * C::kStages + 8));
 
   const int warp = warp_id_uniform();
   const int lane = lane_id();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full(s), 1);
       mbar_init(empty(s), 1);
     }
@@ -146,6 +147,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  // Everything above overlapped the previous kernel; from here on memory is shared.
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int row = static_cast<int>(v.kv0 + static_cast<long long>(kt) * kKeysPerTile);
           tma_load_2d(kdst, &kmap, full(stage), 0, row, pol_stream);
           tma_load_2d(kdst + kKBoxBytes, &kmap, full(stage), 64, row, pol_stream);
-          if (++stage == kStages) {
+          if (++stage == C::kStages) {
             stage = 0;
             sph ^= 1u;
           }
@@ -217,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(empty(stage));
           tc_commit(tfull(acc));
-          if (++stage == kStages) {
+          if (++stage == C::kStages) {
             stage = 0;
             sph ^= 1u;
           }
@@ -359,8 +363,8 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.n_items = items;
     if (items == 0) continue;
     const int grid = std::min(items, a.num_sms);
-    indexer_score_kernel<QT><<<grid, kThreads, C::kSmemBytes, stream>>>(kmap, qmap, P);
-    e = cudaGetLastError();
+    e = launch_pdl(indexer_score_kernel<QT>, dim3(grid), dim3(kThreads), C::kSmemBytes, stream, 0,
+                   kmap, qmap, P);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

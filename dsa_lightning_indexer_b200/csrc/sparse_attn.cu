@@ -8,12 +8,14 @@
 //
 // Only the selected rows are read: each row is gathered once per CTA with
 // 16-byte cp.async copies into shared memory (double-buffered tiles of 32
-// rows) and used for both Q.K^T and P.V.  A CTA owns one query row, up to 64
+// rows) and used for both Q.K^T and P.V.  A CTA owns one query row, a block of
 // heads (16 per warp group of four warps) and a contiguous slice of the
-// selected set (split over CTAs when there are too few rows to fill the GPU;
-// a second kernel merges the slices with the log-sum-exp rule).  Softmax runs
-// online in fp32 in base 2.  P enters the P.V product as bf16 hi + lo parts,
-// so its rounding error stays near 2^-16 relative.
+// selected set.  With many query rows (prefill) a CTA takes 64 heads and the
+// whole set; with few rows (decode) it takes 16 heads and a slice, and the
+// last CTA to finish a (row, head block) merges the slices' partial results
+// with the log-sum-exp rule (an atomic ticket decides who is last; nobody
+// waits).  Softmax runs online in fp32 in base 2.  P enters the P.V product as
+// bf16 hi + lo parts, so its rounding error stays near 2^-16 relative.
 #include <algorithm>
 
 #include "dsa_common.cuh"
@@ -38,6 +40,7 @@ struct AttnParams {
   float* out;
   float* lse;
   float* part;          // [n_split][Nq][H][512 + 2] when n_split > 1
+  int* tickets;         // [Nq][head_blocks] arrival counters, zero between calls
   int B, Nq, H, top_k, n_split, split_len;
   float scale_log2;     // scale * log2(e)
 };
@@ -108,13 +111,15 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
   int* const tidx = reinterpret_cast<int*>(red + HB * 4);          // [2][kTileRows]
 
   const int r = blockIdx.x;
-  const int h0 = blockIdx.y * kHeadsPerCta;
+  const int h0 = blockIdx.y * HB;
   const int sp = blockIdx.z;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int hg = warp >> 2, qd = warp & 3;
   const int g = lane >> 2, c = lane & 3;
 
+  pdl_wait();
+  pdl_launch_dependents();
   const int b = owner_seq(P.q_offsets, P.B, r);
   const long long kv0 = P.kv_offsets[b];
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
@@ -174,6 +179,7 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
     const uint32_t kv_base = smem_u32(kvb);
     // ---- S = Q K^T for heads hrow..+15 and tile rows qd*8..+7 ------------
     float s[4] = {0.f, 0.f, 0.f, 0.f};
+    float s_odd[4] = {0.f, 0.f, 0.f, 0.f};  // second chain halves the MMA dependency depth
     {
       const uint32_t a_addr = q_base + ((hrow + (lane & 15)) * kRowPad + (lane >> 4) * 8) * 2;
       const uint32_t b_addr = kv_base + ((qd * 8 + (lane & 7)) * kRowPad + (lane >> 3) * 8) * 2;
@@ -184,8 +190,10 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
         ldsm_x4(a_addr + ks * 64 + 32, a4, a5, a6, a7);
         ldsm_x4(b_addr + ks * 64, b0, b1, b2, b3);
         mma_bf16_16816(s, a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(s, a4, a5, a6, a7, b2, b3);
+        mma_bf16_16816(s_odd, a4, a5, a6, a7, b2, b3);
       }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] += s_odd[i];
     }
     const int* const ti = tidx + buf * kTileRows;
     const bool v0 = ti[qd * 8 + 2 * c] >= 0, v1 = ti[qd * 8 + 2 * c + 1] >= 0;
@@ -326,36 +334,49 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
         base[static_cast<size_t>(hb8) * kRec + kValue + 1] = L_g8;
       }
     }
+    // The last CTA of this (row, head block) to arrive merges all slices.
+    __shared__ int is_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      int* const ticket = P.tickets + static_cast<size_t>(r) * gridDim.y + blockIdx.y;
+      const int t = atomicAdd(ticket, 1);
+      is_last = (t == P.n_split - 1);
+      if (is_last) *ticket = 0;  // every other slice has arrived: reset for the next call
+    }
+    __syncthreads();
+    if (is_last) {
+      __threadfence();
+      const size_t split_stride = static_cast<size_t>(P.Nq) * P.H * kRec;
+      for (int e = tid; e < HB * (kValue / 4); e += kThreads) {
+        const int hl = e / (kValue / 4), dv = (e - hl * (kValue / 4)) * 4;
+        const int h = h0 + hl;
+        if (h >= P.H) continue;
+        const float* const pr = P.part + (static_cast<size_t>(r) * P.H + h) * kRec;
+        float M = -INFINITY;
+        for (int q = 0; q < P.n_split; ++q) M = fmaxf(M, __ldcg(pr + q * split_stride + kValue));
+        float Lsum = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int q = 0; q < P.n_split; ++q) {
+          const float* const ps = pr + q * split_stride;
+          const float ms = __ldcg(ps + kValue);
+          if (ms == -INFINITY) continue;
+          const float wgt = exp2f(ms - M);
+          Lsum += wgt * __ldcg(ps + kValue + 1);
+          acc.x += wgt * __ldcg(ps + dv + 0);
+          acc.y += wgt * __ldcg(ps + dv + 1);
+          acc.z += wgt * __ldcg(ps + dv + 2);
+          acc.w += wgt * __ldcg(ps + dv + 3);
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        *reinterpret_cast<float4*>(P.out + (static_cast<size_t>(r) * P.H + h) * kValue + dv) =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (P.lse && dv == 0)
+          P.lse[static_cast<size_t>(r) * P.H + h] =
+              Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+      }
+    }
   }
-}
-
-// Merges split partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams P) {
-  constexpr int kRec = kValue + 2;
-  const int r = blockIdx.x, h = blockIdx.y;
-  const size_t rec = static_cast<size_t>(r) * P.H + h;
-  const size_t split_stride = static_cast<size_t>(P.Nq) * P.H * kRec;
-  const float* const base = P.part + rec * kRec;
-  float M = -INFINITY;
-  for (int s = 0; s < P.n_split; ++s) M = fmaxf(M, base[s * split_stride + kValue]);
-  float Lsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int dv = threadIdx.x * 4;
-  for (int s = 0; s < P.n_split; ++s) {
-    const float* const ps = base + s * split_stride;
-    const float ms = ps[kValue];
-    if (ms == -INFINITY) continue;
-    const float wgt = exp2f(ms - M);
-    Lsum += wgt * ps[kValue + 1];
-    acc.x += wgt * ps[dv + 0];
-    acc.y += wgt * ps[dv + 1];
-    acc.z += wgt * ps[dv + 2];
-    acc.w += wgt * ps[dv + 3];
-  }
-  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  *reinterpret_cast<float4*>(P.out + rec * kValue + dv) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (P.lse && threadIdx.x == 0) P.lse[rec] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
 template <int NG>
@@ -372,28 +393,42 @@ cudaError_t launch_ng(const AttnParams& P, int head_blocks, cudaStream_t stream)
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(P.Nq, head_blocks, P.n_split);
-  sparse_attn_kernel<NG><<<grid, NG * 128, smem, stream>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(sparse_attn_kernel<NG>, dim3(P.Nq, head_blocks, P.n_split), dim3(NG * 128),
+                    smem, stream, 0, P);
 }
 
 }  // namespace
 
-int attn_num_splits(int Nq, int H, int top_k, int num_sms) {
-  const long long base = static_cast<long long>(Nq) * ((H + kHeadsPerCta - 1) / kHeadsPerCta);
-  if (base <= 0 || base >= num_sms) return 1;
-  const int max_split = (top_k + kTileRows - 1) / kTileRows;
-  const int want = static_cast<int>((num_sms + base - 1) / base);
-  const int n = std::min(want, max_split);
-  if (n <= 1) return 1;
-  // Every split takes a whole number of tiles; drop splits that would be empty.
-  const int per = ((top_k + n - 1) / n + kTileRows - 1) / kTileRows * kTileRows;
-  return (top_k + per - 1) / per;
+AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms) {
+  AttnPlan p;
+  p.hb = std::min(kHeadsPerCta, (H + 15) / 16 * 16);
+  p.head_blocks = (H + p.hb - 1) / p.hb;
+  p.n_split = 1;
+  const long long rows = Nq;
+  if (rows * p.head_blocks < num_sms && rows > 0) {
+    // Few rows: 16 heads per CTA (two CTAs fit an SM) and slices of the set.
+    p.hb = 16;
+    p.head_blocks = (H + 15) / 16;
+    const long long base = rows * p.head_blocks;
+    const int want = static_cast<int>(std::max<long long>(1, 2LL * num_sms / base));
+    const int n = std::min(want, (top_k + kTileRows - 1) / kTileRows);
+    if (n > 1) {
+      const int per = ((top_k + n - 1) / n + kTileRows - 1) / kTileRows * kTileRows;
+      p.n_split = (top_k + per - 1) / per;
+    }
+  }
+  p.split_len = ((top_k + p.n_split - 1) / p.n_split + kTileRows - 1) / kTileRows * kTileRows;
+  return p;
 }
 
-size_t attn_partial_bytes(int Nq, int H, int n_split) {
-  if (n_split <= 1) return 0;
-  return static_cast<size_t>(n_split) * Nq * H * (kValue + 2) * sizeof(float);
+size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p) {
+  if (p.n_split <= 1) return 0;
+  return static_cast<size_t>(p.n_split) * Nq * H * (kValue + 2) * sizeof(float);
+}
+
+size_t attn_ticket_bytes(int Nq, const AttnPlan& p) {
+  if (p.n_split <= 1) return 0;
+  return static_cast<size_t>(Nq) * p.head_blocks * sizeof(int);
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
@@ -407,25 +442,20 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   P.out = a.out;
   P.lse = a.lse;
   P.part = a.part;
+  P.tickets = a.tickets;
   P.B = a.B;
   P.Nq = a.Nq;
   P.H = a.H;
   P.top_k = a.top_k;
-  P.n_split = std::max(1, a.n_split);
-  P.split_len = ((a.top_k + P.n_split - 1) / P.n_split + kTileRows - 1) / kTileRows * kTileRows;
+  P.n_split = a.plan.n_split;
+  P.split_len = a.plan.split_len;
   P.scale_log2 = a.scale * kLog2e;
-  const int head_blocks = (a.H + kHeadsPerCta - 1) / kHeadsPerCta;
-  const int ng = (std::min(a.H, kHeadsPerCta) + 15) / 16;
-  cudaError_t e;
-  switch (ng) {
-    case 1: e = launch_ng<1>(P, head_blocks, stream); break;
-    case 2: e = launch_ng<2>(P, head_blocks, stream); break;
-    case 3: e = launch_ng<3>(P, head_blocks, stream); break;
-    default: e = launch_ng<4>(P, head_blocks, stream); break;
+  switch (a.plan.hb / 16) {
+    case 1: return launch_ng<1>(P, a.plan.head_blocks, stream);
+    case 2: return launch_ng<2>(P, a.plan.head_blocks, stream);
+    case 3: return launch_ng<3>(P, a.plan.head_blocks, stream);
+    default: return launch_ng<4>(P, a.plan.head_blocks, stream);
   }
-  if (e != cudaSuccess || P.n_split == 1) return e;
-  attn_combine_kernel<<<dim3(a.Nq, a.H), 128, 0, stream>>>(P);
-  return cudaGetLastError();
 }
 
 }  // namespace dsa

@@ -122,9 +122,23 @@ def _score_rows(lens, seed, kind):
     return sc
 
 
+# Row sets that exercise every launch shape of the selection kernel: clusters
+# of 8 CTAs (few long rows), 4, 2 and 1 (many short rows), and the
+# single-CTA fallback for rows longer than eight shared-memory slices.
+ROW_SETS = {
+    "decode_4x128k": [131072] * 4,
+    "mixed_long": [131072, 40000, 2049, 2048, 100],
+    "twenty_50k": [50000] * 20,
+    "five_5000": [5000, 4999, 4097, 3000, 2500],
+    "many_3000": [3000] * 300,
+    "one_400k": [400000],
+}
+
+
+@pytest.mark.parametrize("rows", sorted(ROW_SETS))
 @pytest.mark.parametrize("kind", ["normal", "coarse", "zeros", "heavy"])
-def test_topk_long_rows(kind):
-    lens = [131072, 40000, 2049, 2048, 100]
+def test_topk_long_rows(kind, rows):
+    lens = ROW_SETS[rows]
     wl = synth.Workload("rows", np.arange(len(lens) + 1, dtype=np.int32),
                         np.concatenate([[0], np.cumsum(lens)]).astype(np.int64),
                         np.array(lens, np.int32), None, None, None, None, None, 2048, 1.0)
@@ -238,3 +252,19 @@ def test_layer_prefill_16k_sampled_rows():
     must = list(range(64)) + list(range(2040, 2057)) + [wl.Nq - 1]
     rows = parity.sample_rows(wl, 160, seed=2, must=must)
     _layer_check(wl, rows=rows)
+
+
+def test_repeated_calls_on_one_workspace_agree():
+    """Arrival tickets and other workspace state are left ready for the next call."""
+    wl = synth.custom([3000, 2500], [1, 1], 64, 2048, seed=130)
+    dw = bd.DeviceWorkload(wl)
+    first = [t.cpu().numpy() for t in dw.forward()]
+    for _ in range(3):
+        again = [t.cpu().numpy() for t in dw.forward()]
+        for a, b in zip(first, again):
+            assert np.array_equal(a, b)
+    bd.check_device_status(dw.ws)
+    _, idx, _, _ = oracle.dsa_layer(*_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, 2048,
+                                    wl.scale)
+    ref_out, ref_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, idx, wl.scale)
+    parity.check_attention(first[0], first[1], ref_out, ref_lse)
