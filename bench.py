@@ -259,6 +259,28 @@ def run_ours(args):
     for c in copies:
         bd.check_device_status(c.ws)
 
+    # A serving loop replays the decode step as a CUDA graph (one per input copy).
+    graphs = []
+    if not args.no_graph:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for ci in range(len(copies)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    step(ci)
+                graphs.append(g)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        for i in range(max(args.warmup, 3)):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % len(graphs)].replay()
+        else:
+            step(i)
+
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.05)
@@ -269,7 +291,7 @@ def run_ours(args):
     t0 = time.perf_counter()
     e0.record()
     for i in range(args.steps):
-        step(i)
+        timed_step(i)
     e1.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
@@ -283,6 +305,7 @@ def run_ours(args):
         ms = float(t.item())
     for c in copies:
         bd.check_device_status(c.ws)
+    del graphs
     ms_step = ms / args.steps
     value = wl.Nq * world * args.steps / (ms / 1e3)
 
@@ -297,7 +320,10 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": config_of(wl, len(copies)),
+        "data": "synthetic",
+        "config": dict(config_of(wl, len(copies)),
+                       launch="direct calls" if args.no_graph else "CUDA graph replay of "
+                       "dsa_layer_forward"),
         "roofline": None if args.no_kernel_times else {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": None, "peak_source": peaks["source"],
@@ -325,34 +351,54 @@ def run_ours(args):
 
 
 def kernel_times(bd, copies, wl, steps, dev):
-    """Average device time of each kernel of the step, from CUDA events on the
-    launching stream around the three C-ABI calls that make up the layer."""
-    n = max(3, min(steps, 200))
+    """Average device time of each kernel of the step: every C-ABI call of the
+    step captured alone, `reps` times (alternating input copies), in a CUDA
+    graph, and the graph timed with CUDA events on the launching stream."""
+    reps = 16
     c0 = copies[0]
     ld = (int(wl.ctx_lens.max()) + 3) // 4 * 4
     scores = torch.empty(wl.Nq, ld, dtype=torch.float32, device=dev)
     out, lse, idx = c0.new_outputs()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
-    for i in range(n + 2):
-        c = copies[i % len(copies)]
-        e = ev[i - 2] if i >= 2 else None
-        if e:
-            e[0].record()
+
+    def k1(c):
         bd.indexer_score(c.batch, c.q_idx, c.w, c.k_idx, scores, ld, c.ws)
-        if e:
-            e[1].record()
+
+    def k2(c):
         bd.topk(c.batch, scores, ld, c.top_k, idx, c.ws)
-        if e:
-            e[2].record()
+
+    def k3(c):
         bd.sparse_attn(c.batch, c.q, c.kv, idx, c.top_k, c.scale, out, lse, c.ws)
-        if e:
-            e[3].record()
+
+    for c in copies:  # warm: inputs of every later call are valid
+        k1(c), k2(c), k3(c)
     torch.cuda.synchronize()
-    k1 = np.mean([e[0].elapsed_time(e[1]) for e in ev]) * 1e3
-    k2 = np.mean([e[1].elapsed_time(e[2]) for e in ev]) * 1e3
-    k3 = np.mean([e[2].elapsed_time(e[3]) for e in ev]) * 1e3
-    return {"indexer_score_us": float(k1), "topk_us": float(k2), "sparse_attn_us": float(k3),
-            "launches_timed": n}
+    res = {}
+    side = torch.cuda.Stream(dev)
+    for name, fn in (("indexer_score_us", k1), ("topk_us", k2), ("sparse_attn_us", k3)):
+        g = torch.cuda.CUDAGraph()
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(reps):
+                    fn(copies[i % len(copies)])
+        torch.cuda.current_stream(dev).wait_stream(side)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        n = max(3, min(steps, 50))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = e0.elapsed_time(e1) * 1e3 / (n * reps)
+        del g
+    res["launches_timed"] = n * reps
+    res["method"] = "per-kernel CUDA graphs of 16 launches, CUDA events around replays"
+    for c in copies:
+        bd.check_device_status(c.ws)
+    return res
 
 
 def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
@@ -483,6 +529,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-times", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch each step directly instead of replaying a CUDA graph")
     ap.add_argument("--copies", type=int, default=2,
                     help="rotating copies of the decode inputs (L2 defeat)")
     args = ap.parse_args()

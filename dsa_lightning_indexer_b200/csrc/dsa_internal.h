@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace dsa {
 
 struct IndexerArgs {
@@ -69,6 +71,21 @@ struct AttnArgs {
   AttnPlan plan;
 };
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+
+// Raises a kernel's dynamic shared-memory limit to `bytes`, once per device
+// (the attribute call is not free, and launches may be captured in a graph).
+template <auto Kernel>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0ull && (done.load(std::memory_order_acquire) & bit) != 0ull) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0ull) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Launches `kernel` on `stream` as a programmatic dependent of the work before
 // it (see pdl_wait), optionally as clusters of `cluster_x` CTAs.

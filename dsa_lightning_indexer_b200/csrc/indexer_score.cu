@@ -314,9 +314,7 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
                       C::N)) {
     return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(indexer_score_kernel<QT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+  cudaError_t e = ensure_smem_limit<indexer_score_kernel<QT>>(C::kSmemBytes);
   if (e != cudaSuccess) return e;
 
   // Total key tiles, to size chunks so every SM gets several items.

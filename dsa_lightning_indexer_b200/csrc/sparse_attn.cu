@@ -389,9 +389,7 @@ size_t attn_smem_bytes() {
 template <int NG>
 cudaError_t launch_ng(const AttnParams& P, int head_blocks, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes<NG>();
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<NG>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_smem_limit<sparse_attn_kernel<NG>>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   return launch_pdl(sparse_attn_kernel<NG>, dim3(P.Nq, head_blocks, P.n_split), dim3(NG * 128),
                     smem, stream, 0, P);

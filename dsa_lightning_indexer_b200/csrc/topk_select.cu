@@ -392,9 +392,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   }
   P.slice = static_cast<int>(slice_of(cs));
   const size_t smem = 2 * kBins * sizeof(int) + static_cast<size_t>(P.slice) * sizeof(uint32_t);
-  cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  // The limit is raised once, to the largest slice any launch may use.
+  cudaError_t e = ensure_smem_limit<topk_cluster_kernel>(
+      static_cast<int>(2 * kBins * sizeof(int) + static_cast<size_t>(kMaxSlice) * sizeof(uint32_t)));
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_cluster_kernel, dim3(static_cast<unsigned>(a.Nq) * cs), dim3(kCThreads),
                     smem, stream, cs, P);
