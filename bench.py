@@ -217,12 +217,13 @@ def indexer_causal_flops(wl):
     return float(2 * synth.HI * synth.DI) * float((pos + 1).sum())
 
 
-def launches_per_layer(wl):
+def launches_per_layer(wl, sms=148):
     """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
-    sequences with queries), the top-k selection, the sparse attention (which
-    merges its own slices)."""
+    sequences with queries), the top-k selection, the sparse attention and,
+    when few rows split the selected set over CTAs, the merge of the slices."""
     seqs = int((np.diff(wl.q_offsets) > 0).sum())
-    return (seqs + 63) // 64 + 1 + 1
+    few_rows = wl.Nq * ((wl.H + 63) // 64) < sms
+    return (seqs + 63) // 64 + 1 + 1 + (1 if few_rows and wl.top_k > 32 else 0)
 
 
 def run_ours(args):

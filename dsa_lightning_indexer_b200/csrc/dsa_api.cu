@@ -84,13 +84,21 @@ dsa_status check_ptr(const void* p) {
   return aligned16(p) ? DSA_OK : DSA_ERR_UNSUPPORTED;
 }
 
-// Workspace: [control 256 B][scores, layer forward only][attention partials]
-// [attention arrival tickets].
+// Workspace: [control 256 B][scores][top-k histograms and candidate lists]
+// [attention partials]; the middle regions exist for dsa_layer_forward only.
 struct WsLayout {
-  size_t scores_off, scores_bytes, part_off, part_bytes, ticket_off, ticket_bytes, total;
+  size_t scores_off, scores_bytes, hist_off, hist_bytes, part_off, part_bytes, total;
   int64_t ld;
+  bool hist_topk;  // selection driven by histograms the indexer builds
   AttnPlan plan;
 };
+
+// Few long rows with one query per sequence (decode): the indexer builds the
+// score-key histograms and the selection makes one filtering pass.
+bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
+  return b->Nq > 0 && b->Nq <= kPlanSms && info.max_len >= 8192 &&
+         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B);
+}
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -100,12 +108,13 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.ld = static_cast<int64_t>(round_up(static_cast<size_t>(info.max_len), 4));
   w.scores_off = kControlBytes;
   w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
-  w.part_off = w.scores_off + w.scores_bytes;
+  w.hist_topk = scores && plan_hist_topk(b, info, top_k);
+  w.hist_off = w.scores_off + w.scores_bytes;
+  w.hist_bytes = w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k), 256) : 0;
+  w.part_off = w.hist_off + w.hist_bytes;
   w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
   w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
-  w.ticket_off = w.part_off + w.part_bytes;
-  w.ticket_bytes = attn ? round_up(attn_ticket_bytes(b->Nq, w.plan), 256) : 0;
-  w.total = w.ticket_off + w.ticket_bytes;
+  w.total = w.part_off + w.part_bytes;
   return w;
 }
 
@@ -174,6 +183,7 @@ IndexerArgs indexer_args(const dsa_batch* b, const BatchInfo& info, const uint16
   a.ld = ld;
   a.err = err_word(ws);
   a.num_sms = num_sms;
+  a.hist = nullptr;
   return a;
 }
 
@@ -271,7 +281,9 @@ dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.out = out;
   a.lse = lse;
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
-  a.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.ticket_off);
+  a.err = err_word(ws);
+  a.ctx_lens = batch->ctx_lens;
+  a.idx_prefix = false;
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
@@ -303,8 +315,10 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* const scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.scores_off);
 
-  DSA_TRY(cuda_status(launch_indexer_score(
-      indexer_args(batch, info, q_idx, w, k_idx, scores, L.ld, ws, sms), st)));
+  IndexerArgs ia = indexer_args(batch, info, q_idx, w, k_idx, scores, L.ld, ws, sms);
+  void* const hist_region = static_cast<uint8_t*>(ws) + L.hist_off;
+  if (L.hist_topk) ia.hist = static_cast<int*>(hist_region);
+  DSA_TRY(cuda_status(launch_indexer_score(ia, st)));
 
   TopkArgs t;
   t.B = batch->B;
@@ -317,7 +331,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   t.idx = idx;
   t.max_len = info.max_len;
   t.num_sms = sms;
-  DSA_TRY(cuda_status(launch_topk(t, st)));
+  DSA_TRY(cuda_status(L.hist_topk ? launch_topk_hist(t, hist_region, st) : launch_topk(t, st)));
 
   AttnArgs a;
   a.B = batch->B;
@@ -333,7 +347,9 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   a.out = out;
   a.lse = lse;
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.part_off);
-  a.tickets = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.ticket_off);
+  a.err = err_word(ws);
+  a.ctx_lens = batch->ctx_lens;
+  a.idx_prefix = true;  // produced by dsa_topk: valid positions first, then -1
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, st));
 }

@@ -17,6 +17,10 @@ constexpr int kValue = 512;      // value width (leading part of the latent row)
 constexpr int kMaxTopK = 2048;
 constexpr int kMaxHeads = 128;
 constexpr int kMaxSeqPerLaunch = 64;
+// Score-key histogram fused into the indexer for the top-k filter: the top
+// 12 bits of the order-preserving key.
+constexpr int kHistShift = 20;
+constexpr int kHistBins = 1 << (32 - kHistShift);
 
 // Error bits in the workspace control block.
 constexpr unsigned kErrTimeout = 1u;

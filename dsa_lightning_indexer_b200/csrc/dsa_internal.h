@@ -25,7 +25,11 @@ struct IndexerArgs {
   int64_t ld;
   unsigned* err;
   int num_sms;
+  int* hist;          // per-row score-key histograms to accumulate, or null
 };
+// True when the indexer launch for this batch processes one query per item
+// (the only case in which it can build the histograms).
+bool indexer_single_query_items(const int32_t* h_q_offsets, int B);
 cudaError_t launch_indexer_score(const IndexerArgs& a, cudaStream_t stream);
 
 struct TopkArgs {
@@ -41,9 +45,15 @@ struct TopkArgs {
   int num_sms;
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+// Selection driven by the histograms the indexer built (see IndexerArgs.hist):
+// `ws_region` holds them followed by the per-row candidate lists and
+// counters, topk_hist_ws_bytes() bytes in all, zero between calls.
+size_t topk_hist_ws_bytes(int Nq, int top_k);
+cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream);
 
 // How the attention launch covers (query row, head block, slice of the set).
 struct AttnPlan {
+  int tc;           // 1: tcgen05 kernel (many rows, 64 heads per CTA, no slices)
   int hb;           // heads per CTA: 16, 32, 48 or 64
   int head_blocks;  // ceil(H / hb)
   int n_split;      // slices of the selected set per (row, head block)
@@ -51,13 +61,13 @@ struct AttnPlan {
 };
 AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms);
 size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p);
-size_t attn_ticket_bytes(int Nq, const AttnPlan& p);
 
 struct AttnArgs {
   int B;
   int Nq;
   const int32_t* q_offsets;   // device
   const int64_t* kv_offsets;  // device
+  const int32_t* ctx_lens;    // device
   const uint16_t* q;
   int H;
   const uint16_t* kv;
@@ -67,9 +77,11 @@ struct AttnArgs {
   float* out;
   float* lse;
   float* part;        // split partials (workspace); unused when plan.n_split == 1
-  int* tickets;       // arrival counters (workspace, zero between calls)
+  unsigned* err;      // workspace error word (bounded waits)
+  bool idx_prefix;    // valid entries are the first min(top_k, p+1) slots of each row
   AttnPlan plan;
 };
+cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes`, once per device

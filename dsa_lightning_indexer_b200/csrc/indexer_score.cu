@@ -20,6 +20,12 @@
 //   warps 2-5  epilogue: tcgen05.ld, ReLU, weighted head sum, fp32 store.
 // A work item is (sequence, group of QT queries, chunk of key tiles); items
 // are dealt to CTAs in snake order so causal prefill work balances.
+//
+// Optionally (one query per item), the epilogue also counts each stored score
+// into a 4096-bin histogram of the top 12 bits of its order-preserving key
+// (shared memory, one aggregated atomic per warp per distinct bin), flushed to
+// the row's global histogram after each item; the top-k selection then needs
+// only one filtering pass over the row.
 #include <string.h>
 
 #include <algorithm>
@@ -49,6 +55,7 @@ struct IdxParams {
   float* scores;
   long long ld;
   unsigned* err;
+  int* hist;  // [Nq][kHistBins] score-key histograms, or null
 };
 
 template <int QT>
@@ -56,11 +63,12 @@ struct Cfg {
   static constexpr int N = 32 * QT;
   static constexpr int kQBufs = QT <= 4 ? 2 : 1;
   // K ring depth: deep for decode (HBM streaming), shallower when Q is large.
-  static constexpr int kStages = QT <= 2 ? 6 : 4;
+  static constexpr int kStages = QT == 1 ? 5 : (QT == 2 ? 6 : 4);
+  static constexpr int kHistBytes = QT == 1 ? kHistBins * 4 : 0;
   static constexpr int kQBoxBytes = N * 128;
   static constexpr int kQBytes = 2 * kQBoxBytes;
   static constexpr int kTmemCols = 2 * N < 32 ? 32 : 2 * N;
-  static constexpr int kSmemData = kQBufs * kQBytes + kStages * kKTileBytes;
+  static constexpr int kSmemData = kQBufs * kQBytes + kStages * kKTileBytes + kHistBytes;
   static constexpr int kBarBytes = 8 * (2 * kStages + 8) + 16;
   static constexpr int kSmemBytes = kSmemData + kBarBytes + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, N);
@@ -91,6 +99,10 @@ __device__ __forceinline__ bool decode_item(const IdxParams& P, int item, ItemVi
   return v.kt0 < v.kt1;
 }
 
+__device__ __forceinline__ void named_bar_sync_idx(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ int snake_item(int j) {
   const int G = static_cast<int>(gridDim.x);
   const int k = static_cast<int>(blockIdx.x);
@@ -109,6 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const base_ptr = smem_raw + (base - raw);
   const uint32_t q_smem = base;
   const uint32_t k_smem = base + C::kQBufs * C::kQBytes;
+  int* const shist =
+      reinterpret_cast<int*>(base_ptr + C::kQBufs * C::kQBytes + C::kStages * kKTileBytes);
   const uint32_t bars = base + C::kSmemData;
   auto full = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (C::kStages + s); };
@@ -240,6 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127
+    const bool do_hist = (QT == 1) && P.hist != nullptr;
+    if (do_hist) {
+      for (int i = et; i < kHistBins; i += kEpiThreads) shist[i] = 0;
+      named_bar_sync_idx(1, kEpiThreads);
+    }
     int acc = 0;
     uint32_t aph = 0;
     bool ok = true;
@@ -272,12 +292,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           float s = (s0 + s1) + (s2 + s3);
           if (s == 0.f) s = 0.f;  // one zero: -0 and +0 are the same score
-          if (key <= v.pos0 + jq) P.scores[static_cast<size_t>(v.row0 + jq) * P.ld + key] = s;
+          const bool valid = key <= v.pos0 + jq;
+          if (valid) P.scores[static_cast<size_t>(v.row0 + jq) * P.ld + key] = s;
+          if (do_hist) {
+            const uint32_t bin = valid ? (score_key(s) >> kHistShift) : 0xFFFFFFFFu;
+            const unsigned grp = __match_any_sync(0xffffffffu, bin);
+            if (valid && lane == __ffs(grp) - 1) atomicAdd(&shist[bin], __popc(grp));
+          }
         }
         tc_fence_before();
         mbar_arrive(tempty(acc));
         acc ^= 1;
         if (acc == 0) aph ^= 1u;
+      }
+      if (do_hist) {  // flush this item's counts into the row's histogram
+        named_bar_sync_idx(1, kEpiThreads);
+        int* const gh = P.hist + static_cast<size_t>(v.row0) * kHistBins;
+        for (int i = et; i < kHistBins; i += kEpiThreads) {
+          const int c = shist[i];
+          if (c != 0) {
+            atomicAdd(gh + i, c);
+            shist[i] = 0;
+          }
+        }
+        named_bar_sync_idx(1, kEpiThreads);
       }
     }
   }
@@ -342,6 +380,7 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.scores = a.scores;
     P.ld = a.ld;
     P.err = a.err;
+    P.hist = QT == 1 ? a.hist : nullptr;
     int items = 0, n = 0;
     for (; b < a.B && n < kMaxSeqPerLaunch; ++b) {
       const int nq = a.h_q_offsets[b + 1] - a.h_q_offsets[b];
@@ -369,6 +408,13 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool indexer_single_query_items(const int32_t* h_q_offsets, int B) {
+  for (int b = 0; b < B; ++b) {
+    if (h_q_offsets[b + 1] - h_q_offsets[b] > 1) return false;
+  }
+  return true;
+}
 
 cudaError_t launch_indexer_score(const IndexerArgs& a, cudaStream_t stream) {
   int max_nq = 0;

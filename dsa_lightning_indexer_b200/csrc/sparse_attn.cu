@@ -10,12 +10,12 @@
 // 16-byte cp.async copies into shared memory (double-buffered tiles of 32
 // rows) and used for both Q.K^T and P.V.  A CTA owns one query row, a block of
 // heads (16 per warp group of four warps) and a contiguous slice of the
-// selected set.  With many query rows (prefill) a CTA takes 64 heads and the
-// whole set; with few rows (decode) it takes 16 heads and a slice, and the
-// last CTA to finish a (row, head block) merges the slices' partial results
-// with the log-sum-exp rule (an atomic ticket decides who is last; nobody
-// waits).  Softmax runs online in fp32 in base 2.  P enters the P.V product as
-// bf16 hi + lo parts, so its rounding error stays near 2^-16 relative.
+// selected set.  With few rows (decode) it takes 16 heads and a slice of the
+// set; a second kernel, spread over the whole GPU, merges the slices' partial
+// results with the log-sum-exp rule.  (Many-row launches use the tcgen05
+// kernel in sparse_attn_tc.cu.)  Softmax runs online in fp32 in base 2.  P
+// enters the P.V product as bf16 hi + lo parts, so its rounding error stays
+// near 2^-16 relative.
 #include <algorithm>
 
 #include "dsa_common.cuh"
@@ -39,8 +39,8 @@ struct AttnParams {
   const int32_t* idx;
   float* out;
   float* lse;
-  float* part;          // [n_split][Nq][H][512 + 2] when n_split > 1
-  int* tickets;         // [Nq][head_blocks] arrival counters, zero between calls
+  float* part_o;        // [n_split][Nq][H][512] unnormalised slice outputs
+  float2* part_ml;      // [n_split][Nq][H] (running max in log2 units, row sum)
   int B, Nq, H, top_k, n_split, split_len;
   float scale_log2;     // scale * log2(e)
 };
@@ -310,73 +310,82 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
             L_g8 > 0.f ? (m_g8 + log2f(L_g8)) * kLn2 : -INFINITY;
     }
   } else {
-    constexpr int kRec = kValue + 2;
-    float* const base = P.part + (static_cast<size_t>(sp) * P.Nq + r) * P.H * kRec;
+    const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int dv = qd * 128 + i * 8 + 2 * c;
-      if (ha < P.H) {
-        base[static_cast<size_t>(ha) * kRec + dv] = o[i][0];
-        base[static_cast<size_t>(ha) * kRec + dv + 1] = o[i][1];
-      }
-      if (hb8 < P.H) {
-        base[static_cast<size_t>(hb8) * kRec + dv] = o[i][2];
-        base[static_cast<size_t>(hb8) * kRec + dv + 1] = o[i][3];
-      }
+      if (ha < P.H)
+        *reinterpret_cast<float2*>(P.part_o + (rec + ha) * kValue + dv) =
+            make_float2(o[i][0], o[i][1]);
+      if (hb8 < P.H)
+        *reinterpret_cast<float2*>(P.part_o + (rec + hb8) * kValue + dv) =
+            make_float2(o[i][2], o[i][3]);
     }
     if (qd == 0 && c == 0) {
-      if (ha < P.H) {
-        base[static_cast<size_t>(ha) * kRec + kValue] = m_g;
-        base[static_cast<size_t>(ha) * kRec + kValue + 1] = L_g;
-      }
-      if (hb8 < P.H) {
-        base[static_cast<size_t>(hb8) * kRec + kValue] = m_g8;
-        base[static_cast<size_t>(hb8) * kRec + kValue + 1] = L_g8;
-      }
-    }
-    // The last CTA of this (row, head block) to arrive merges all slices.
-    __shared__ int is_last;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      int* const ticket = P.tickets + static_cast<size_t>(r) * gridDim.y + blockIdx.y;
-      const int t = atomicAdd(ticket, 1);
-      is_last = (t == P.n_split - 1);
-      if (is_last) *ticket = 0;  // every other slice has arrived: reset for the next call
-    }
-    __syncthreads();
-    if (is_last) {
-      __threadfence();
-      const size_t split_stride = static_cast<size_t>(P.Nq) * P.H * kRec;
-      for (int e = tid; e < HB * (kValue / 4); e += kThreads) {
-        const int hl = e / (kValue / 4), dv = (e - hl * (kValue / 4)) * 4;
-        const int h = h0 + hl;
-        if (h >= P.H) continue;
-        const float* const pr = P.part + (static_cast<size_t>(r) * P.H + h) * kRec;
-        float M = -INFINITY;
-        for (int q = 0; q < P.n_split; ++q) M = fmaxf(M, __ldcg(pr + q * split_stride + kValue));
-        float Lsum = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int q = 0; q < P.n_split; ++q) {
-          const float* const ps = pr + q * split_stride;
-          const float ms = __ldcg(ps + kValue);
-          if (ms == -INFINITY) continue;
-          const float wgt = exp2f(ms - M);
-          Lsum += wgt * __ldcg(ps + kValue + 1);
-          acc.x += wgt * __ldcg(ps + dv + 0);
-          acc.y += wgt * __ldcg(ps + dv + 1);
-          acc.z += wgt * __ldcg(ps + dv + 2);
-          acc.w += wgt * __ldcg(ps + dv + 3);
-        }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        *reinterpret_cast<float4*>(P.out + (static_cast<size_t>(r) * P.H + h) * kValue + dv) =
-            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        if (P.lse && dv == 0)
-          P.lse[static_cast<size_t>(r) * P.H + h] =
-              Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
-      }
+      if (ha < P.H) P.part_ml[rec + ha] = make_float2(m_g, L_g);
+      if (hb8 < P.H) P.part_ml[rec + hb8] = make_float2(m_g8, L_g8);
     }
   }
+}
+
+// Merges the slices of one (query row, head): O = sum_s 2^(m_s - M) O_s /
+// sum_s 2^(m_s - M) l_s.  One CTA per (row, head), one float4 of O per thread;
+// the slices' loads are independent so they overlap.
+constexpr int kMaxSplit = 64;
+__global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams P) {
+  __shared__ float wgt[kMaxSplit];
+  __shared__ float inv_total, lse_val;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x, h = blockIdx.y;
+  const size_t rec = static_cast<size_t>(r) * P.H + h;
+  const size_t stride = static_cast<size_t>(P.Nq) * P.H;
+  if (threadIdx.x < 32) {
+    float m[kMaxSplit / 32], l[kMaxSplit / 32];
+    float M = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit / 32; ++j) {
+      const int sp = threadIdx.x + 32 * j;
+      const float2 ml = sp < P.n_split ? __ldcg(P.part_ml + sp * stride + rec)
+                                       : make_float2(-INFINITY, 0.f);
+      m[j] = ml.x;
+      l[j] = ml.y;
+      M = fmaxf(M, ml.x);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit / 32; ++j) {
+      const float w = m[j] == -INFINITY ? 0.f : exp2f(m[j] - M);
+      const int sp = threadIdx.x + 32 * j;
+      if (sp < P.n_split) wgt[sp] = w;
+      L += w * l[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (threadIdx.x == 0) {
+      inv_total = L > 0.f ? 1.f / L : 0.f;
+      lse_val = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  const int dv = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* const po = P.part_o + rec * kValue + dv;
+#pragma unroll 8
+  for (int sp = 0; sp < P.n_split; ++sp) {
+    const float w = wgt[sp];
+    const float4 x = __ldcg(reinterpret_cast<const float4*>(po + sp * stride * kValue));
+    acc.x = fmaf(w, x.x, acc.x);
+    acc.y = fmaf(w, x.y, acc.y);
+    acc.z = fmaf(w, x.z, acc.z);
+    acc.w = fmaf(w, x.w, acc.w);
+  }
+  const float inv = inv_total;
+  *reinterpret_cast<float4*>(P.out + rec * kValue + dv) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (P.lse && threadIdx.x == 0) P.lse[rec] = lse_val;
 }
 
 template <int NG>
@@ -399,17 +408,23 @@ cudaError_t launch_ng(const AttnParams& P, int head_blocks, cudaStream_t stream)
 
 AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms) {
   AttnPlan p;
+  p.tc = 0;
   p.hb = std::min(kHeadsPerCta, (H + 15) / 16 * 16);
   p.head_blocks = (H + p.hb - 1) / p.hb;
   p.n_split = 1;
   const long long rows = Nq;
-  if (rows * p.head_blocks < num_sms && rows > 0) {
+  if (rows * ((H + kHeadsPerCta - 1) / kHeadsPerCta) >= num_sms) {
+    // Many rows: the tcgen05 kernel, 64 heads per CTA, whole selected set.
+    p.tc = 1;
+    p.hb = kHeadsPerCta;
+    p.head_blocks = (H + kHeadsPerCta - 1) / kHeadsPerCta;
+  } else if (rows > 0) {
     // Few rows: 16 heads per CTA (two CTAs fit an SM) and slices of the set.
     p.hb = 16;
     p.head_blocks = (H + 15) / 16;
     const long long base = rows * p.head_blocks;
     const int want = static_cast<int>(std::max<long long>(1, 2LL * num_sms / base));
-    const int n = std::min(want, (top_k + kTileRows - 1) / kTileRows);
+    const int n = std::min(std::min(want, kMaxSplit), (top_k + kTileRows - 1) / kTileRows);
     if (n > 1) {
       const int per = ((top_k + n - 1) / n + kTileRows - 1) / kTileRows * kTileRows;
       p.n_split = (top_k + per - 1) / per;
@@ -424,13 +439,9 @@ size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p) {
   return static_cast<size_t>(p.n_split) * Nq * H * (kValue + 2) * sizeof(float);
 }
 
-size_t attn_ticket_bytes(int Nq, const AttnPlan& p) {
-  if (p.n_split <= 1) return 0;
-  return static_cast<size_t>(Nq) * p.head_blocks * sizeof(int);
-}
-
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   if (a.Nq == 0) return cudaSuccess;
+  if (a.plan.tc) return launch_sparse_attn_tc(a, stream);
   AttnParams P;
   P.q_offsets = a.q_offsets;
   P.kv_offsets = a.kv_offsets;
@@ -439,8 +450,9 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   P.idx = a.idx;
   P.out = a.out;
   P.lse = a.lse;
-  P.part = a.part;
-  P.tickets = a.tickets;
+  const size_t n_rec = static_cast<size_t>(a.plan.n_split) * a.Nq * a.H;
+  P.part_o = a.part;
+  P.part_ml = reinterpret_cast<float2*>(a.part + n_rec * kValue);
   P.B = a.B;
   P.Nq = a.Nq;
   P.H = a.H;
@@ -448,12 +460,15 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   P.n_split = a.plan.n_split;
   P.split_len = a.plan.split_len;
   P.scale_log2 = a.scale * kLog2e;
+  cudaError_t e;
   switch (a.plan.hb / 16) {
-    case 1: return launch_ng<1>(P, a.plan.head_blocks, stream);
-    case 2: return launch_ng<2>(P, a.plan.head_blocks, stream);
-    case 3: return launch_ng<3>(P, a.plan.head_blocks, stream);
-    default: return launch_ng<4>(P, a.plan.head_blocks, stream);
+    case 1: e = launch_ng<1>(P, a.plan.head_blocks, stream); break;
+    case 2: e = launch_ng<2>(P, a.plan.head_blocks, stream); break;
+    case 3: e = launch_ng<3>(P, a.plan.head_blocks, stream); break;
+    default: e = launch_ng<4>(P, a.plan.head_blocks, stream); break;
   }
+  if (e != cudaSuccess || P.n_split == 1) return e;
+  return launch_pdl(attn_merge_kernel, dim3(a.Nq, a.H), dim3(128), 0, stream, 0, P);
 }
 
 }  // namespace dsa

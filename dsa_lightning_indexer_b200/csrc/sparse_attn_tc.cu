@@ -1,0 +1,483 @@
+// Attention over the selected latent rows on tcgen05 tensor cores, for
+// launches with many query rows (prefill).
+//
+//   O[q, g, :] = sum_{s in S_q} softmax_s( scale * q[q, g, :] . kv[s, :] ) * kv[s, :512]
+//
+// (llama.cpp b12180 news: aiaulis.com paragraph 2 — attention only over the
+// selected tokens; devotd.net section 2 — one key-only latent cache whose
+// leading 512 entries serve as V.)
+//
+// One CTA owns one query row and a block of 64 heads, and walks the row's
+// selected set in tiles of 48 gathered cache rows:
+//   S    = Q[64 heads, 576] . K_tile[48, 576]^T      M = 64,  N = 48, K = 576
+//   O^T += V_tile^T[512, 48] . P^T[48, 64 heads]     M = 128 (x4), N = 64, K = 48
+// S lands in TMEM with one head per lane, so each softmax thread owns one
+// head row: max, exp2 and row sum stay in registers.  P is written to shared
+// memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
+// 2^-16.  The gathered tile is stored once, in the 128-byte swizzled layout,
+// and read by both MMAs: K-major as the B operand of S, MN-major as the A
+// operand of O^T.  The running maximum is raised lazily (only when a tile's
+// maximum exceeds it by more than 2^8), and O^T in TMEM is then rescaled.
+//
+// Warp roles (288 threads): warps 0-3 softmax and output (TMEM quadrants
+// 0-3), warp 4 TMEM allocation, the Q load (TMA) and single-thread MMA issue,
+// warps 5-6 and 7-8 gather even and odd tiles with 16-byte cp.async.
+#include <algorithm>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kT = 48;                    // gathered rows per tile
+constexpr int kHB = 64;                   // heads per CTA
+constexpr int kBoxes = kLatent / 64;      // 64-dim column boxes of a latent row
+constexpr int kQBox = kHB * 128;          // bytes of one Q box
+constexpr int kKVBox = kT * 128;          // bytes of one gathered-tile box
+constexpr int kKVStage = kBoxes * kKVBox;
+constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 48 used)
+constexpr int kThreadsTc = 288;
+constexpr int kSoftThreads = 128;
+constexpr int kGroupThreads = 64;         // one gather group
+constexpr float kLog2eTc = 1.4426950408889634f;
+constexpr float kLn2Tc = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
+
+constexpr int kOffQ = 0;
+constexpr int kOffKV = kOffQ + kBoxes * kQBox;
+constexpr int kOffP = kOffKV + 2 * kKVStage;           // [stage][hi, lo]
+constexpr int kOffBar = kOffP + 4 * kPBuf;
+constexpr int kNumBars = 14;
+constexpr int kOffTmem = kOffBar + 8 * kNumBars;
+constexpr int kOffIdx = kOffTmem + 16;                  // [2][kT] int
+constexpr int kOffAlpha = kOffIdx + 2 * kT * 4;         // [64] float
+constexpr int kOffM = kOffAlpha + kHB * 4;              // [64] float
+constexpr int kOffL = kOffM + kHB * 4;                  // [64] float
+constexpr int kSmemUsed = kOffL + kHB * 4;
+constexpr int kSmemTc = kSmemUsed + 1024;               // alignment slack
+static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
+
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;     // S buffers at columns 0 and 64 (M = 64 layout)
+constexpr uint32_t kColO = 128;   // O^T blocks at 128, 192, 256, 320
+
+// kind::f16 instruction descriptors (bf16 in, fp32 accumulate).
+constexpr uint32_t kIdescS = idesc_bf16_f32(64, kT);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
+
+struct TcParams {
+  const int32_t* q_offsets;
+  const int64_t* kv_offsets;
+  const int32_t* ctx_lens;
+  const __nv_bfloat16* kv;
+  const int32_t* idx;
+  float* out;
+  float* lse;
+  unsigned* err;
+  int B, Nq, H, top_k;
+  int idx_prefix;       // valid entries are the first min(top_k, p+1) slots
+  float scale_log2;
+};
+
+// MN-major operand in the 128-byte swizzle layout: 64-element chunks along
+// M/N `lbo` bytes apart, groups of 8 K-rows 1024 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16_tc(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// OR of `pred` over the `threads` threads meeting at named barrier `id`.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(res)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
+      : "memory");
+  return res != 0;
+}
+
+__device__ __forceinline__ int owner_seq_tc(const int32_t* q_offsets, int B, int r) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (q_offsets[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const bp = smem_raw + (base - raw);
+  const uint32_t sQ = base + kOffQ, sKV = base + kOffKV, sP = base + kOffP;
+  const uint32_t bars = base + kOffBar;
+  const uint32_t b_qfull = bars;
+  auto b_kvfull = [&](int s) { return bars + 8u * (1 + s); };
+  auto b_kvempty = [&](int s) { return bars + 8u * (3 + s); };
+  auto b_sfull = [&](int s) { return bars + 8u * (5 + s); };
+  auto b_sempty = [&](int s) { return bars + 8u * (7 + s); };
+  auto b_pfull = [&](int s) { return bars + 8u * (9 + s); };
+  auto b_pempty = [&](int s) { return bars + 8u * (11 + s); };
+  const uint32_t b_odone = bars + 8u * 13;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
+  int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
+  float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
+  float* const m_s = reinterpret_cast<float*>(bp + kOffM);
+  float* const l_s = reinterpret_cast<float*>(bp + kOffL);
+
+  const int warp = warp_id_uniform();
+  const int lane = lane_id();
+  const int r = blockIdx.x;
+  const int h0 = blockIdx.y * kHB;
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qfull, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_kvfull(s), kGroupThreads);
+      mbar_init(b_kvempty(s), 1);
+      mbar_init(b_sfull(s), 1);
+      mbar_init(b_sempty(s), kSoftThreads);
+      mbar_init(b_pfull(s), kSoftThreads);
+      mbar_init(b_pempty(s), 1);
+    }
+    mbar_init(b_odone, 1);
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  pdl_wait();
+  pdl_launch_dependents();
+
+  const int b = owner_seq_tc(P.q_offsets, P.B, r);
+  const long long kv0 = P.kv_offsets[b];
+  const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
+  int n_slots = P.top_k;
+  if (P.idx_prefix) {  // slots past min(top_k, p+1) hold -1: skip their tiles
+    const int q0 = P.q_offsets[b];
+    const int pos = P.ctx_lens[b] - (P.q_offsets[b + 1] - q0) + (r - q0);
+    n_slots = min(P.top_k, pos + 1);
+  }
+  const int n_tiles = (n_slots + kT - 1) / kT;
+
+  if (warp >= 5) {
+    // ------------------------------------------------------------ gather --
+    const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
+    const int gt = threadIdx.x - (5 + 2 * grp) * 32;
+    bool ok = true;
+    for (int t = grp; t < n_tiles && ok; t += 2) {
+      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
+      if (!ok) break;
+      const uint32_t stage = sKV + grp * kKVStage;
+      for (int e = gt; e < kT * (kLatent / 8); e += kGroupThreads) {
+        const int i = e / (kLatent / 8), ch = e - i * (kLatent / 8);
+        const int slot = t * kT + i;
+        const int pos = slot < n_slots ? __ldg(idx_row + slot) : -1;
+        if (ch == 0) tidx[grp * kT + i] = pos;
+        const int box = ch >> 3, c = ch & 7;
+        const uint32_t dst = stage + box * kKVBox + i * 128 + ((c ^ (i & 7)) << 4);
+        if (pos >= 0) {
+          cp_async16_tc(dst, P.kv + static_cast<size_t>(kv0 + pos) * kLatent + ch * 8);
+        } else {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
+                       : "memory");
+        }
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      fence_proxy_async_smem();
+      mbar_arrive(b_kvfull(grp));
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------ Q load + MMA issue --
+    if (lane == 0) {
+      tma_prefetch_map(&qmap);
+      mbar_arrive_expect_tx(b_qfull, kBoxes * kQBox);
+      const uint64_t pol = l2_policy_evict_first();
+      for (int j = 0; j < kBoxes; ++j) {
+        tma_load_2d(sQ + j * kQBox, &qmap, b_qfull, 64 * j, r * P.H + h0, pol);
+      }
+      bool ok = mbar_wait(b_qfull, 0, P.err);
+      auto issue_pv = [&](int u) -> bool {
+        const int st = u & 1;
+        const uint32_t ph = static_cast<uint32_t>((u >> 1) & 1);
+        if (!mbar_wait(b_pfull(st), ph, P.err)) return false;
+        tc_fence_after();
+        const uint32_t kvs = sKV + st * kKVStage;
+        const uint32_t phi = sP + (2 * st) * kPBuf, plo = phi + kPBuf;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+          for (int kk = 0; kk < kT / 16; ++kk) {
+            const uint64_t a = sdesc_sw128_mn(kvs + (2 * blk) * kKVBox + kk * 2048, kKVBox);
+            const uint32_t d = tmem + kColO + 64u * blk;
+            tc_mma_bf16(d, a, sdesc_sw128(phi + kk * 32), kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_bf16(d, a, sdesc_sw128(plo + kk * 32), kIdescPV, 1u);
+          }
+        }
+        tc_commit(b_kvempty(st));
+        tc_commit(b_pempty(st));
+        tc_commit(b_odone);
+        return true;
+      };
+      for (int t = 0; t < n_tiles && ok; ++t) {
+        const int st = t & 1;
+        const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+        ok = mbar_wait(b_kvfull(st), ph, P.err) && mbar_wait(b_sempty(st), ph ^ 1u, P.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kvs = sKV + st * kKVStage;
+        const uint32_t d = tmem + kColS + 64u * st;
+#pragma unroll 4
+        for (int ks = 0; ks < kLatent / 16; ++ks) {
+          const uint32_t off = (ks & 3) * 32;
+          tc_mma_bf16(d, sdesc_sw128(sQ + (ks >> 2) * kQBox + off),
+                      sdesc_sw128(kvs + (ks >> 2) * kKVBox + off), kIdescS, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(b_sfull(st));
+        if (t > 0) ok = issue_pv(t - 1);
+      }
+      if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+    }
+  } else {
+    // ----------------------------------------------------------- softmax --
+    const int q = warp;                          // TMEM lane quadrant
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const bool owner = lane < 16;                // owns head row 16q + lane
+    const int hl = 16 * q + (lane & 15);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int st = t & 1;
+      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      ok = mbar_wait(b_sfull(st), ph, P.err);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t va[32], vb[16];
+      tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64u * st, va);
+      tmem_ld_32x32b_x16(tmem + lane_base + kColS + 64u * st + 32u, vb);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(b_sempty(st));
+      // The tile's slot list was written by its gather group before kv_full.
+      ok = mbar_wait(b_kvfull(st), ph, P.err);
+      if (!ok) break;
+      // Logits in base 2; unused slots masked.
+      float s[kT];
+      const int* const ti = tidx + st * kT;
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kT; ++k) {
+        const float raw_s = __uint_as_float(k < 32 ? va[k] : vb[k - 32]);
+        s[k] = ti[k] >= 0 ? raw_s * P.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[k]);
+      }
+      const bool raise = tmax > m_run + kRescaleLog2 || (m_run == -INFINITY && tmax > -INFINITY);
+      const float m_new = raise ? tmax : m_run;
+      const float alpha = raise ? exp2f(m_run - m_new) : 1.f;
+      float sum = 0.f;
+      uint32_t hi[kT / 2], lo[kT / 2];
+#pragma unroll
+      for (int k = 0; k < kT; k += 2) {
+        const float p0 = s[k] == -INFINITY ? 0.f : exp2f(s[k] - m_new);
+        const float p1 = s[k + 1] == -INFINITY ? 0.f : exp2f(s[k + 1] - m_new);
+        sum += p0 + p1;
+        const uint32_t h2 = pack2_bf16(p0, p1);
+        const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&h2);
+        hi[k / 2] = h2;
+        lo[k / 2] = pack2_bf16(p0 - __low2float(hb), p1 - __high2float(hb));
+      }
+      if (owner) {
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        alpha_s[hl] = alpha;
+      }
+      // P buffer `st` is free once the P.V of tile t-2 has completed.
+      ok = mbar_wait(b_pempty(st), ph ^ 1u, P.err);
+      if (!ok) break;
+      if (owner) {
+        const uint32_t prow_hi = sP + (2 * st) * kPBuf + hl * 128;
+        const uint32_t prow_lo = prow_hi + kPBuf;
+#pragma unroll
+        for (int c = 0; c < kT / 8; ++c) {
+          const uint32_t off = static_cast<uint32_t>((c ^ (hl & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_hi + off),
+                       "r"(hi[4 * c]), "r"(hi[4 * c + 1]), "r"(hi[4 * c + 2]), "r"(hi[4 * c + 3])
+                       : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_lo + off),
+                       "r"(lo[4 * c]), "r"(lo[4 * c + 1]), "r"(lo[4 * c + 2]), "r"(lo[4 * c + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      // If any head raised its running max, scale O^T (after the previous P.V).
+      const bool any = named_bar_or(1, kSoftThreads, owner && raise && t > 0);
+      if (any) {
+        ok = mbar_wait(b_odone, static_cast<uint32_t>((t - 1) & 1), P.err);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_base + kColO + 64u * blk + 32u * half;
+            tmem_ld_32x32b_x32(ta, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha_s[32 * half + j]);
+            }
+            tmem_st_32x32b_x32(ta, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      mbar_arrive(b_pfull(st));
+    }
+    // ------------------------------------------------------------ output --
+    if (owner) {
+      m_s[hl] = m_run;
+      l_s[hl] = l_run;
+    }
+    named_bar_sync(1, kSoftThreads);
+    if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
+    tc_fence_after();
+    if (ok) {
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        const int dv = 128 * blk + 32 * q + lane;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int hh = 32 * half + j;
+            const int h = h0 + hh;
+            if (h < P.H) {
+              const float L = l_s[hh];
+              P.out[(static_cast<size_t>(r) * P.H + h) * kValue + dv] =
+                  L > 0.f ? __uint_as_float(o[j]) / L : 0.f;
+            }
+          }
+        }
+      }
+      if (P.lse && owner && h0 + hl < P.H) {
+        P.lse[static_cast<size_t>(r) * P.H + h0 + hl] =
+            l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+  if (a.Nq == 0) return cudaSuccess;
+  EncodeTiledFn fn = get_encode_tiled();
+  if (!fn) return cudaErrorInvalidValue;
+  CUtensorMap qmap;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLatent),
+                              static_cast<cuuint64_t>(a.Nq) * a.H};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLatent) * 2};
+  const cuuint32_t box[2] = {64, kHB};
+  const cuuint32_t estr[2] = {1, 1};
+  if (fn(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides,
+         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e = ensure_smem_limit<sparse_attn_tc_kernel>(kSmemTc);
+  if (e != cudaSuccess) return e;
+  TcParams P;
+  P.q_offsets = a.q_offsets;
+  P.kv_offsets = a.kv_offsets;
+  P.ctx_lens = a.ctx_lens;
+  P.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
+  P.idx = a.idx;
+  P.out = a.out;
+  P.lse = a.lse;
+  P.err = a.err;
+  P.idx_prefix = a.idx_prefix ? 1 : 0;
+  P.B = a.B;
+  P.Nq = a.Nq;
+  P.H = a.H;
+  P.top_k = a.top_k;
+  P.scale_log2 = a.scale * kLog2eTc;
+  const int head_blocks = (a.H + kHB - 1) / kHB;
+  return launch_pdl(sparse_attn_tc_kernel, dim3(a.Nq, head_blocks), dim3(kThreadsTc),
+                    static_cast<size_t>(kSmemTc), stream, 0, qmap, P);
+}
+
+}  // namespace dsa

@@ -21,6 +21,8 @@
 // than 8 slices use the single-CTA kernel that re-reads the row each pass.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -59,136 +61,6 @@ __device__ __forceinline__ int owner_seq(const int32_t* q_offsets, int B, int r)
   return lo;
 }
 
-// Exclusive prefix sum over the block in thread order; also returns the total.
-__device__ __forceinline__ int block_excl_sum(int v, int* buf /*[kWarps + 1]*/, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) buf[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int wv = buf[lane];
-    int wi = wv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += t;
-    }
-    buf[lane] = wi - wv;
-    if (lane == 31) buf[kWarps] = wi;
-  }
-  __syncthreads();
-  const int res = buf[warp] + incl - v;
-  total = buf[kWarps];
-  __syncthreads();
-  return res;
-}
-
-__device__ __forceinline__ int block_excl_count(bool flag, int* buf, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned m = __ballot_sync(0xffffffffu, flag);
-  if (lane == 0) buf[warp] = __popc(m);
-  __syncthreads();
-  if (warp == 0) {
-    const int wv = buf[lane];
-    int wi = wv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += t;
-    }
-    buf[lane] = wi - wv;
-    if (lane == 31) buf[kWarps] = wi;
-  }
-  __syncthreads();
-  const int res = buf[warp] + __popc(m & ((1u << lane) - 1u));
-  total = buf[kWarps];
-  __syncthreads();
-  return res;
-}
-
-__global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const TopkParams P) {
-  __shared__ int hist[2048];
-  __shared__ int buf[kWarps + 1];
-  __shared__ int pick_digit, pick_above;
-
-  pdl_wait();
-  pdl_launch_dependents();
-  const int r = blockIdx.x;
-  const int b = owner_seq(P.q_offsets, P.B, r);
-  const int q0 = P.q_offsets[b];
-  const int nq = P.q_offsets[b + 1] - q0;
-  const int pos = P.ctx_lens[b] - nq + (r - q0);
-  const int n = pos + 1;
-  const int k = P.top_k;
-  int32_t* const out = P.idx + static_cast<size_t>(r) * k;
-  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
-
-  if (n <= k) {  // every causal position is kept
-    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
-    return;
-  }
-
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = k;  // keys still to take at or below the current prefix
-#pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
-    for (int i = threadIdx.x; i < 2048; i += kThreads) hist[i] = 0;
-    __syncthreads();
-    for (int s = threadIdx.x; s < n; s += kThreads) {
-      const uint32_t key = score_key(sc[s]);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
-    }
-    __syncthreads();
-    // Thread t looks at digit pair u = 1023 - t, so the exclusive prefix in
-    // thread order counts the keys in higher digits.
-    const int u = kThreads - 1 - static_cast<int>(threadIdx.x);
-    const int c_hi = hist[2 * u + 1], c_lo = hist[2 * u];
-    int total;
-    const int above = block_excl_sum(c_hi + c_lo, buf, total);
-    if (above < remaining && remaining <= above + c_hi + c_lo) {
-      if (above + c_hi >= remaining) {
-        pick_digit = 2 * u + 1;
-        pick_above = above;
-      } else {
-        pick_digit = 2 * u;
-        pick_above = above + c_hi;
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(pick_digit) << shift;
-    pmask |= dmask << shift;
-    remaining -= pick_above;
-    __syncthreads();
-  }
-
-  const uint32_t theta = prefix;
-  const int need = remaining;  // keys equal to theta to keep, lowest positions first
-  int taken_eq = 0, out_pos = 0;
-#pragma unroll 1
-  for (int base = 0; base < n && out_pos < k; base += kThreads) {
-    const int s = base + static_cast<int>(threadIdx.x);
-    const bool valid = s < n;
-    const uint32_t key = valid ? score_key(sc[s]) : 0u;
-    const bool gt = valid && key > theta;
-    const bool eq = valid && key == theta;
-    int eq_total, sel_total;
-    const int eq_rank = taken_eq + block_excl_count(eq, buf, eq_total);
-    const bool sel = gt || (eq && eq_rank < need);
-    const int slot = out_pos + block_excl_count(sel, buf, sel_total);
-    if (sel) out[slot] = s;
-    taken_eq += eq_total;
-    out_pos += sel_total;
-  }
-}
-
-
 // Exclusive prefix sum over a block of NW warps, in thread order.
 template <int NW>
 __device__ __forceinline__ int block_excl_sum_nw(int v, int* buf /*[NW + 1]*/, int& total) {
@@ -217,6 +89,108 @@ __device__ __forceinline__ int block_excl_sum_nw(int v, int* buf /*[NW + 1]*/, i
   total = buf[NW];
   __syncthreads();
   return res;
+}
+
+
+// Exclusive count of `flag` over a block of NW warps, in thread order.
+template <int NW>
+__device__ __forceinline__ int block_excl_count_nw(bool flag, int* buf /*[NW + 1]*/, int& total) {
+  const int lane = threadIdx.x & 31;
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  const int res = block_excl_sum_nw<NW>(lane == 0 ? __popc(m) : 0, buf, total);
+  // res counts whole warps before this one (lane 0 carried each warp's count)
+  const int before_warp = __shfl_sync(0xffffffffu, res, 0);
+  return before_warp + __popc(m & ((1u << lane) - 1u));
+}
+
+// Exact top-k of one row read from global memory, by a block of NW warps:
+// three MSB radix passes (11 + 11 + 10 bits) re-reading the row, then an
+// ordered emission of keys > theta and the first ties at theta.
+template <int NW>
+__device__ void row_select_global(const float* sc, int n, int k, int32_t* out, int* hist,
+                                  int* buf) {
+  constexpr int NT = NW * 32;
+  __shared__ int pick_digit_g, pick_above_g;
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+    for (int i = threadIdx.x; i < 2048; i += NT) hist[i] = 0;
+    __syncthreads();
+    for (int s = threadIdx.x; s < n; s += NT) {
+      const uint32_t key = score_key(sc[s]);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
+    }
+    __syncthreads();
+    // Thread t looks at the digits of group u = NT-1-t (2048/NT digits each),
+    // so the exclusive prefix in thread order counts keys in higher digits.
+    constexpr int D = 2048 / NT;
+    const int u = NT - 1 - static_cast<int>(threadIdx.x);
+    int cnt[D];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < D; ++j) {
+      cnt[j] = hist[D * u + j];
+      tot += cnt[j];
+    }
+    int total;
+    int above = block_excl_sum_nw<NW>(tot, buf, total);
+    if (above < remaining && remaining <= above + tot) {
+#pragma unroll
+      for (int j = D - 1; j >= 0; --j) {
+        if (above + cnt[j] >= remaining) {
+          pick_digit_g = D * u + j;
+          pick_above_g = above;
+          break;
+        }
+        above += cnt[j];
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(pick_digit_g) << shift;
+    pmask |= dmask << shift;
+    remaining -= pick_above_g;
+    __syncthreads();
+  }
+  const uint32_t theta = prefix;
+  const int need = remaining;
+  int taken_eq = 0, out_pos = 0;
+#pragma unroll 1
+  for (int base = 0; base < n && out_pos < k; base += NT) {
+    const int s = base + static_cast<int>(threadIdx.x);
+    const bool valid = s < n;
+    const uint32_t key = valid ? score_key(sc[s]) : 0u;
+    const bool gt = valid && key > theta;
+    const bool eq = valid && key == theta;
+    int eq_total, sel_total;
+    const int eq_rank = taken_eq + block_excl_count_nw<NW>(eq, buf, eq_total);
+    const bool sel = gt || (eq && eq_rank < need);
+    const int slot = out_pos + block_excl_count_nw<NW>(sel, buf, sel_total);
+    if (sel) out[slot] = s;
+    taken_eq += eq_total;
+    out_pos += sel_total;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const TopkParams P) {
+  __shared__ int hist[2048];
+  __shared__ int buf[kWarps + 1];
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const int b = owner_seq(P.q_offsets, P.B, r);
+  const int q0 = P.q_offsets[b];
+  const int nq = P.q_offsets[b + 1] - q0;
+  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;
+  const int k = P.top_k;
+  int32_t* const out = P.idx + static_cast<size_t>(r) * k;
+  if (n <= k) {  // every causal position is kept
+    for (int i = threadIdx.x; i < k; i += kThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+  row_select_global<kWarps>(P.scores + static_cast<size_t>(r) * P.ld, n, k, out, hist, buf);
 }
 
 __global__ void __launch_bounds__(kCThreads) topk_cluster_kernel(const TopkParams P) {
@@ -363,7 +337,290 @@ __global__ void __launch_bounds__(kCThreads) topk_cluster_kernel(const TopkParam
   }
 }
 
+
+// ------------------------------------------------- histogram-driven path --
+// For few long rows whose indexer launch built the score-key histograms.
+constexpr int kHThreads = 512;
+constexpr int kHWarps = kHThreads / 32;
+constexpr int kCandMax = 8192;   // keys of the threshold bin kept for the exact pass
+constexpr int kSortMax = 2048;   // >= top_k, power of two
+
+struct HistParams {
+  const int32_t* q_offsets;
+  const int32_t* ctx_lens;
+  const float* scores;
+  long long ld;
+  int32_t* idx;
+  int B, top_k, chunk, chunks;
+  int* hist;            // [Nq][kHistBins], zero again on exit
+  int* gt_list;         // [Nq][top_k]
+  uint32_t* cand_key;   // [Nq][kCandMax]
+  int* cand_pos;        // [Nq][kCandMax]
+  int* counters;        // [Nq][4]: above count, candidate count, arrival ticket; zero on exit
+};
+
+// Finds, among `n` shared-memory keys, the `want`-th largest key theta and how
+// many keys equal to theta are needed.  Every key has the bits `known_mask`
+// equal to `known`; radix passes cover the bits in [lo_bit, hi_bit].
+__device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, int hi_bit,
+                            uint32_t known, uint32_t known_mask, int* hist /*[2048]*/, int* buf,
+                            uint32_t& theta, int& need) {
+  __shared__ int pd, pa;
+  uint32_t prefix = known, pmask = known_mask;
+  int remaining = want;
+  for (int top = hi_bit; top >= lo_bit;) {
+    const int nbits = min(11, top - lo_bit + 1);
+    const int shift = top - nbits + 1;
+    const uint32_t dmask = (1u << nbits) - 1u;
+    for (int i = threadIdx.x; i < 2048; i += kHThreads) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kHThreads) {
+      const uint32_t key = keys[i];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
+    }
+    __syncthreads();
+    const int u = kHThreads - 1 - static_cast<int>(threadIdx.x);
+    const int c0 = hist[4 * u], c1 = hist[4 * u + 1], c2 = hist[4 * u + 2], c3 = hist[4 * u + 3];
+    const int tot = c0 + c1 + c2 + c3;
+    int total;
+    const int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
+    if (above < remaining && remaining <= above + tot) {
+      if (above + c3 >= remaining) {
+        pd = 4 * u + 3; pa = above;
+      } else if (above + c3 + c2 >= remaining) {
+        pd = 4 * u + 2; pa = above + c3;
+      } else if (above + c3 + c2 + c1 >= remaining) {
+        pd = 4 * u + 1; pa = above + c3 + c2;
+      } else {
+        pd = 4 * u; pa = above + c3 + c2 + c1;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(pd) << shift;
+    pmask |= dmask << shift;
+    remaining -= pa;
+    __syncthreads();
+    top = shift - 1;
+  }
+  theta = prefix;
+  need = remaining;
+}
+
+__global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P) {
+  extern __shared__ __align__(16) uint8_t hsm[];
+  uint32_t* const ck = reinterpret_cast<uint32_t*>(hsm);           // [kCandMax] keys
+  int* const cp = reinterpret_cast<int*>(ck + kCandMax);            // [kCandMax] positions
+  uint32_t* const tk = reinterpret_cast<uint32_t*>(cp + kCandMax);  // [kCandMax] tie keys
+  int* const fin = reinterpret_cast<int*>(tk + kCandMax);           // [kSortMax] result
+  int* const hist = fin + kSortMax;                                 // [2048]
+  __shared__ int buf[kHWarps + 1];
+  __shared__ int s_bin, s_above, s_inbin, s_last, s_nfin;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int r = blockIdx.x / P.chunks, c = blockIdx.x % P.chunks;
+  const int b = owner_seq(P.q_offsets, P.B, r);
+  const int q0 = P.q_offsets[b];
+  const int n = P.ctx_lens[b] - (P.q_offsets[b + 1] - q0) + (r - q0) + 1;
+  const int k = P.top_k;
+  int* const gh = P.hist + static_cast<size_t>(r) * kHistBins;
+  int* const cnt = P.counters + static_cast<size_t>(r) * 4;
+  int32_t* const out = P.idx + static_cast<size_t>(r) * k;
+  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
+
+  if (n <= k) {  // every causal position is kept; clear the row's histogram
+    if (c == 0) {
+      for (int i = tid; i < k; i += kHThreads) out[i] = i < n ? i : -1;
+      for (int i = tid; i < kHistBins; i += kHThreads) gh[i] = 0;
+    }
+    return;
+  }
+
+  // 1. The bin that holds the k-th largest key: thread t reads bins
+  //    8u .. 8u+7, u = 511 - t, so the prefix in thread order counts higher bins.
+  {
+    const int u = kHThreads - 1 - tid;
+    int cb[8];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cb[j] = __ldcg(gh + 8 * u + j);
+      tot += cb[j];
+    }
+    int total;
+    int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
+    if (above < k && k <= above + tot) {
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        if (above + cb[j] >= k) {
+          s_bin = 8 * u + j;
+          s_above = above;
+          s_inbin = cb[j];
+          break;
+        }
+        above += cb[j];
+      }
+    }
+    __syncthreads();
+  }
+  const uint32_t bstar = static_cast<uint32_t>(s_bin);
+  const int c_above = s_above, c_in = s_inbin;
+
+  // 2. One pass over this CTA's chunk: keys above the bin are selected,
+  //    keys in the bin become candidates.
+  if (c_in <= kCandMax) {
+    const int s0 = c * P.chunk, s1 = min(n, s0 + P.chunk);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = s0; base < s1; base += kHThreads) {
+      const int s = base + tid;
+      const bool in = s < s1;
+      const uint32_t key = in ? score_key(sc[s]) : 0u;
+      const uint32_t bin = key >> kHistShift;
+      const bool gt = in && bin > bstar;
+      const bool eq = in && bin == bstar;
+      const unsigned mg = __ballot_sync(0xffffffffu, gt);
+      const unsigned me = __ballot_sync(0xffffffffu, eq);
+      if (mg) {
+        int at = 0;
+        if (lane == 0) at = atomicAdd(&cnt[0], __popc(mg));
+        at = __shfl_sync(0xffffffffu, at, 0);
+        if (gt) P.gt_list[static_cast<size_t>(r) * k + at + __popc(mg & lt)] = s;
+      }
+      if (me) {
+        int at = 0;
+        if (lane == 0) at = atomicAdd(&cnt[1], __popc(me));
+        at = __shfl_sync(0xffffffffu, at, 0);
+        if (eq) {
+          const size_t slot = static_cast<size_t>(r) * kCandMax + at + __popc(me & lt);
+          P.cand_key[slot] = key;
+          P.cand_pos[slot] = s;
+        }
+      }
+    }
+  }
+
+  // 3. The last CTA of the row to arrive finishes it (nobody waits).
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&cnt[2], 1) == P.chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  if (c_in > kCandMax) {
+    // Too many keys share the threshold bin (heavily tied scores): exact
+    // selection over the whole row instead.
+    row_select_global<kHWarps>(sc, n, k, out, hist, buf);
+  } else {
+    const int need = k - c_above;  // candidates to keep, 1 <= need <= c_in
+    for (int i = tid; i < c_in; i += kHThreads) {
+      ck[i] = __ldcg(P.cand_key + static_cast<size_t>(r) * kCandMax + i);
+      cp[i] = __ldcg(P.cand_pos + static_cast<size_t>(r) * kCandMax + i);
+    }
+    for (int i = tid; i < c_above; i += kHThreads) {
+      fin[i] = __ldcg(P.gt_list + static_cast<size_t>(r) * k + i);
+    }
+    if (tid == 0) s_nfin = c_above;
+    __syncthreads();
+    // Exact threshold among the candidates (their top 12 bits are bstar).
+    uint32_t theta;
+    int need_eq;
+    smem_select(ck, c_in, need, 0, kHistShift - 1, bstar << kHistShift,
+                ~((1u << kHistShift) - 1u), hist, buf, theta, need_eq);
+    // Ties at theta: keep the need_eq lowest positions (largest ~position).
+    int n_tie = 0;
+    for (int i = tid; i < c_in; i += kHThreads) n_tie += ck[i] == theta;
+    int total_tie;
+    block_excl_sum_nw<kHWarps>(n_tie, buf, total_tie);
+    const bool cut_ties = need_eq < total_tie;
+    uint32_t pos_cut = 0u;
+    if (cut_ties) {
+      for (int i = tid; i < c_in; i += kHThreads) {
+        tk[i] = ck[i] == theta ? ~static_cast<uint32_t>(cp[i]) : 0u;  // 0: not a tie
+      }
+      __syncthreads();
+      int unique;
+      smem_select(tk, c_in, need_eq, 0, 31, 0u, 0u, hist, buf, pos_cut, unique);
+    }
+    // Append kept candidates to the result list.
+    for (int i = tid; i < c_in; i += kHThreads) {
+      const uint32_t key = ck[i];
+      const bool keep =
+          key > theta || (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
+      if (keep) fin[atomicAdd(&s_nfin, 1)] = cp[i];
+    }
+    __syncthreads();
+    // Ascending positions: bitonic sort of the k kept positions.
+    for (int i = k + tid; i < kSortMax; i += kHThreads) fin[i] = 0x7FFFFFFF;
+    __syncthreads();
+    for (int size = 2; size <= kSortMax; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int i = tid; i < kSortMax; i += kHThreads) {
+          const int j = i ^ stride;
+          if (j > i) {
+            const int a = fin[i], bb = fin[j];
+            const bool up = (i & size) == 0;
+            if ((a > bb) == up) {
+              fin[i] = bb;
+              fin[j] = a;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = tid; i < k; i += kHThreads) out[i] = fin[i];
+  }
+  // Leave the row's histogram and counters zero for the next call.
+  for (int i = tid; i < kHistBins; i += kHThreads) gh[i] = 0;
+  if (tid == 0) {
+    cnt[0] = 0;
+    cnt[1] = 0;
+    cnt[2] = 0;
+  }
+}
+
 }  // namespace
+
+size_t topk_hist_ws_bytes(int Nq, int top_k) {
+  return static_cast<size_t>(Nq) *
+         (kHistBins * sizeof(int) + top_k * sizeof(int) +
+          kCandMax * (sizeof(uint32_t) + sizeof(int)) + 4 * sizeof(int));
+}
+
+cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream) {
+  if (a.Nq == 0) return cudaSuccess;
+  HistParams P;
+  P.q_offsets = a.q_offsets;
+  P.ctx_lens = a.ctx_lens;
+  P.scores = a.scores;
+  P.ld = a.ld;
+  P.idx = a.idx;
+  P.B = a.B;
+  P.top_k = a.top_k;
+  uint8_t* p = static_cast<uint8_t*>(ws_region);
+  P.hist = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * kHistBins * sizeof(int);
+  P.cand_key = reinterpret_cast<uint32_t*>(p);
+  p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(uint32_t);
+  P.cand_pos = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(int);
+  P.gt_list = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * a.top_k * sizeof(int);
+  P.counters = reinterpret_cast<int*>(p);
+  // About two CTAs per SM in total, chunks of whole 512-key blocks.
+  const long long target = 2LL * a.num_sms;
+  P.chunks = static_cast<int>(std::max<long long>(1, target / std::max(1, a.Nq)));
+  P.chunk = static_cast<int>(((a.max_len + P.chunks - 1) / P.chunks + kHThreads - 1) /
+                             kHThreads * kHThreads);
+  P.chunks = static_cast<int>((a.max_len + P.chunk - 1) / P.chunk);
+  const size_t smem = static_cast<size_t>(kCandMax) * 12 + (kSortMax + 2048) * sizeof(int);
+  cudaError_t e = ensure_smem_limit<topk_hist_kernel>(static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_hist_kernel, dim3(static_cast<unsigned>(a.Nq) * P.chunks),
+                    dim3(kHThreads), smem, stream, 0, P);
+}
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   if (a.Nq == 0) return cudaSuccess;

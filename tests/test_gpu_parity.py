@@ -254,9 +254,40 @@ def test_layer_prefill_16k_sampled_rows():
     _layer_check(wl, rows=rows)
 
 
+def _hist_batch():
+    """Decode rows long enough for the histogram-driven selection, with special rows:
+    0 normal, 1 shorter than top_k, 2 small-integer inputs (exact ties at the
+    threshold), 3 all-zero indexer queries (every score ties: the threshold bin
+    overflows the candidate buffer), 4 normal and long."""
+    wl = synth.custom([9000, 1500, 20000, 12000, 40000], [1] * 5, 16, 2048, seed=140)
+    g = np.random.Generator(np.random.PCG64(141))
+    k0 = int(wl.kv_offsets[2])
+    wl.q_idx[2] = synth.bf16_bits(g.integers(-1, 2, size=(32, 128)).astype(np.float32))
+    wl.k_idx[k0:k0 + 20000] = synth.bf16_bits(
+        g.integers(-1, 2, size=(20000, 128)).astype(np.float32))
+    wl.w[2] = g.integers(-2, 3, size=32).astype(np.float32)
+    wl.q_idx[3] = 0
+    return wl
+
+
+def test_layer_histogram_selection_special_rows():
+    wl = _hist_batch()
+    got_out, got_lse, got_idx = gpu_layer(wl)
+    ld = _up4(wl.ctx_lens.max())
+    ref_scores, ref_idx, _, _ = oracle.dsa_layer(*_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q,
+                                                 wl.kv, wl.top_k, wl.scale, ld=ld)
+    # rows 1-3 have exactly representable scores: the selection must be identical
+    for r in (1, 2, 3):
+        assert np.array_equal(got_idx[r], ref_idx[r]), r
+    assert np.array_equal(got_idx[3], np.arange(2048))  # all ties: lowest positions
+    parity.check_selection(got_idx, ref_idx, ref_scores, wl)
+    att_out, att_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, got_idx, wl.scale)
+    parity.check_attention(got_out, got_lse, att_out, att_lse)
+
+
 def test_repeated_calls_on_one_workspace_agree():
-    """Arrival tickets and other workspace state are left ready for the next call."""
-    wl = synth.custom([3000, 2500], [1, 1], 64, 2048, seed=130)
+    """Histograms, counters and other workspace state are left ready for the next call."""
+    wl = _hist_batch()
     dw = bd.DeviceWorkload(wl)
     first = [t.cpu().numpy() for t in dw.forward()]
     for _ in range(3):
