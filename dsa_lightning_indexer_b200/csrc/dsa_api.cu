@@ -317,7 +317,13 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
 
   IndexerArgs ia = indexer_args(batch, info, q_idx, w, k_idx, scores, L.ld, ws, sms);
   void* const hist_region = static_cast<uint8_t*>(ws) + L.hist_off;
-  if (L.hist_topk) ia.hist = static_cast<int*>(hist_region);
+  if (L.hist_topk) {
+    // The histograms and counters start from zero on every call: no state is
+    // carried in the workspace from one call to the next.
+    DSA_TRY(cuda_status(
+        cudaMemsetAsync(hist_region, 0, topk_hist_zero_bytes(batch->Nq), st)));
+    ia.hist = static_cast<int*>(hist_region);
+  }
   DSA_TRY(cuda_status(launch_indexer_score(ia, st)));
 
   TopkArgs t;

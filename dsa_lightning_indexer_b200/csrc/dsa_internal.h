@@ -46,8 +46,10 @@ struct TopkArgs {
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 // Selection driven by the histograms the indexer built (see IndexerArgs.hist):
-// `ws_region` holds them followed by the per-row candidate lists and
-// counters, topk_hist_ws_bytes() bytes in all, zero between calls.
+// `ws_region` holds them, the per-row counters and the candidate lists,
+// topk_hist_ws_bytes() bytes in all; its first topk_hist_zero_bytes() bytes
+// (histograms and counters) must be zero when the indexer starts.
+size_t topk_hist_zero_bytes(int Nq);
 size_t topk_hist_ws_bytes(int Nq, int top_k);
 cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream);
 

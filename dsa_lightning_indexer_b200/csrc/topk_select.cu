@@ -344,6 +344,7 @@ constexpr int kHThreads = 512;
 constexpr int kHWarps = kHThreads / 32;
 constexpr int kCandMax = 8192;   // keys of the threshold bin kept for the exact pass
 constexpr int kSortMax = 2048;   // >= top_k, power of two
+constexpr int kBitmapMax = kCandMax * 32;  // rows up to this length order by bitmap
 
 struct HistParams {
   const int32_t* q_offsets;
@@ -352,11 +353,11 @@ struct HistParams {
   long long ld;
   int32_t* idx;
   int B, top_k, chunk, chunks;
-  int* hist;            // [Nq][kHistBins], zero again on exit
-  int* gt_list;         // [Nq][top_k]
+  int* hist;            // [Nq][kHistBins], zeroed before the indexer runs
+  int* counters;        // [Nq][4]: above count, candidate count, arrival ticket; zeroed too
   uint32_t* cand_key;   // [Nq][kCandMax]
   int* cand_pos;        // [Nq][kCandMax]
-  int* counters;        // [Nq][4]: above count, candidate count, arrival ticket; zero on exit
+  int* gt_list;         // [Nq][top_k]
 };
 
 // Finds, among `n` shared-memory keys, the `want`-th largest key theta and how
@@ -429,10 +430,9 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
   int32_t* const out = P.idx + static_cast<size_t>(r) * k;
   const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
 
-  if (n <= k) {  // every causal position is kept; clear the row's histogram
+  if (n <= k) {  // every causal position is kept
     if (c == 0) {
       for (int i = tid; i < k; i += kHThreads) out[i] = i < n ? i : -1;
-      for (int i = tid; i < kHistBins; i += kHThreads) gh[i] = 0;
     }
     return;
   }
@@ -467,8 +467,17 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
   const uint32_t bstar = static_cast<uint32_t>(s_bin);
   const int c_above = s_above, c_in = s_inbin;
 
-  // 2. One pass over this CTA's chunk: keys above the bin are selected,
-  //    keys in the bin become candidates.
+  // 2. One pass over this CTA's chunk: keys above the bin are selected, keys
+  //    in the bin become candidates.  Hits are staged in shared memory (the
+  //    finalize arrays, unused until then) and published with one global
+  //    reservation per list.
+  __shared__ int s_ngt, s_nc, s_gbase, s_cbase;
+  if (tid == 0) {
+    s_ngt = 0;
+    s_nc = 0;
+  }
+  __syncthreads();
+  int* const st_gt = reinterpret_cast<int*>(tk);
   if (c_in <= kCandMax) {
     const int s0 = c * P.chunk, s1 = min(n, s0 + P.chunk);
     const unsigned lt = (1u << lane) - 1u;
@@ -483,19 +492,35 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
       const unsigned me = __ballot_sync(0xffffffffu, eq);
       if (mg) {
         int at = 0;
-        if (lane == 0) at = atomicAdd(&cnt[0], __popc(mg));
-        at = __shfl_sync(0xffffffffu, at, 0);
-        if (gt) P.gt_list[static_cast<size_t>(r) * k + at + __popc(mg & lt)] = s;
+        if (lane == 0) at = atomicAdd(&s_ngt, __popc(mg));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(mg & lt);
+        if (gt) st_gt[at] = s;
       }
       if (me) {
         int at = 0;
-        if (lane == 0) at = atomicAdd(&cnt[1], __popc(me));
-        at = __shfl_sync(0xffffffffu, at, 0);
+        if (lane == 0) at = atomicAdd(&s_nc, __popc(me));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(me & lt);
         if (eq) {
-          const size_t slot = static_cast<size_t>(r) * kCandMax + at + __popc(me & lt);
-          P.cand_key[slot] = key;
-          P.cand_pos[slot] = s;
+          ck[at] = key;
+          cp[at] = s;
         }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      s_gbase = atomicAdd(&cnt[0], s_ngt);
+      s_cbase = atomicAdd(&cnt[1], s_nc);
+    }
+    __syncthreads();
+    for (int i = tid; i < s_ngt; i += kHThreads) {
+      const int slot = s_gbase + i;
+      if (slot < k) P.gt_list[static_cast<size_t>(r) * k + slot] = st_gt[i];
+    }
+    for (int i = tid; i < s_nc; i += kHThreads) {
+      const int slot = s_cbase + i;
+      if (slot < kCandMax) {
+        P.cand_key[static_cast<size_t>(r) * kCandMax + slot] = ck[i];
+        P.cand_pos[static_cast<size_t>(r) * kCandMax + slot] = cp[i];
       }
     }
   }
@@ -518,7 +543,7 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
       ck[i] = __ldcg(P.cand_key + static_cast<size_t>(r) * kCandMax + i);
       cp[i] = __ldcg(P.cand_pos + static_cast<size_t>(r) * kCandMax + i);
     }
-    for (int i = tid; i < c_above; i += kHThreads) {
+    for (int i = tid; i < c_above && i < k; i += kHThreads) {
       fin[i] = __ldcg(P.gt_list + static_cast<size_t>(r) * k + i);
     }
     if (tid == 0) s_nfin = c_above;
@@ -543,50 +568,90 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
       int unique;
       smem_select(tk, c_in, need_eq, 0, 31, 0u, 0u, hist, buf, pos_cut, unique);
     }
-    // Append kept candidates to the result list.
-    for (int i = tid; i < c_in; i += kHThreads) {
-      const uint32_t key = ck[i];
-      const bool keep =
-          key > theta || (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
-      if (keep) fin[atomicAdd(&s_nfin, 1)] = cp[i];
-    }
-    __syncthreads();
-    // Ascending positions: bitonic sort of the k kept positions.
-    for (int i = k + tid; i < kSortMax; i += kHThreads) fin[i] = 0x7FFFFFFF;
-    __syncthreads();
-    for (int size = 2; size <= kSortMax; size <<= 1) {
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        for (int i = tid; i < kSortMax; i += kHThreads) {
-          const int j = i ^ stride;
-          if (j > i) {
-            const int a = fin[i], bb = fin[j];
-            const bool up = (i & size) == 0;
-            if ((a > bb) == up) {
-              fin[i] = bb;
-              fin[j] = a;
-            }
-          }
+    if (n <= kBitmapMax) {
+      // Ascending order from a bitmap of the kept positions: mark them, then
+      // each thread emits the set bits of its run of words after a prefix sum.
+      uint32_t* const bm = tk;
+      const int words = (n + 31) >> 5;
+      __syncthreads();
+      for (int i = tid; i < words; i += kHThreads) bm[i] = 0u;
+      __syncthreads();
+      for (int i = tid; i < c_above && i < k; i += kHThreads) {
+        const int pos = fin[i];
+        atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+      }
+      for (int i = tid; i < c_in; i += kHThreads) {
+        const uint32_t key = ck[i];
+        const bool keep = key > theta ||
+                          (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
+        if (keep) atomicOr(&bm[cp[i] >> 5], 1u << (cp[i] & 31));
+      }
+      __syncthreads();
+      const int per = (words + kHThreads - 1) / kHThreads;
+      const int w0 = tid * per, w1 = min(words, w0 + per);
+      int mine = 0;
+      for (int wi = w0; wi < w1; ++wi) mine += __popc(bm[wi]);
+      int total;
+      int at = block_excl_sum_nw<kHWarps>(mine, buf, total);
+      for (int wi = w0; wi < w1; ++wi) {
+        uint32_t bits = bm[wi];
+        while (bits != 0u) {
+          const int bit = __ffs(bits) - 1;
+          bits &= bits - 1u;
+          if (at < k) out[at] = (wi << 5) + bit;
+          ++at;
         }
+      }
+    } else {
+      // Long rows: append the kept candidates and sort the k positions.
+      for (int base = 0; base < c_in; base += kHThreads) {
+        const int i = base + tid;
+        bool keep = false;
+        if (i < c_in) {
+          const uint32_t key = ck[i];
+          keep = key > theta ||
+                 (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
+        }
+        int tot_keep;
+        const int slot = s_nfin + block_excl_count_nw<kHWarps>(keep, buf, tot_keep);
+        if (keep && slot < kSortMax) fin[slot] = cp[i];
+        __syncthreads();
+        if (tid == 0) s_nfin += tot_keep;
         __syncthreads();
       }
+      for (int i = k + tid; i < kSortMax; i += kHThreads) fin[i] = 0x7FFFFFFF;
+      __syncthreads();
+      for (int size = 2; size <= kSortMax; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          for (int i = tid; i < kSortMax; i += kHThreads) {
+            const int j = i ^ stride;
+            if (j > i) {
+              const int a = fin[i], bb = fin[j];
+              const bool up = (i & size) == 0;
+              if ((a > bb) == up) {
+                fin[i] = bb;
+                fin[j] = a;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      for (int i = tid; i < k; i += kHThreads) out[i] = fin[i];
     }
-    for (int i = tid; i < k; i += kHThreads) out[i] = fin[i];
-  }
-  // Leave the row's histogram and counters zero for the next call.
-  for (int i = tid; i < kHistBins; i += kHThreads) gh[i] = 0;
-  if (tid == 0) {
-    cnt[0] = 0;
-    cnt[1] = 0;
-    cnt[2] = 0;
   }
 }
 
 }  // namespace
 
+size_t topk_hist_zero_bytes(int Nq) {
+  return static_cast<size_t>(Nq) * (kHistBins + 4) * sizeof(int);
+}
+
 size_t topk_hist_ws_bytes(int Nq, int top_k) {
-  return static_cast<size_t>(Nq) *
-         (kHistBins * sizeof(int) + top_k * sizeof(int) +
-          kCandMax * (sizeof(uint32_t) + sizeof(int)) + 4 * sizeof(int));
+  return topk_hist_zero_bytes(Nq) +
+         static_cast<size_t>(Nq) * (kCandMax * (sizeof(uint32_t) + sizeof(int)) +
+                                    top_k * sizeof(int));
 }
 
 cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream) {
@@ -602,18 +667,20 @@ cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t st
   uint8_t* p = static_cast<uint8_t*>(ws_region);
   P.hist = reinterpret_cast<int*>(p);
   p += static_cast<size_t>(a.Nq) * kHistBins * sizeof(int);
+  P.counters = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * 4 * sizeof(int);
   P.cand_key = reinterpret_cast<uint32_t*>(p);
   p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(uint32_t);
   P.cand_pos = reinterpret_cast<int*>(p);
   p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(int);
   P.gt_list = reinterpret_cast<int*>(p);
-  p += static_cast<size_t>(a.Nq) * a.top_k * sizeof(int);
-  P.counters = reinterpret_cast<int*>(p);
   // About two CTAs per SM in total, chunks of whole 512-key blocks.
   const long long target = 2LL * a.num_sms;
   P.chunks = static_cast<int>(std::max<long long>(1, target / std::max(1, a.Nq)));
   P.chunk = static_cast<int>(((a.max_len + P.chunks - 1) / P.chunks + kHThreads - 1) /
                              kHThreads * kHThreads);
+  // A chunk's hits are staged in shared arrays of kCandMax entries.
+  P.chunk = std::min(P.chunk, kCandMax);
   P.chunks = static_cast<int>((a.max_len + P.chunk - 1) / P.chunk);
   const size_t smem = static_cast<size_t>(kCandMax) * 12 + (kSortMax + 2048) * sizeof(int);
   cudaError_t e = ensure_smem_limit<topk_hist_kernel>(static_cast<int>(smem));

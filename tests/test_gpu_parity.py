@@ -299,3 +299,21 @@ def test_repeated_calls_on_one_workspace_agree():
                                     wl.scale)
     ref_out, ref_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, idx, wl.scale)
     parity.check_attention(first[0], first[1], ref_out, ref_lse)
+
+
+def test_standalone_calls_between_layer_calls_leave_it_unchanged():
+    """Standalone calls may use the layer's workspace as scratch in between."""
+    wl = _hist_batch()
+    dw = bd.DeviceWorkload(wl)
+    first = [t.cpu().numpy() for t in dw.forward()]
+    ld = _up4(wl.ctx_lens.max())
+    scores = torch.zeros(wl.Nq, ld, device="cuda")
+    out, lse, idx = dw.new_outputs()
+    bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws)
+    bd.topk(dw.batch, scores, ld, wl.top_k, idx, dw.ws)
+    bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, out, lse, dw.ws)
+    again = [t.cpu().numpy() for t in dw.forward()]
+    for a, b in zip(first, again):
+        assert np.array_equal(a, b)
+    assert np.array_equal(idx.cpu().numpy(), first[2])
+    bd.check_device_status(dw.ws)
