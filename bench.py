@@ -230,6 +230,10 @@ def run_ours(args):
     rank, local_rank, world = env_rank()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.prefill_only:  # profiling aid: the prefill object alone
+        from dsa_lightning_indexer_b200 import binding as bd
+        print(json.dumps({"prefill": prefill_bench(bd, dev, load_peaks(), args)}), flush=True)
+        return 0
     dist = None
     if world > 1:
         import datetime
@@ -458,8 +462,12 @@ def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
 
 
 def prefill_bench(bd, dev, peaks, args):
-    """One 16384-token causal prefill (64 heads, top_k 2048, planted indexer keys)."""
-    wl = synth.prefill_16k()
+    """One causal prefill (64 heads, top_k 2048, planted indexer keys): the
+    specified 16384 tokens, or --prefill-tokens for a smaller profiling case."""
+    if args.prefill_tokens == 16384:
+        wl = synth.prefill_16k()
+    else:
+        wl = synth.prefill(args.prefill_tokens, 64, 2048, seed=2, planted=True)
     dw = bd.DeviceWorkload(wl, dev)
     out, lse, idx = dw.new_outputs()
     ld = (int(wl.ctx_lens.max()) + 3) // 4 * 4
@@ -527,6 +535,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the prefill measurement (profiling aid)")
+    ap.add_argument("--prefill-tokens", type=int, default=16384)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-kernel-times", action="store_true")
