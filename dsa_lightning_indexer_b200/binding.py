@@ -45,6 +45,8 @@ SIGNATURES = {
     "dsa_layer_forward": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                          ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t,
                                          ctypes.c_uint32, _P]),
+    "dsa_sparse_attn_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, ctypes.c_int,
+                                               ctypes.c_float, _P, _P, _P]),
     "dsa_check_device_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -174,6 +176,14 @@ def sparse_attn(batch, q, kv, idx, top_k, scale, out, lse, ws, stream=None):
     _check(lib.dsa_sparse_attn(batch.ref, _bf16(q), H, _bf16(kv), _i32(idx), int(top_k),
                                float(scale), _f32(out), _f32(lse), _ptr(ws), ws.numel(),
                                _stream(stream)), "dsa_sparse_attn")
+
+
+def sparse_attn_noalloc(batch, q, kv, idx, top_k, scale, out, lse, stream=None):
+    """dsa_sparse_attn without a workspace (scratch in a static device array)."""
+    H = int(q.shape[1])
+    _check(lib.dsa_sparse_attn_noalloc(batch.ref, _bf16(q), H, _bf16(kv), _i32(idx), int(top_k),
+                                       float(scale), _f32(out), _f32(lse), _stream(stream)),
+           "dsa_sparse_attn_noalloc")
 
 
 def layer_forward(batch, q, q_idx, w, k_idx, kv, top_k, scale, out, lse, idx, ws, stream=None):

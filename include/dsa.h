@@ -163,6 +163,30 @@ DSA_API dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, 
                              int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags,
                              void* stream);
 
+/*
+ * dsa_sparse_attn without a workspace, for callers that cannot allocate
+ * device memory when they run the layer (a fixed pre-sized memory pool, a
+ * runtime that hands kernels only the tensors it owns, a plugin host that
+ * forbids allocation after start-up).  There is no counterpart on the source
+ * pages: this is a deployment convenience of this library.
+ *
+ * Arguments, results and errors are those of dsa_sparse_attn, minus ws and
+ * ws_bytes.  Its scratch (the partial results of a query's selected set split
+ * over CTAs) lives in one static device array of 10 MiB that every GPU
+ * holding this library keeps until process exit; a launch needing more
+ * returns DSA_ERR_WORKSPACE and runs nothing (no shape within the fixed limits
+ * needs more than about 9.3 MiB).  It allocates nothing and calls no
+ * allocating routine.  The first call on each device looks up the array's
+ * address; make it before capturing a stream into a CUDA graph.  Calls share
+ * the array: calls that may overlap on the GPU (different streams) race and
+ * must be serialised by the caller.  It always runs the CUDA-core attention
+ * kernels, so results agree with dsa_sparse_attn within the library's
+ * tolerances (not bit for bit).
+ */
+DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, const uint16_t* q, int H,
+                                           const uint16_t* kv, const int32_t* idx, int top_k,
+                                           float scale, float* out, float* lse, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that the
  * kernels of earlier calls on this workspace may have set.  Returns DSA_OK,
  * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the stream itself reports an
