@@ -223,7 +223,7 @@ def launches_per_layer(wl, sms=148):
     when few rows split the selected set over CTAs, the merge of the slices."""
     seqs = int((np.diff(wl.q_offsets) > 0).sum())
     few_rows = wl.Nq * ((wl.H + 63) // 64) < sms
-    return (seqs + 63) // 64 + 1 + 1 + (1 if few_rows and wl.top_k > 32 else 0)
+    return (seqs + 63) // 64 + 1 + 1 + (1 if few_rows and wl.top_k > 16 else 0)
 
 
 def run_ours(args):

@@ -61,7 +61,10 @@ struct AttnPlan {
   int n_split;      // slices of the selected set per (row, head block)
   int split_len;    // index slots per slice (multiple of 32)
 };
+// Plan of the tcgen05 kernel (dsa_sparse_attn, dsa_layer_forward).
 AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms);
+// Plan of the CUDA-core kernels (16 heads per CTA, slices for few rows).
+AttnPlan attn_plan_core(int Nq, int H, int top_k, int num_sms);
 size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p);
 
 struct AttnArgs {
@@ -84,6 +87,8 @@ struct AttnArgs {
   AttnPlan plan;
 };
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream);
+// Merges the slices of a split launch (plan.n_split > 1) into out and lse.
+cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes`, once per device

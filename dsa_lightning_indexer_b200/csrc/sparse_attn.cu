@@ -407,18 +407,35 @@ cudaError_t launch_ng(const AttnParams& P, int head_blocks, cudaStream_t stream)
 }  // namespace
 
 AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms) {
+  // tcgen05 kernel: 64 heads per CTA (one CTA per SM).  With few rows the
+  // selected set is sliced so the GPU fills; slices hold whole 16-slot groups.
+  AttnPlan p;
+  p.tc = 1;
+  p.hb = kHeadsPerCta;
+  p.head_blocks = (H + kHeadsPerCta - 1) / kHeadsPerCta;
+  p.n_split = 1;
+  p.split_len = top_k;
+  const long long base = static_cast<long long>(Nq) * p.head_blocks;
+  if (base > 0 && base < num_sms) {
+    const int want = static_cast<int>(num_sms / base);
+    const int n = std::min(std::min(want, kMaxSplit), (top_k + 15) / 16);
+    if (n > 1) {
+      const int per = ((top_k + n - 1) / n + 15) / 16 * 16;
+      p.n_split = (top_k + per - 1) / per;
+      p.split_len = per;
+    }
+  }
+  return p;
+}
+
+AttnPlan attn_plan_core(int Nq, int H, int top_k, int num_sms) {
   AttnPlan p;
   p.tc = 0;
   p.hb = std::min(kHeadsPerCta, (H + 15) / 16 * 16);
   p.head_blocks = (H + p.hb - 1) / p.hb;
   p.n_split = 1;
   const long long rows = Nq;
-  if (rows * ((H + kHeadsPerCta - 1) / kHeadsPerCta) >= num_sms) {
-    // Many rows: the tcgen05 kernel, 64 heads per CTA, whole selected set.
-    p.tc = 1;
-    p.hb = kHeadsPerCta;
-    p.head_blocks = (H + kHeadsPerCta - 1) / kHeadsPerCta;
-  } else if (rows > 0) {
+  if (rows * p.head_blocks < num_sms && rows > 0) {
     // Few rows: 16 heads per CTA (two CTAs fit an SM) and slices of the set.
     p.hb = 16;
     p.head_blocks = (H + 15) / 16;
@@ -468,6 +485,19 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
     default: e = launch_ng<4>(P, a.plan.head_blocks, stream); break;
   }
   if (e != cudaSuccess || P.n_split == 1) return e;
+  return launch_pdl(attn_merge_kernel, dim3(a.Nq, a.H), dim3(128), 0, stream, 0, P);
+}
+
+cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t stream) {
+  AttnParams P = {};
+  P.Nq = a.Nq;
+  P.H = a.H;
+  P.n_split = a.plan.n_split;
+  const size_t n_rec = static_cast<size_t>(a.plan.n_split) * a.Nq * a.H;
+  P.part_o = a.part;
+  P.part_ml = reinterpret_cast<float2*>(a.part + n_rec * kValue);
+  P.out = a.out;
+  P.lse = a.lse;
   return launch_pdl(attn_merge_kernel, dim3(a.Nq, a.H), dim3(128), 0, stream, 0, P);
 }
 

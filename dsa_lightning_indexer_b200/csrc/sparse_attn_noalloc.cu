@@ -96,15 +96,8 @@ extern "C" DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, co
   }
   if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
 
-  // The CUDA-core kernels, split as dsa_sparse_attn would split them.
-  AttnPlan plan = attn_plan(batch->Nq, H, top_k, 148);
-  if (plan.tc) {  // many rows: whole selected set per CTA, no partials
-    plan.tc = 0;
-    plan.hb = H < 64 ? (H + 15) / 16 * 16 : 64;
-    plan.head_blocks = (H + plan.hb - 1) / plan.hb;
-    plan.n_split = 1;
-    plan.split_len = (top_k + 31) / 32 * 32;
-  }
+  // The CUDA-core kernels and their split plan.
+  const AttnPlan plan = attn_plan_core(batch->Nq, H, top_k, 148);
   if (attn_partial_bytes(batch->Nq, H, plan) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
 
   int dev = 0, major = 0, minor = 0;

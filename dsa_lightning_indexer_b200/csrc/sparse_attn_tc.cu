@@ -75,7 +75,10 @@ struct TcParams {
   float* out;
   float* lse;
   unsigned* err;
+  float* part_o;        // [n_split][Nq][H][512] unnormalised slice outputs (n_split > 1)
+  float2* part_ml;      // [n_split][Nq][H] (running max in log2 units, row sum)
   int B, Nq, H, top_k;
+  int n_split, split_len;  // slices of the selected set, slots per slice
   int idx_prefix;       // valid entries are the first min(top_k, p+1) slots
   float scale_log2;
 };
@@ -185,6 +188,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int lane = lane_id();
   const int r = blockIdx.x;
   const int h0 = blockIdx.y * kHB;
+  const int sp = blockIdx.z;
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
@@ -219,30 +223,45 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int pos = P.ctx_lens[b] - (P.q_offsets[b + 1] - q0) + (r - q0);
     n_slots = min(P.top_k, pos + 1);
   }
-  const int n_tiles = (n_slots + kT - 1) / kT;
+  // This CTA's slice of the slots.
+  const int slot_lo = sp * P.split_len;
+  const int slot_hi = min(n_slots, slot_lo + P.split_len);
+  const int n_tiles = slot_hi > slot_lo ? (slot_hi - slot_lo + kT - 1) / kT : 0;
 
   if (warp >= 5) {
     // ------------------------------------------------------------ gather --
+    // Each thread copies whole 128-byte box rows (eight 16-byte pieces with
+    // the swizzle applied), after the group has staged the tile's positions.
     const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
     const int gt = threadIdx.x - (5 + 2 * grp) * 32;
+    int* const gidx = tidx + grp * kT;
     bool ok = true;
     for (int t = grp; t < n_tiles && ok; t += 2) {
       const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
+      if (gt < kT) {
+        const int slot = slot_lo + t * kT + gt;
+        gidx[gt] = slot < slot_hi ? __ldg(idx_row + slot) : -1;
+      }
+      named_bar_sync(2 + grp, kGroupThreads);
       const uint32_t stage = sKV + grp * kKVStage;
-      for (int e = gt; e < kT * (kLatent / 8); e += kGroupThreads) {
-        const int i = e / (kLatent / 8), ch = e - i * (kLatent / 8);
-        const int slot = t * kT + i;
-        const int pos = slot < n_slots ? __ldg(idx_row + slot) : -1;
-        if (ch == 0) tidx[grp * kT + i] = pos;
-        const int box = ch >> 3, c = ch & 7;
-        const uint32_t dst = stage + box * kKVBox + i * 128 + ((c ^ (i & 7)) << 4);
+      for (int item = gt; item < kT * kBoxes; item += kGroupThreads) {
+        const int i = item / kBoxes, bx = item - i * kBoxes;
+        const int pos = gidx[i];
+        const uint32_t drow = stage + bx * kKVBox + i * 128;
+        const uint32_t x = static_cast<uint32_t>(i & 7);
         if (pos >= 0) {
-          cp_async16_tc(dst, P.kv + static_cast<size_t>(kv0 + pos) * kLatent + ch * 8);
+          const __nv_bfloat16* src = P.kv + static_cast<size_t>(kv0 + pos) * kLatent + bx * 64;
+#pragma unroll
+          for (uint32_t c = 0; c < 8; ++c) cp_async16_tc(drow + ((c ^ x) << 4), src + c * 8);
         } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u)
-                       : "memory");
+#pragma unroll
+          for (uint32_t c = 0; c < 8; ++c) {
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(drow + (c << 4)),
+                         "r"(0u)
+                         : "memory");
+          }
         }
       }
       asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
@@ -405,7 +424,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     named_bar_sync(1, kSoftThreads);
     if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     tc_fence_after();
-    if (ok) {
+    if (ok && P.n_split == 1) {
 #pragma unroll 1
       for (int blk = 0; blk < 4; ++blk) {
         const int dv = 128 * blk + 32 * q + lane;
@@ -430,6 +449,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         P.lse[static_cast<size_t>(r) * P.H + h0 + hl] =
             l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
       }
+    } else if (ok) {
+      // One slice of the set: unnormalised O and (max, sum) for the merge.
+      const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        const int dv = 128 * blk + 32 * q + lane;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          if (n_tiles > 0) {
+            tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int h = h0 + 32 * half + j;
+            if (h < P.H) P.part_o[(rec + h) * kValue + dv] = __uint_as_float(o[j]);
+          }
+        }
+      }
+      if (owner && h0 + hl < P.H) P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
     }
   }
 
@@ -470,14 +513,21 @@ cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   P.lse = a.lse;
   P.err = a.err;
   P.idx_prefix = a.idx_prefix ? 1 : 0;
+  P.n_split = a.plan.n_split;
+  P.split_len = a.plan.split_len;
+  const size_t n_rec = static_cast<size_t>(a.plan.n_split) * a.Nq * a.H;
+  P.part_o = a.part;
+  P.part_ml = a.part ? reinterpret_cast<float2*>(a.part + n_rec * kValue) : nullptr;
   P.B = a.B;
   P.Nq = a.Nq;
   P.H = a.H;
   P.top_k = a.top_k;
   P.scale_log2 = a.scale * kLog2eTc;
   const int head_blocks = (a.H + kHB - 1) / kHB;
-  return launch_pdl(sparse_attn_tc_kernel, dim3(a.Nq, head_blocks), dim3(kThreadsTc),
-                    static_cast<size_t>(kSmemTc), stream, 0, qmap, P);
+  e = launch_pdl(sparse_attn_tc_kernel, dim3(a.Nq, head_blocks, a.plan.n_split),
+                 dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, P);
+  if (e != cudaSuccess || a.plan.n_split == 1) return e;
+  return launch_attn_merge(a, stream);
 }
 
 }  // namespace dsa
