@@ -407,7 +407,7 @@ __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, i
   need = remaining;
 }
 
-__global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P) {
+__global__ void __launch_bounds__(kHThreads, 2) topk_hist_kernel(const HistParams P) {
   extern __shared__ __align__(16) uint8_t hsm[];
   uint32_t* const ck = reinterpret_cast<uint32_t*>(hsm);           // [kCandMax] keys
   int* const cp = reinterpret_cast<int*>(ck + kCandMax);            // [kCandMax] positions
@@ -481,10 +481,20 @@ __global__ void __launch_bounds__(kHThreads) topk_hist_kernel(const HistParams P
   if (c_in <= kCandMax) {
     const int s0 = c * P.chunk, s1 = min(n, s0 + P.chunk);
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = s0; base < s1; base += kHThreads) {
-      const int s = base + tid;
+    // All of the chunk's loads are issued before any is used.
+    constexpr int kPer = kCandMax / kHThreads;
+    uint32_t keys[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int s = s0 + j * kHThreads + tid;
+      keys[j] = s < s1 ? score_key(__ldcg(sc + s)) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (s0 + j * kHThreads >= s1) break;
+      const int s = s0 + j * kHThreads + tid;
       const bool in = s < s1;
-      const uint32_t key = in ? score_key(sc[s]) : 0u;
+      const uint32_t key = keys[j];
       const uint32_t bin = key >> kHistShift;
       const bool gt = in && bin > bstar;
       const bool eq = in && bin == bstar;
