@@ -7,21 +7,17 @@
 // selected tokens; devotd.net section 2 — one key-only latent cache whose
 // leading 512 entries serve as V.)
 //
-// One CTA owns one query row (or one slice of its selected set) and a block of
-// 64 heads, and walks the selected rows in tiles of 48 gathered cache rows:
-//   S  = Q[64 heads, 576] . K_tile[48, 576]^T      M = 64, N = 48,  K = 576
-//   O += P[64 heads, 48] . V_tile[48, 512]         M = 64, N = 256 (x2), K = 48
-// Heads are the M dimension of both products, so each head row lives in one
-// TMEM lane: O in the lower 16 lanes of each lane quadrant, S in the upper 16
-// (the two halves an M = 64 accumulator can occupy).  V is therefore read once
-// per key block for all 64 heads.  A head row's softmax is split between a
-// pair of threads (24 keys each), exchanging max and sum with one shuffle; P
-// goes to shared memory as bf16 hi + lo parts (two MMAs), keeping its rounding
-// error near 2^-16.  The gathered tile is stored once, in the 128-byte
-// swizzled layout, and read by both MMAs: K-major as the B operand of S,
-// MN-major as the B operand of O.  The running maximum is raised lazily (only
-// when a tile's maximum exceeds it by more than 2^8), and O is then rescaled
-// in TMEM by the threads that own its rows.
+// One CTA owns one query row and a block of 64 heads, and walks the row's
+// selected set in tiles of 48 gathered cache rows:
+//   S    = Q[64 heads, 576] . K_tile[48, 576]^T      M = 64,  N = 48, K = 576
+//   O^T += V_tile^T[512, 48] . P^T[48, 64 heads]     M = 128 (x4), N = 64, K = 48
+// S lands in TMEM with one head per lane, so each softmax thread owns one
+// head row: max, exp2 and row sum stay in registers.  P is written to shared
+// memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
+// 2^-16.  The gathered tile is stored once, in the 128-byte swizzled layout,
+// and read by both MMAs: K-major as the B operand of S, MN-major as the A
+// operand of O^T.  The running maximum is raised lazily (only when a tile's
+// maximum exceeds it by more than 2^8), and O^T in TMEM is then rescaled.
 //
 // Warp roles (288 threads): warps 0-3 softmax and output (TMEM quadrants
 // 0-3), warp 4 TMEM allocation, the Q load (TMA) and single-thread MMA issue,
@@ -63,13 +59,12 @@ constexpr int kSmemTc = kSmemUsed + 1024;               // alignment slack
 static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-// O: lanes 0-15 of each quadrant, columns 0-511 (two N = 256 accumulators).
-// S: lanes 16-31 of each quadrant, buffers at columns 0 and 64.
-constexpr uint32_t kLaneS = 16u << 16;
+constexpr uint32_t kColS = 0;     // S buffers at columns 0 and 64 (M = 64 layout)
+constexpr uint32_t kColO = 128;   // O^T blocks at 128, 192, 256, 320
 
 // kind::f16 instruction descriptors (bf16 in, fp32 accumulate).
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, kT);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(64, 256) | (1u << 16);  // B (V) MN-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
 
 struct TcParams {
   const int32_t* q_offsets;
@@ -112,53 +107,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-// 16 TMEM lanes (from the address's lane) by a whole warp: threads 0-15 read
-// columns [c, c+N), threads 16-31 columns [c+off, c+off+N) of the same lanes.
-__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16], 24;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_16x32bx2_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], 24;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_16x32bx2_x32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32], 32;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st_16x32bx2_x32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
       "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
           taddr),
@@ -338,13 +286,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         const uint32_t kvs = sKV + st * kKVStage;
         const uint32_t phi = sP + (2 * st) * kPBuf, plo = phi + kPBuf;
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {  // value dims 256*nh .. +255 (four boxes)
+        for (int blk = 0; blk < 4; ++blk) {
 #pragma unroll
           for (int kk = 0; kk < kT / 16; ++kk) {
-            const uint64_t bv = sdesc_sw128_mn(kvs + (4 * nh) * kKVBox + kk * 2048, kKVBox);
-            const uint32_t d = tmem + 256u * nh;
-            tc_mma_bf16(d, sdesc_sw128(phi + kk * 32), bv, kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_bf16(d, sdesc_sw128(plo + kk * 32), bv, kIdescPV, 1u);
+            const uint64_t a = sdesc_sw128_mn(kvs + (2 * blk) * kKVBox + kk * 2048, kKVBox);
+            const uint32_t d = tmem + kColO + 64u * blk;
+            tc_mma_bf16(d, a, sdesc_sw128(phi + kk * 32), kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_bf16(d, a, sdesc_sw128(plo + kk * 32), kIdescPV, 1u);
           }
         }
         tc_commit(b_kvempty(st));
@@ -359,7 +307,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t kvs = sKV + st * kKVStage;
-        const uint32_t d = tmem + kLaneS + 64u * st;
+        const uint32_t d = tmem + kColS + 64u * st;
 #pragma unroll 4
         for (int ks = 0; ks < kLatent / 16; ++ks) {
           const uint32_t off = (ks & 3) * 32;
@@ -373,14 +321,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else {
     // ----------------------------------------------------------- softmax --
-    // Warp q owns head rows 16q .. 16q+15: S rows in TMEM lanes 32q+16.., O
-    // rows in lanes 32q.. .  Thread pair (l, l+16) shares head 16q + l%16:
-    // keys 0-23 / 24-47 of S, value dims [64j, 64j+32) / [64j+32, 64j+64) of O.
-    const int q = warp;
-    const int half = lane >> 4;
+    const int q = warp;                          // TMEM lane quadrant
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const bool owner = lane < 16;                // owns head row 16q + lane
     const int hl = 16 * q + (lane & 15);
-    const uint32_t s_base = tmem + (static_cast<uint32_t>(32 * q) << 16) + kLaneS;
-    const uint32_t o_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
@@ -389,80 +333,83 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       ok = mbar_wait(b_sfull(st), ph, P.err);
       if (!ok) break;
       tc_fence_after();
-      uint32_t va[16], vb[8];
-      tmem_ld_16x32bx2_x16(s_base + 64u * st, va);       // keys 0-15 | 24-39
-      tmem_ld_16x32bx2_x8(s_base + 64u * st + 16u, vb);  // keys 16-23 | 40-47
+      uint32_t va[32], vb[16];
+      tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64u * st, va);
+      tmem_ld_32x32b_x16(tmem + lane_base + kColS + 64u * st + 32u, vb);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(b_sempty(st));
       // The tile's slot list was written by its gather group before kv_full.
       ok = mbar_wait(b_kvfull(st), ph, P.err);
       if (!ok) break;
-      // Logits in base 2; unused slots masked.  This thread's 24 keys.
-      constexpr int kHalf = kT / 2;
-      float sv[kHalf];
-      const int* const ti = tidx + st * kT + half * kHalf;
+      // Logits in base 2; unused slots masked.
+      float s[kT];
+      const int* const ti = tidx + st * kT;
       float tmax = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < kHalf; ++k) {
-        const float raw_s = __uint_as_float(k < 16 ? va[k] : vb[k - 16]);
-        sv[k] = ti[k] >= 0 ? raw_s * P.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, sv[k]);
+      for (int k = 0; k < kT; ++k) {
+        const float raw_s = __uint_as_float(k < 32 ? va[k] : vb[k - 32]);
+        s[k] = ti[k] >= 0 ? raw_s * P.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, s[k]);
       }
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
       const bool raise = tmax > m_run + kRescaleLog2 || (m_run == -INFINITY && tmax > -INFINITY);
       const float m_new = raise ? tmax : m_run;
       const float alpha = raise ? exp2f(m_run - m_new) : 1.f;
       float sum = 0.f;
-      uint32_t hi[kHalf / 2], lo[kHalf / 2];
+      uint32_t hi[kT / 2], lo[kT / 2];
 #pragma unroll
-      for (int k = 0; k < kHalf; k += 2) {
-        const float p0 = sv[k] == -INFINITY ? 0.f : exp2f(sv[k] - m_new);
-        const float p1 = sv[k + 1] == -INFINITY ? 0.f : exp2f(sv[k + 1] - m_new);
+      for (int k = 0; k < kT; k += 2) {
+        const float p0 = s[k] == -INFINITY ? 0.f : exp2f(s[k] - m_new);
+        const float p1 = s[k + 1] == -INFINITY ? 0.f : exp2f(s[k + 1] - m_new);
         sum += p0 + p1;
         const uint32_t h2 = pack2_bf16(p0, p1);
         const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&h2);
         hi[k / 2] = h2;
         lo[k / 2] = pack2_bf16(p0 - __low2float(hb), p1 - __high2float(hb));
       }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
+      if (owner) {
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        alpha_s[hl] = alpha;
+      }
       // P buffer `st` is free once the P.V of tile t-2 has completed.
       ok = mbar_wait(b_pempty(st), ph ^ 1u, P.err);
       if (!ok) break;
-      {
+      if (owner) {
         const uint32_t prow_hi = sP + (2 * st) * kPBuf + hl * 128;
         const uint32_t prow_lo = prow_hi + kPBuf;
 #pragma unroll
-        for (int cc = 0; cc < kHalf / 8; ++cc) {
-          const int c = half * (kHalf / 8) + cc;  // 16-byte chunk of the 128-byte row
+        for (int c = 0; c < kT / 8; ++c) {
           const uint32_t off = static_cast<uint32_t>((c ^ (hl & 7)) << 4);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_hi + off),
-                       "r"(hi[4 * cc]), "r"(hi[4 * cc + 1]), "r"(hi[4 * cc + 2]),
-                       "r"(hi[4 * cc + 3])
+                       "r"(hi[4 * c]), "r"(hi[4 * c + 1]), "r"(hi[4 * c + 2]), "r"(hi[4 * c + 3])
                        : "memory");
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_lo + off),
-                       "r"(lo[4 * cc]), "r"(lo[4 * cc + 1]), "r"(lo[4 * cc + 2]),
-                       "r"(lo[4 * cc + 3])
+                       "r"(lo[4 * c]), "r"(lo[4 * c + 1]), "r"(lo[4 * c + 2]), "r"(lo[4 * c + 3])
                        : "memory");
         }
       }
       fence_proxy_async_smem();
-      // If any head raised its running max, scale its O row (after the previous P.V).
-      const bool any = named_bar_or(1, kSoftThreads, raise && t > 0);
+      // If any head raised its running max, scale O^T (after the previous P.V).
+      const bool any = named_bar_or(1, kSoftThreads, owner && raise && t > 0);
       if (any) {
         ok = mbar_wait(b_odone, static_cast<uint32_t>((t - 1) & 1), P.err);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int j = 0; j < kValue / 64; ++j) {
-          uint32_t o[32];
-          tmem_ld_16x32bx2_x32(o_base + 64u * j, o);
-          tmem_ld_wait();
+        for (int blk = 0; blk < 4; ++blk) {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-          tmem_st_16x32bx2_x32(o_base + 64u * j, o);
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_base + kColO + 64u * blk + 32u * half;
+            tmem_ld_32x32b_x32(ta, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha_s[32 * half + j]);
+            }
+            tmem_st_32x32b_x32(ta, o);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -470,50 +417,62 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_arrive(b_pfull(st));
     }
     // ------------------------------------------------------------ output --
+    if (owner) {
+      m_s[hl] = m_run;
+      l_s[hl] = l_run;
+    }
+    named_bar_sync(1, kSoftThreads);
     if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     tc_fence_after();
-    const int h = h0 + hl;
-    if (ok) {
-      const bool split = P.n_split > 1;
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float scale_o = split ? 1.f : inv;
-      float* dst = nullptr;
-      if (split) {
-        const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
-        dst = P.part_o + (rec + h) * kValue;
-      } else {
-        dst = P.out + (static_cast<size_t>(r) * P.H + h) * kValue;
-      }
+    if (ok && P.n_split == 1) {
 #pragma unroll 1
-      for (int j = 0; j < kValue / 64; ++j) {
-        uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld_16x32bx2_x32(o_base + 64u * j, o);
+      for (int blk = 0; blk < 4; ++blk) {
+        const int dv = 128 * blk + 32 * q + lane;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
           tmem_ld_wait();
-        } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = 0u;
-        }
-        if (h < P.H) {
-          float4* const d4 = reinterpret_cast<float4*>(dst + 64 * j + 32 * half);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            d4[x] = make_float4(__uint_as_float(o[4 * x]) * scale_o,
-                                __uint_as_float(o[4 * x + 1]) * scale_o,
-                                __uint_as_float(o[4 * x + 2]) * scale_o,
-                                __uint_as_float(o[4 * x + 3]) * scale_o);
+          for (int j = 0; j < 32; ++j) {
+            const int hh = 32 * half + j;
+            const int h = h0 + hh;
+            if (h < P.H) {
+              const float L = l_s[hh];
+              P.out[(static_cast<size_t>(r) * P.H + h) * kValue + dv] =
+                  L > 0.f ? __uint_as_float(o[j]) / L : 0.f;
+            }
           }
         }
       }
-      if (half == 0 && h < P.H) {
-        if (split) {
-          const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
-          P.part_ml[rec + h] = make_float2(m_run, l_run);
-        } else if (P.lse) {
-          P.lse[static_cast<size_t>(r) * P.H + h] =
-              l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
+      if (P.lse && owner && h0 + hl < P.H) {
+        P.lse[static_cast<size_t>(r) * P.H + h0 + hl] =
+            l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
+      }
+    } else if (ok) {
+      // One slice of the set: unnormalised O and (max, sum) for the merge.
+      const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
+#pragma unroll 1
+      for (int blk = 0; blk < 4; ++blk) {
+        const int dv = 128 * blk + 32 * q + lane;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          if (n_tiles > 0) {
+            tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int h = h0 + 32 * half + j;
+            if (h < P.H) P.part_o[(rec + h) * kValue + dv] = __uint_as_float(o[j]);
+          }
         }
       }
+      if (owner && h0 + hl < P.H) P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
     }
   }
 
