@@ -379,7 +379,8 @@ def kernel_times(bd, copies, wl, steps, dev):
     torch.cuda.synchronize()
     res = {}
     side = torch.cuda.Stream(dev)
-    for name, fn in (("indexer_score_us", k1), ("topk_us", k2), ("sparse_attn_us", k3)):
+    for name, fn in (("indexer_score_us", k1), ("topk_standalone_us", k2),
+                     ("sparse_attn_us", k3)):
         g = torch.cuda.CUDAGraph()
         side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(side):
@@ -401,6 +402,8 @@ def kernel_times(bd, copies, wl, steps, dev):
         del g
     res["launches_timed"] = n * reps
     res["method"] = "per-kernel CUDA graphs of 16 launches, CUDA events around replays"
+    res["note"] = ("each C-ABI call alone; the standalone top-k has no indexer histogram and "
+                   "takes the cluster path, the layer's takes the histogram path")
     for c in copies:
         bd.check_device_status(c.ws)
     return res

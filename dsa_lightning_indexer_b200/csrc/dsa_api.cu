@@ -97,7 +97,8 @@ struct WsLayout {
 // score-key histograms and the selection makes one filtering pass.
 bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
   return b->Nq > 0 && b->Nq <= kPlanSms && info.max_len >= 8192 &&
-         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B);
+         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B) &&
+         topk_hist_supported(b->Nq, info.max_len);
 }
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -110,7 +111,8 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
   w.hist_topk = scores && plan_hist_topk(b, info, top_k);
   w.hist_off = w.scores_off + w.scores_bytes;
-  w.hist_bytes = w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k), 256) : 0;
+  w.hist_bytes =
+      w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0;
   w.part_off = w.hist_off + w.hist_bytes;
   w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
   w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;

@@ -50,7 +50,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 // topk_hist_ws_bytes() bytes in all; its first topk_hist_zero_bytes() bytes
 // (histograms and counters) must be zero when the indexer starts.
 size_t topk_hist_zero_bytes(int Nq);
-size_t topk_hist_ws_bytes(int Nq, int top_k);
+size_t topk_hist_ws_bytes(int Nq, int top_k, int64_t max_len);
+int topk_hist_chunks(int Nq, int64_t max_len, int* chunk_len);
+bool topk_hist_supported(int Nq, int64_t max_len);
 cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream);
 
 // How the attention launch covers (query row, head block, slice of the set).

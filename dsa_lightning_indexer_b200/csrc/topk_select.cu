@@ -344,7 +344,9 @@ constexpr int kHThreads = 512;
 constexpr int kHWarps = kHThreads / 32;
 constexpr int kCandMax = 8192;   // keys of the threshold bin kept for the exact pass
 constexpr int kSortMax = 2048;   // >= top_k, power of two
-constexpr int kBitmapMax = kCandMax * 32;  // rows up to this length order by bitmap
+constexpr int kFineBits = 11;    // sub-histogram of the threshold bin: the next 11 key bits
+constexpr int kFineShift = kHistShift - kFineBits;
+constexpr int kFineBins = 1 << kFineBits;
 
 struct HistParams {
   const int32_t* q_offsets;
@@ -354,10 +356,12 @@ struct HistParams {
   int32_t* idx;
   int B, top_k, chunk, chunks;
   int* hist;            // [Nq][kHistBins], zeroed before the indexer runs
-  int* counters;        // [Nq][4]: above count, candidate count, arrival ticket; zeroed too
-  uint32_t* cand_key;   // [Nq][kCandMax]
-  int* cand_pos;        // [Nq][kCandMax]
-  int* gt_list;         // [Nq][top_k]
+  int* fine;            // [Nq][kFineBins] sub-histogram of the threshold bin; zeroed too
+  int* counters;        // [Nq][4]: keys above the bin, candidates, fallback flag; zeroed too
+  uint32_t* cand_key;   // [Nq][kCandMax] keys of the threshold bin (any order)
+  int* cand_pos;        // [Nq][kCandMax] their positions
+  int* chunk_gt;        // [Nq][chunks][top_k] positions above the bin, per chunk
+  int* chunk_ngt;       // [Nq][chunks] how many
 };
 
 // Finds, among `n` shared-memory keys, the `want`-th largest key theta and how
@@ -407,47 +411,94 @@ __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, i
   need = remaining;
 }
 
-__global__ void __launch_bounds__(kHThreads, 2) topk_hist_kernel(const HistParams P) {
+// Row bookkeeping shared by the two kernels of the histogram path.
+struct HistRow {
+  int r, c;
+  int* gh;
+  int* cnt;
+  int32_t* out;
+  const float* sc;
+};
+
+__device__ __forceinline__ HistRow hist_row(const HistParams& P) {
+  HistRow h;
+  h.r = blockIdx.x / P.chunks;
+  h.c = blockIdx.x - h.r * P.chunks;
+  h.gh = P.hist + static_cast<size_t>(h.r) * kHistBins;
+  h.cnt = P.counters + static_cast<size_t>(h.r) * 4;
+  h.out = P.idx + static_cast<size_t>(h.r) * P.top_k;
+  h.sc = P.scores + static_cast<size_t>(h.r) * P.ld;
+  return h;
+}
+
+// Causal length of query row r, looked up by one warp with all of its loads
+// in flight at once (lane l checks sequences l, l + 32, ...).
+__device__ __forceinline__ int row_causal_len_warp(const HistParams& P, int r) {
+  int n = 0;
+  for (int b = threadIdx.x & 31; b < P.B; b += 32) {
+    const int q0 = __ldg(P.q_offsets + b), q1 = __ldg(P.q_offsets + b + 1);
+    const int L = __ldg(P.ctx_lens + b);
+    if (r >= q0 && r < q1) n = L - (q1 - q0) + (r - q0) + 1;
+  }
+  return __reduce_max_sync(0xffffffffu, n);
+}
+
+// Filter: the bin holding the k-th largest key comes from the histogram the
+// indexer built; one pass over this CTA's chunk keeps the positions above
+// the bin (per chunk, for the emit kernel) and the keys in the bin (the
+// row's candidates), and counts the candidates by the next kFineBits key
+// bits into the row's sub-histogram.
+__global__ void __launch_bounds__(kHThreads, 2) topk_filter_kernel(const HistParams P) {
   extern __shared__ __align__(16) uint8_t hsm[];
-  uint32_t* const ck = reinterpret_cast<uint32_t*>(hsm);           // [kCandMax] keys
-  int* const cp = reinterpret_cast<int*>(ck + kCandMax);            // [kCandMax] positions
-  uint32_t* const tk = reinterpret_cast<uint32_t*>(cp + kCandMax);  // [kCandMax] tie keys
-  int* const fin = reinterpret_cast<int*>(tk + kCandMax);           // [kSortMax] result
-  int* const hist = fin + kSortMax;                                 // [2048]
+  int* const st_gt = reinterpret_cast<int*>(hsm);                         // [kSortMax]
+  uint32_t* const st_ck = reinterpret_cast<uint32_t*>(st_gt + kSortMax);  // [kCandMax]
+  int* const st_cp = reinterpret_cast<int*>(st_ck + kCandMax);            // [kCandMax]
   __shared__ int buf[kHWarps + 1];
-  __shared__ int s_bin, s_above, s_inbin, s_last, s_nfin;
+  __shared__ int s_bin, s_above, s_inbin, s_ngt, s_nc, s_cbase;
 
   pdl_wait();
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31;
-  const int r = blockIdx.x / P.chunks, c = blockIdx.x % P.chunks;
-  const int b = owner_seq(P.q_offsets, P.B, r);
-  const int q0 = P.q_offsets[b];
-  const int n = P.ctx_lens[b] - (P.q_offsets[b + 1] - q0) + (r - q0) + 1;
+  const HistRow R = hist_row(P);
   const int k = P.top_k;
-  int* const gh = P.hist + static_cast<size_t>(r) * kHistBins;
-  int* const cnt = P.counters + static_cast<size_t>(r) * 4;
-  int32_t* const out = P.idx + static_cast<size_t>(r) * k;
-  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
-
+  __shared__ int s_n;
+  if (tid < 32) {  // the row's length, while the other warps' loads go out
+    const int n = row_causal_len_warp(P, R.r);
+    if (tid == 0) s_n = n;
+  }
+  // The chunk's scores (within the row's stride; masked by the length below)
+  // and the row's histogram are loaded before anything waits on them.
+  const int s0 = R.c * P.chunk;
+  const int s_end = static_cast<int>(min(static_cast<long long>(s0 + P.chunk), P.ld));
+  constexpr int kPer = kCandMax / kHThreads;
+  uint32_t keys[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int s = s0 + j * kHThreads + tid;
+    keys[j] = s < s_end ? score_key(__ldcg(R.sc + s)) : 0u;
+  }
+  const int u = kHThreads - 1 - tid;  // thread t reads bins 8u .. 8u+7, u = 511 - t
+  int cb[8];
+  int tot = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    cb[j] = __ldcg(R.gh + 8 * u + j);
+    tot += cb[j];
+  }
+  __syncthreads();
+  const int n = s_n;
+  if (R.c == 0 && tid == 0) R.cnt[3] = n;
   if (n <= k) {  // every causal position is kept
-    if (c == 0) {
-      for (int i = tid; i < k; i += kHThreads) out[i] = i < n ? i : -1;
+    if (R.c == 0) {
+      for (int i = tid; i < k; i += kHThreads) R.out[i] = i < n ? i : -1;
     }
     return;
   }
-
-  // 1. The bin that holds the k-th largest key: thread t reads bins
-  //    8u .. 8u+7, u = 511 - t, so the prefix in thread order counts higher bins.
+  if (s0 >= n) return;  // chunk past the row's end (chunk 0 never is)
+  const int s1 = min(n, s0 + P.chunk);
+  // The bin of the k-th largest key: the prefix in thread order counts the
+  // keys in higher bins.
   {
-    const int u = kHThreads - 1 - tid;
-    int cb[8];
-    int tot = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cb[j] = __ldcg(gh + 8 * u + j);
-      tot += cb[j];
-    }
     int total;
     int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
     if (above < k && k <= above + tot) {
@@ -462,206 +513,280 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_hist_kernel(const HistParam
         above += cb[j];
       }
     }
+    if (tid == 0) {
+      s_ngt = 0;
+      s_nc = 0;
+    }
     __syncthreads();
   }
   const uint32_t bstar = static_cast<uint32_t>(s_bin);
   const int c_above = s_above, c_in = s_inbin;
-
-  // 2. One pass over this CTA's chunk: keys above the bin are selected, keys
-  //    in the bin become candidates.  Hits are staged in shared memory (the
-  //    finalize arrays, unused until then) and published with one global
-  //    reservation per list.
-  __shared__ int s_ngt, s_nc, s_gbase, s_cbase;
-  if (tid == 0) {
-    s_ngt = 0;
-    s_nc = 0;
+  if (R.c == 0 && tid == 0) {
+    R.cnt[0] = c_above;
+    R.cnt[2] = c_in > kCandMax;  // too many keys in the bin: whole-row fallback
   }
-  __syncthreads();
-  int* const st_gt = reinterpret_cast<int*>(tk);
-  if (c_in <= kCandMax) {
-    const int s0 = c * P.chunk, s1 = min(n, s0 + P.chunk);
-    const unsigned lt = (1u << lane) - 1u;
-    // All of the chunk's loads are issued before any is used.
-    constexpr int kPer = kCandMax / kHThreads;
-    uint32_t keys[kPer];
+  if (c_in > kCandMax) return;
+
+  const unsigned lt = (1u << lane) - 1u;
+  int* const fine = P.fine + static_cast<size_t>(R.r) * kFineBins;
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int s = s0 + j * kHThreads + tid;
-      keys[j] = s < s1 ? score_key(__ldcg(sc + s)) : 0u;
+  for (int j = 0; j < kPer; ++j) {
+    if (s0 + j * kHThreads >= s1) break;
+    const int s = s0 + j * kHThreads + tid;
+    const bool in = s < s1;
+    const uint32_t bin = keys[j] >> kHistShift;
+    const bool gt = in && bin > bstar;
+    const bool eq = in && bin == bstar;
+    const unsigned mg = __ballot_sync(0xffffffffu, gt);
+    const unsigned me = __ballot_sync(0xffffffffu, eq);
+    if (mg) {
+      int at = 0;
+      if (lane == 0) at = atomicAdd(&s_ngt, __popc(mg));
+      at = __shfl_sync(0xffffffffu, at, 0) + __popc(mg & lt);
+      if (gt && at < kSortMax) st_gt[at] = s;
     }
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (s0 + j * kHThreads >= s1) break;
-      const int s = s0 + j * kHThreads + tid;
-      const bool in = s < s1;
-      const uint32_t key = keys[j];
-      const uint32_t bin = key >> kHistShift;
-      const bool gt = in && bin > bstar;
-      const bool eq = in && bin == bstar;
-      const unsigned mg = __ballot_sync(0xffffffffu, gt);
-      const unsigned me = __ballot_sync(0xffffffffu, eq);
-      if (mg) {
-        int at = 0;
-        if (lane == 0) at = atomicAdd(&s_ngt, __popc(mg));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(mg & lt);
-        if (gt) st_gt[at] = s;
-      }
-      if (me) {
-        int at = 0;
-        if (lane == 0) at = atomicAdd(&s_nc, __popc(me));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(me & lt);
-        if (eq) {
-          ck[at] = key;
-          cp[at] = s;
+    if (me) {
+      int at = 0;
+      if (lane == 0) at = atomicAdd(&s_nc, __popc(me));
+      at = __shfl_sync(0xffffffffu, at, 0) + __popc(me & lt);
+      if (eq) {
+        atomicAdd(fine + ((keys[j] >> kFineShift) & (kFineBins - 1)), 1);
+        if (at < kCandMax) {
+          st_ck[at] = keys[j];
+          st_cp[at] = s;
         }
       }
     }
-    __syncthreads();
+  }
+  __syncthreads();
+  if (tid == 0) s_cbase = atomicAdd(&R.cnt[1], s_nc);
+  __syncthreads();
+  const int ngt = min(s_ngt, k);
+  int* const cg = P.chunk_gt + (static_cast<size_t>(R.r) * P.chunks + R.c) * k;
+  for (int i = tid; i < ngt; i += kHThreads) cg[i] = st_gt[i];
+  if (tid == 0) P.chunk_ngt[static_cast<size_t>(R.r) * P.chunks + R.c] = ngt;
+  for (int i = tid; i < s_nc; i += kHThreads) {
+    const int slot = s_cbase + i;
+    if (slot < kCandMax) {
+      P.cand_key[static_cast<size_t>(R.r) * kCandMax + slot] = st_ck[i];
+      P.cand_pos[static_cast<size_t>(R.r) * kCandMax + slot] = st_cp[i];
+    }
+  }
+}
+
+// Emit: from the row's sub-histogram every CTA of the row finds the sub-bin
+// holding the k-th largest key (the same, redundantly, in parallel) and
+// ranks the few candidates inside it exactly (score desc, position asc);
+// then it counts the selected candidates of earlier chunks and writes its
+// own chunk's selected positions, sorted, after those of earlier chunks.
+constexpr int kMaxChunks = 512;
+constexpr int kMemberMax = 2048;  // keys of the sub-bin ranked in shared memory
+constexpr int kRankDirect = 64;   // up to this many, by pairwise comparison
+__global__ void __launch_bounds__(kHThreads, 2) topk_emit_kernel(const HistParams P) {
+  __shared__ uint32_t mk[kMemberMax];  // sub-bin keys
+  __shared__ int mp[kMemberMax];       // their positions
+  __shared__ uint32_t tk[kMemberMax];  // tie keys for the position cut
+  __shared__ uint8_t mkeep[kMemberMax];
+  __shared__ int fin[kSortMax];        // this chunk's selected positions
+  __shared__ int hist[2048];
+  __shared__ int buf[kHWarps + 1];
+  __shared__ int s_b2, s_above2, s_c2, s_nm, s_nown;
+
+  pdl_wait();
+  pdl_launch_dependents();
+  const int tid = threadIdx.x;
+  const HistRow R = hist_row(P);
+  const int k = P.top_k;
+  // Everything the first decisions need, loaded at once: the row's counters
+  // (keys above the bin, candidates, fallback flag, causal length), the
+  // per-chunk counts of positions above the bin, and the sub-histogram.
+  const int4 cn = __ldcg(reinterpret_cast<const int4*>(R.cnt));
+  const int* const ngt = P.chunk_ngt + static_cast<size_t>(R.r) * P.chunks;
+  const int own_gt_raw = __ldcg(ngt + R.c);
+  int gt_before = tid < R.c ? __ldcg(ngt + tid) : 0;  // chunks <= kMaxChunks = threads
+  const int4 f = __ldcg(reinterpret_cast<const int4*>(P.fine + static_cast<size_t>(R.r) *
+                                                                   kFineBins) +
+                        (kHThreads - 1 - tid));
+  const int c_above = cn.x, c_in = cn.y, fallback = cn.z, n = cn.w;
+  if (n <= k || R.c * P.chunk >= n) return;
+  if (fallback != 0) {  // heavily tied scores: whole-row selection by one CTA
+    if (R.c == 0) row_select_global<kHWarps>(R.sc, n, k, R.out, hist, buf);
+    return;
+  }
+  const int own_gt = min(own_gt_raw, k);
+  constexpr int kPer = kCandMax / kHThreads;
+  uint32_t ck[kPer];
+  int cp[kPer];
+  const uint32_t* const gk = P.cand_key + static_cast<size_t>(R.r) * kCandMax;
+  const int* const gp = P.cand_pos + static_cast<size_t>(R.r) * kCandMax;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = j * kHThreads + tid;
+    ck[j] = i < c_in ? __ldcg(gk + i) : 0u;
+    cp[j] = i < c_in ? __ldcg(gp + i) : 0;
+  }
+  const int* const cg = P.chunk_gt + (static_cast<size_t>(R.r) * P.chunks + R.c) * k;
+  const int gt_mine = tid < own_gt ? __ldcg(cg + tid) : 0;  // the first two of up to four rounds
+  const int gt_mine2 = tid + kHThreads < own_gt ? __ldcg(cg + tid + kHThreads) : 0;
+  // Sub-bin of the k-th largest key; thread t reads sub-bins 4u .. 4u+3, u = 511 - t.
+  const int need = k - c_above;  // candidates to keep, 1 <= need <= c_in
+  {
+    const int tot = f.x + f.y + f.z + f.w;
+    int total;
+    const int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
+    const int u = kHThreads - 1 - tid;
+    if (above < need && need <= above + tot) {
+      if (above + f.w >= need) {
+        s_b2 = 4 * u + 3; s_above2 = above; s_c2 = f.w;
+      } else if (above + f.w + f.z >= need) {
+        s_b2 = 4 * u + 2; s_above2 = above + f.w; s_c2 = f.z;
+      } else if (above + f.w + f.z + f.y >= need) {
+        s_b2 = 4 * u + 1; s_above2 = above + f.w + f.z; s_c2 = f.y;
+      } else {
+        s_b2 = 4 * u; s_above2 = above + f.w + f.z + f.y; s_c2 = f.x;
+      }
+    }
     if (tid == 0) {
-      s_gbase = atomicAdd(&cnt[0], s_ngt);
-      s_cbase = atomicAdd(&cnt[1], s_nc);
+      s_nm = 0;
+      s_nown = 0;
     }
     __syncthreads();
-    for (int i = tid; i < s_ngt; i += kHThreads) {
-      const int slot = s_gbase + i;
-      if (slot < k) P.gt_list[static_cast<size_t>(r) * k + slot] = st_gt[i];
-    }
-    for (int i = tid; i < s_nc; i += kHThreads) {
-      const int slot = s_cbase + i;
-      if (slot < kCandMax) {
-        P.cand_key[static_cast<size_t>(r) * kCandMax + slot] = ck[i];
-        P.cand_pos[static_cast<size_t>(r) * kCandMax + slot] = cp[i];
+  }
+  const uint32_t b2 = static_cast<uint32_t>(s_b2);
+  const int need2 = need - s_above2;  // members of the sub-bin to keep, 1 <= need2 <= c2
+  if (s_c2 > kMemberMax) {            // every CTA of the row sees the same count
+    if (R.c == 0) row_select_global<kHWarps>(R.sc, n, k, R.out, hist, buf);
+    return;
+  }
+  const int lo = R.c * P.chunk, hi = lo + P.chunk;
+  int before = gt_before;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (j * kHThreads >= c_in) break;
+    if (j * kHThreads + tid >= c_in) continue;
+    const uint32_t sub = (ck[j] >> kFineShift) & (kFineBins - 1);
+    if (sub > b2) {
+      before += cp[j] < lo;
+      if (cp[j] >= lo && cp[j] < hi) {
+        const int at = atomicAdd(&s_nown, 1);
+        if (at < kSortMax) fin[at] = cp[j];
+      }
+    } else if (sub == b2) {
+      const int at = atomicAdd(&s_nm, 1);
+      if (at < kMemberMax) {
+        mk[at] = ck[j];
+        mp[at] = cp[j];
       }
     }
   }
-
-  // 3. The last CTA of the row to arrive finishes it (nobody waits).
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&cnt[2], 1) == P.chunks - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  if (c_in > kCandMax) {
-    // Too many keys share the threshold bin (heavily tied scores): exact
-    // selection over the whole row instead.
-    row_select_global<kHWarps>(sc, n, k, out, hist, buf);
+  const int nm = min(s_nm, kMemberMax);  // == c2
+  if (need2 >= nm) {
+    for (int i = tid; i < nm; i += kHThreads) mkeep[i] = 1;
+  } else if (nm <= kRankDirect) {
+    for (int i = tid; i < nm; i += kHThreads) {
+      int rank = 0;
+      for (int j = 0; j < nm; ++j) {
+        rank += mk[j] > mk[i] || (mk[j] == mk[i] && mp[j] < mp[i]);
+      }
+      mkeep[i] = rank < need2;
+    }
   } else {
-    const int need = k - c_above;  // candidates to keep, 1 <= need <= c_in
-    for (int i = tid; i < c_in; i += kHThreads) {
-      ck[i] = __ldcg(P.cand_key + static_cast<size_t>(r) * kCandMax + i);
-      cp[i] = __ldcg(P.cand_pos + static_cast<size_t>(r) * kCandMax + i);
-    }
-    for (int i = tid; i < c_above && i < k; i += kHThreads) {
-      fin[i] = __ldcg(P.gt_list + static_cast<size_t>(r) * k + i);
-    }
-    if (tid == 0) s_nfin = c_above;
-    __syncthreads();
-    // Exact threshold among the candidates (their top 12 bits are bstar).
+    const uint32_t known_mask = ~((1u << kFineShift) - 1u);
     uint32_t theta;
     int need_eq;
-    smem_select(ck, c_in, need, 0, kHistShift - 1, bstar << kHistShift,
-                ~((1u << kHistShift) - 1u), hist, buf, theta, need_eq);
-    // Ties at theta: keep the need_eq lowest positions (largest ~position).
+    smem_select(mk, nm, need2, 0, kFineShift - 1, mk[0] & known_mask, known_mask, hist, buf,
+                theta, need_eq);
     int n_tie = 0;
-    for (int i = tid; i < c_in; i += kHThreads) n_tie += ck[i] == theta;
+    for (int i = tid; i < nm; i += kHThreads) n_tie += mk[i] == theta;
     int total_tie;
     block_excl_sum_nw<kHWarps>(n_tie, buf, total_tie);
+    uint32_t pos_cut = 0u;  // ties kept: ~position >= pos_cut (the lowest positions)
     const bool cut_ties = need_eq < total_tie;
-    uint32_t pos_cut = 0u;
     if (cut_ties) {
-      for (int i = tid; i < c_in; i += kHThreads) {
-        tk[i] = ck[i] == theta ? ~static_cast<uint32_t>(cp[i]) : 0u;  // 0: not a tie
+      for (int i = tid; i < nm; i += kHThreads) {
+        tk[i] = mk[i] == theta ? ~static_cast<uint32_t>(mp[i]) : 0u;
       }
       __syncthreads();
       int unique;
-      smem_select(tk, c_in, need_eq, 0, 31, 0u, 0u, hist, buf, pos_cut, unique);
+      smem_select(tk, nm, need_eq, 0, 31, 0u, 0u, hist, buf, pos_cut, unique);
     }
-    if (n <= kBitmapMax) {
-      // Ascending order from a bitmap of the kept positions: mark them, then
-      // each thread emits the set bits of its run of words after a prefix sum.
-      uint32_t* const bm = tk;
-      const int words = (n + 31) >> 5;
-      __syncthreads();
-      for (int i = tid; i < words; i += kHThreads) bm[i] = 0u;
-      __syncthreads();
-      for (int i = tid; i < c_above && i < k; i += kHThreads) {
-        const int pos = fin[i];
-        atomicOr(&bm[pos >> 5], 1u << (pos & 31));
+    for (int i = tid; i < nm; i += kHThreads) {
+      mkeep[i] = mk[i] > theta ||
+                 (mk[i] == theta && (!cut_ties || ~static_cast<uint32_t>(mp[i]) >= pos_cut));
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < nm; i += kHThreads) {
+    if (mkeep[i]) {
+      before += mp[i] < lo;
+      if (mp[i] >= lo && mp[i] < hi) {
+        const int at = atomicAdd(&s_nown, 1);
+        if (at < kSortMax) fin[at] = mp[i];
       }
-      for (int i = tid; i < c_in; i += kHThreads) {
-        const uint32_t key = ck[i];
-        const bool keep = key > theta ||
-                          (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
-        if (keep) atomicOr(&bm[cp[i] >> 5], 1u << (cp[i] & 31));
-      }
-      __syncthreads();
-      const int per = (words + kHThreads - 1) / kHThreads;
-      const int w0 = tid * per, w1 = min(words, w0 + per);
-      int mine = 0;
-      for (int wi = w0; wi < w1; ++wi) mine += __popc(bm[wi]);
-      int total;
-      int at = block_excl_sum_nw<kHWarps>(mine, buf, total);
-      for (int wi = w0; wi < w1; ++wi) {
-        uint32_t bits = bm[wi];
-        while (bits != 0u) {
-          const int bit = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          if (at < k) out[at] = (wi << 5) + bit;
-          ++at;
-        }
-      }
-    } else {
-      // Long rows: append the kept candidates and sort the k positions.
-      for (int base = 0; base < c_in; base += kHThreads) {
-        const int i = base + tid;
-        bool keep = false;
-        if (i < c_in) {
-          const uint32_t key = ck[i];
-          keep = key > theta ||
-                 (key == theta && (!cut_ties || ~static_cast<uint32_t>(cp[i]) >= pos_cut));
-        }
-        int tot_keep;
-        const int slot = s_nfin + block_excl_count_nw<kHWarps>(keep, buf, tot_keep);
-        if (keep && slot < kSortMax) fin[slot] = cp[i];
-        __syncthreads();
-        if (tid == 0) s_nfin += tot_keep;
-        __syncthreads();
-      }
-      for (int i = k + tid; i < kSortMax; i += kHThreads) fin[i] = 0x7FFFFFFF;
-      __syncthreads();
-      for (int size = 2; size <= kSortMax; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int i = tid; i < kSortMax; i += kHThreads) {
-            const int j = i ^ stride;
-            if (j > i) {
-              const int a = fin[i], bb = fin[j];
-              const bool up = (i & size) == 0;
-              if ((a > bb) == up) {
-                fin[i] = bb;
-                fin[j] = a;
-              }
-            }
+    }
+  }
+  int offset;
+  block_excl_sum_nw<kHWarps>(before, buf, offset);  // total: selections in earlier chunks
+  const int n_cand_own = min(s_nown, kSortMax);
+  const int m = min(n_cand_own + own_gt, kSortMax);
+  if (tid + n_cand_own < m) fin[n_cand_own + tid] = gt_mine;
+  if (tid + kHThreads + n_cand_own < m) fin[n_cand_own + kHThreads + tid] = gt_mine2;
+  for (int i = tid + 2 * kHThreads; i + n_cand_own < m; i += kHThreads) {
+    fin[n_cand_own + i] = __ldcg(cg + i);
+  }
+  int size = 1;
+  while (size < m) size <<= 1;
+  for (int i = m + tid; i < size; i += kHThreads) fin[i] = 0x7FFFFFFF;
+  __syncthreads();
+  for (int sz = 2; sz <= size; sz <<= 1) {  // ascending bitonic sort of the m positions
+    for (int stride = sz >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < size; i += kHThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const int a = fin[i], bb = fin[j];
+          const bool up = (i & sz) == 0;
+          if ((a > bb) == up) {
+            fin[i] = bb;
+            fin[j] = a;
           }
-          __syncthreads();
         }
       }
-      for (int i = tid; i < k; i += kHThreads) out[i] = fin[i];
+      __syncthreads();
     }
+  }
+  for (int i = tid; i < m; i += kHThreads) {
+    if (offset + i < k) R.out[offset + i] = fin[i];
   }
 }
 
 }  // namespace
 
-size_t topk_hist_zero_bytes(int Nq) {
-  return static_cast<size_t>(Nq) * (kHistBins + 4) * sizeof(int);
+int topk_hist_chunks(int Nq, int64_t max_len, int* chunk_len) {
+  // About two CTAs per SM of a 148-SM part in all, chunks of whole 512-key
+  // blocks, at most kCandMax keys (the shared staging arrays) per chunk.
+  int chunks = std::max(1, 2 * 148 / std::max(1, Nq));
+  int chunk = static_cast<int>(((max_len + chunks - 1) / chunks + kHThreads - 1) / kHThreads *
+                               kHThreads);
+  chunk = std::max(kHThreads, std::min(chunk, kCandMax));
+  chunks = static_cast<int>((max_len + chunk - 1) / chunk);
+  if (chunk_len) *chunk_len = chunk;
+  return chunks;
 }
 
-size_t topk_hist_ws_bytes(int Nq, int top_k) {
+bool topk_hist_supported(int Nq, int64_t max_len) {
+  return topk_hist_chunks(Nq, max_len, nullptr) <= kMaxChunks;
+}
+
+size_t topk_hist_zero_bytes(int Nq) {
+  return static_cast<size_t>(Nq) * (kHistBins + kFineBins + 4) * sizeof(int);
+}
+
+size_t topk_hist_ws_bytes(int Nq, int top_k, int64_t max_len) {
+  const int chunks = topk_hist_chunks(Nq, max_len, nullptr);
   return topk_hist_zero_bytes(Nq) +
-         static_cast<size_t>(Nq) * (kCandMax * (sizeof(uint32_t) + sizeof(int)) +
-                                    top_k * sizeof(int));
+         static_cast<size_t>(Nq) * (kCandMax * (sizeof(uint32_t) + sizeof(int))) +
+         static_cast<size_t>(Nq) * chunks * (static_cast<size_t>(top_k) + 1) * sizeof(int);
 }
 
 cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream) {
@@ -674,29 +799,28 @@ cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t st
   P.idx = a.idx;
   P.B = a.B;
   P.top_k = a.top_k;
+  P.chunks = topk_hist_chunks(a.Nq, a.max_len, &P.chunk);
   uint8_t* p = static_cast<uint8_t*>(ws_region);
   P.hist = reinterpret_cast<int*>(p);
   p += static_cast<size_t>(a.Nq) * kHistBins * sizeof(int);
+  P.fine = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * kFineBins * sizeof(int);
   P.counters = reinterpret_cast<int*>(p);
   p += static_cast<size_t>(a.Nq) * 4 * sizeof(int);
   P.cand_key = reinterpret_cast<uint32_t*>(p);
   p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(uint32_t);
   P.cand_pos = reinterpret_cast<int*>(p);
   p += static_cast<size_t>(a.Nq) * kCandMax * sizeof(int);
-  P.gt_list = reinterpret_cast<int*>(p);
-  // About two CTAs per SM in total, chunks of whole 512-key blocks.
-  const long long target = 2LL * a.num_sms;
-  P.chunks = static_cast<int>(std::max<long long>(1, target / std::max(1, a.Nq)));
-  P.chunk = static_cast<int>(((a.max_len + P.chunks - 1) / P.chunks + kHThreads - 1) /
-                             kHThreads * kHThreads);
-  // A chunk's hits are staged in shared arrays of kCandMax entries.
-  P.chunk = std::min(P.chunk, kCandMax);
-  P.chunks = static_cast<int>((a.max_len + P.chunk - 1) / P.chunk);
-  const size_t smem = static_cast<size_t>(kCandMax) * 12 + (kSortMax + 2048) * sizeof(int);
-  cudaError_t e = ensure_smem_limit<topk_hist_kernel>(static_cast<int>(smem));
+  P.chunk_gt = reinterpret_cast<int*>(p);
+  p += static_cast<size_t>(a.Nq) * P.chunks * a.top_k * sizeof(int);
+  P.chunk_ngt = reinterpret_cast<int*>(p);
+  const size_t smem_f = static_cast<size_t>(kSortMax) * 4 + static_cast<size_t>(kCandMax) * 8;
+  cudaError_t e = ensure_smem_limit<topk_filter_kernel>(static_cast<int>(smem_f));
   if (e != cudaSuccess) return e;
-  return launch_pdl(topk_hist_kernel, dim3(static_cast<unsigned>(a.Nq) * P.chunks),
-                    dim3(kHThreads), smem, stream, 0, P);
+  const dim3 grid(static_cast<unsigned>(a.Nq) * P.chunks);
+  e = launch_pdl(topk_filter_kernel, grid, dim3(kHThreads), smem_f, stream, 0, P);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_emit_kernel, grid, dim3(kHThreads), 0, stream, 0, P);
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
