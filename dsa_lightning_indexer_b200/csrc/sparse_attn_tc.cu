@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp == 4) {
     // ------------------------------------------------ Q load + MMA issue --
+    // The whole warp runs the loop (waits and descriptor arithmetic stay
+    // warp-uniform); one elected lane issues each MMA and commit.
     if (lane == 0) {
       tma_prefetch_map(&qmap);
       mbar_arrive_expect_tx(b_qfull, kBoxes * kQBox);
@@ -277,48 +279,61 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       for (int j = 0; j < kBoxes; ++j) {
         tma_load_2d(sQ + j * kQBox, &qmap, b_qfull, 64 * j, r * P.H + h0, pol);
       }
-      bool ok = mbar_wait(b_qfull, 0, P.err);
-      auto issue_pv = [&](int u) -> bool {
-        const int st = u & 1;
-        const uint32_t ph = static_cast<uint32_t>((u >> 1) & 1);
-        if (!mbar_wait(b_pfull(st), ph, P.err)) return false;
-        tc_fence_after();
-        const uint32_t kvs = sKV + st * kKVStage;
-        const uint32_t phi = sP + (2 * st) * kPBuf, plo = phi + kPBuf;
-#pragma unroll
-        for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll
-          for (int kk = 0; kk < kT / 16; ++kk) {
-            const uint64_t a = sdesc_sw128_mn(kvs + (2 * blk) * kKVBox + kk * 2048, kKVBox);
-            const uint32_t d = tmem + kColO + 64u * blk;
-            tc_mma_bf16(d, a, sdesc_sw128(phi + kk * 32), kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_bf16(d, a, sdesc_sw128(plo + kk * 32), kIdescPV, 1u);
-          }
-        }
-        tc_commit(b_kvempty(st));
-        tc_commit(b_pempty(st));
-        tc_commit(b_odone);
-        return true;
-      };
-      for (int t = 0; t < n_tiles && ok; ++t) {
-        const int st = t & 1;
-        const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
-        ok = mbar_wait(b_kvfull(st), ph, P.err) && mbar_wait(b_sempty(st), ph ^ 1u, P.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t kvs = sKV + st * kKVStage;
-        const uint32_t d = tmem + kColS + 64u * st;
-#pragma unroll 4
-        for (int ks = 0; ks < kLatent / 16; ++ks) {
-          const uint32_t off = (ks & 3) * 32;
-          tc_mma_bf16(d, sdesc_sw128(sQ + (ks >> 2) * kQBox + off),
-                      sdesc_sw128(kvs + (ks >> 2) * kKVBox + off), kIdescS, ks > 0 ? 1u : 0u);
-        }
-        tc_commit(b_sfull(st));
-        if (t > 0) ok = issue_pv(t - 1);
-      }
-      if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
     }
+    __syncwarp();
+    // Descriptors of the first K slice of each operand; later slices add
+    // their byte offset / 16 to the address field.
+    const uint64_t dq = sdesc_sw128(sQ);
+    const uint64_t dkv0 = sdesc_sw128(sKV);
+    const uint64_t dv0 = sdesc_sw128_mn(sKV, kKVBox);
+    const uint64_t dp0 = sdesc_sw128(sP);
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, P.err));
+    };
+    bool ok = wait_all(b_qfull, 0);
+    auto issue_pv = [&](int u) -> bool {
+      const int st = u & 1;
+      const uint32_t ph = static_cast<uint32_t>((u >> 1) & 1);
+      if (!wait_all(b_pfull(st), ph)) return false;
+      tc_fence_after();
+      const uint64_t dv = dv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
+      const uint64_t dhi = dp0 + static_cast<uint64_t>((2 * st * kPBuf) >> 4);
+      const uint64_t dlo = dhi + static_cast<uint64_t>(kPBuf >> 4);
+#pragma unroll
+      for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+        for (int kk = 0; kk < kT / 16; ++kk) {
+          const uint64_t a = dv + static_cast<uint64_t>(((2 * blk) * kKVBox + kk * 2048) >> 4);
+          const uint32_t d = tmem + kColO + 64u * blk;
+          const uint64_t ko = static_cast<uint64_t>((kk * 32) >> 4);
+          tc_mma_bf16_warp(d, a, dhi + ko, kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_warp(d, a, dlo + ko, kIdescPV, 1u);
+        }
+      }
+      tc_commit_warp(b_kvempty(st));
+      tc_commit_warp(b_pempty(st));
+      tc_commit_warp(b_odone);
+      return true;
+    };
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      const int st = t & 1;
+      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      ok = wait_all(b_kvfull(st), ph) && wait_all(b_sempty(st), ph ^ 1u);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t dk = dkv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
+      const uint32_t d = tmem + kColS + 64u * st;
+#pragma unroll
+      for (int ks = 0; ks < kLatent / 16; ++ks) {
+        const uint32_t off = (ks & 3) * 32;
+        tc_mma_bf16_warp(d, dq + static_cast<uint64_t>(((ks >> 2) * kQBox + off) >> 4),
+                         dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4), kIdescS,
+                         ks > 0 ? 1u : 0u);
+      }
+      tc_commit_warp(b_sfull(st));
+      if (t > 0) ok = issue_pv(t - 1);
+    }
+    if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
   } else {
     // ----------------------------------------------------------- softmax --
     const int q = warp;                          // TMEM lane quadrant
