@@ -94,14 +94,35 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo)
   return d;
 }
 
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+// 16x32bx2 shape: threads 0-15 read TMEM lanes base..base+15 at the given
+// column, threads 16-31 the same lanes kSplitCols columns further.  With the
+// M = 64 accumulator layout (head row 16q + j at lane 32q + j) the two half
+// warps split each head row's tile of logits between them.
+constexpr int kSplitCols = kT / 2;
+static_assert(kSplitCols == 24, "the logit loads below cover 16 + 8 columns per half warp");
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16], %17;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+      : "r"(taddr), "n"(kSplitCols));
+}
+
+__device__ __forceinline__ void tmem_ld_16x32bx2_x8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr), "n"(kSplitCols));
+}
+
+// 2^x on the special-function unit (relative error about 2^-22); 2^-inf = 0.
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -291,11 +312,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, P.err));
     };
     bool ok = wait_all(b_qfull, 0);
-    auto issue_pv = [&](int u) -> bool {
+    auto issue_pv = [&](int u) {
       const int st = u & 1;
-      const uint32_t ph = static_cast<uint32_t>((u >> 1) & 1);
-      if (!wait_all(b_pfull(st), ph)) return false;
-      tc_fence_after();
       const uint64_t dv = dv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
       const uint64_t dhi = dp0 + static_cast<uint64_t>((2 * st * kPBuf) >> 4);
       const uint64_t dlo = dhi + static_cast<uint64_t>(kPBuf >> 4);
@@ -313,12 +331,36 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tc_commit_warp(b_kvempty(st));
       tc_commit_warp(b_pempty(st));
       tc_commit_warp(b_odone);
-      return true;
+    };
+    auto p_ready = [&](int u) {
+      return mbar_try_wait(b_pfull(u & 1), static_cast<uint32_t>((u >> 1) & 1));
     };
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int st = t & 1;
       const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
-      ok = wait_all(b_kvfull(st), ph) && wait_all(b_sempty(st), ph ^ 1u);
+      // While tile t's rows are still arriving, issue the previous tile's
+      // P.V as soon as its P is ready: that frees its gather stage early.
+      bool pv_pending = t > 0;
+      const long long w0 = clock64();
+      for (unsigned it = 1;; ++it) {
+        if (pv_pending && __all_sync(0xffffffffu, p_ready(t - 1))) {
+          tc_fence_after();
+          issue_pv(t - 1);
+          pv_pending = false;
+        }
+        if (__all_sync(0xffffffffu, mbar_try_wait(b_kvfull(st), ph) &&
+                                        mbar_try_wait(b_sempty(st), ph ^ 1u))) {
+          break;
+        }
+        if ((it & 63u) == 0u) {
+          const bool late = clock64() - w0 > kWaitCycles;
+          if (__any_sync(0xffffffffu, late || *reinterpret_cast<volatile unsigned*>(P.err) != 0u)) {
+            if (lane == 0 && late) atomicOr(P.err, kErrTimeout);
+            ok = false;
+            break;
+          }
+        }
+      }
       if (!ok) break;
       tc_fence_after();
       const uint64_t dk = dkv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
@@ -331,9 +373,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                          ks > 0 ? 1u : 0u);
       }
       tc_commit_warp(b_sfull(st));
-      if (t > 0) ok = issue_pv(t - 1);
+      if (pv_pending) {
+        ok = wait_all(b_pfull((t - 1) & 1), static_cast<uint32_t>(((t - 1) >> 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(t - 1);
+      }
     }
-    if (ok && n_tiles > 0) issue_pv(n_tiles - 1);
+    if (ok && n_tiles > 0 &&
+        wait_all(b_pfull((n_tiles - 1) & 1), static_cast<uint32_t>(((n_tiles - 1) >> 1) & 1))) {
+      tc_fence_after();
+      issue_pv(n_tiles - 1);
+    }
   } else {
     // ----------------------------------------------------------- softmax --
     const int q = warp;                          // TMEM lane quadrant
@@ -348,9 +399,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       ok = mbar_wait(b_sfull(st), ph, P.err);
       if (!ok) break;
       tc_fence_after();
-      uint32_t va[32], vb[16];
-      tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64u * st, va);
-      tmem_ld_32x32b_x16(tmem + lane_base + kColS + 64u * st + 32u, vb);
+      // This thread's half of its head row: keys k0 .. k0 + 23 of the tile.
+      uint32_t va[16], vb[8];
+      const uint32_t sa = tmem + lane_base + kColS + 64u * st;
+      tmem_ld_16x32bx2_x16(sa, va);
+      tmem_ld_16x32bx2_x8(sa + 16u, vb);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(b_sempty(st));
@@ -358,49 +411,55 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       ok = mbar_wait(b_kvfull(st), ph, P.err);
       if (!ok) break;
       // Logits in base 2; unused slots masked.
-      float s[kT];
       const int* const ti = tidx + st * kT;
+      const unsigned v_lo = __ballot_sync(0xffffffffu, ti[lane] >= 0);
+      const unsigned v_hi = __ballot_sync(0xffffffffu, lane < kT - 32 && ti[32 + lane] >= 0);
+      const int k0 = (lane >> 4) * kSplitCols;
+      const unsigned long long valid =
+          ((static_cast<unsigned long long>(v_hi) << 32) | v_lo) >> k0;
+      float s[kSplitCols];
       float tmax = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < kT; ++k) {
-        const float raw_s = __uint_as_float(k < 32 ? va[k] : vb[k - 32]);
-        s[k] = ti[k] >= 0 ? raw_s * P.scale_log2 : -INFINITY;
+      for (int k = 0; k < kSplitCols; ++k) {
+        const float raw_s = __uint_as_float(k < 16 ? va[k] : vb[k - 16]);
+        s[k] = ((valid >> k) & 1ull) ? raw_s * P.scale_log2 : -INFINITY;
         tmax = fmaxf(tmax, s[k]);
       }
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
       const bool raise = tmax > m_run + kRescaleLog2 || (m_run == -INFINITY && tmax > -INFINITY);
       const float m_new = raise ? tmax : m_run;
-      const float alpha = raise ? exp2f(m_run - m_new) : 1.f;
+      const float alpha = raise ? exp2_fast(m_run - m_new) : 1.f;
+      const float m_ref = m_new == -INFINITY ? 0.f : m_new;  // masked logits give 2^-inf = 0
       float sum = 0.f;
-      uint32_t hi[kT / 2], lo[kT / 2];
+      uint32_t hi[kSplitCols / 2], lo[kSplitCols / 2];
 #pragma unroll
-      for (int k = 0; k < kT; k += 2) {
-        const float p0 = s[k] == -INFINITY ? 0.f : exp2f(s[k] - m_new);
-        const float p1 = s[k + 1] == -INFINITY ? 0.f : exp2f(s[k + 1] - m_new);
+      for (int k = 0; k < kSplitCols; k += 2) {
+        const float p0 = exp2_fast(s[k] - m_ref);
+        const float p1 = exp2_fast(s[k + 1] - m_ref);
         sum += p0 + p1;
         const uint32_t h2 = pack2_bf16(p0, p1);
-        const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&h2);
         hi[k / 2] = h2;
-        lo[k / 2] = pack2_bf16(p0 - __low2float(hb), p1 - __high2float(hb));
+        lo[k / 2] = pack2_bf16(p0 - __uint_as_float(h2 << 16), p1 - __uint_as_float(h2 & 0xFFFF0000u));
       }
-      if (owner) {
-        l_run = l_run * alpha + sum;
-        m_run = m_new;
-        alpha_s[hl] = alpha;
-      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+      if (owner) alpha_s[hl] = alpha;
       // P buffer `st` is free once the P.V of tile t-2 has completed.
       ok = mbar_wait(b_pempty(st), ph ^ 1u, P.err);
       if (!ok) break;
-      if (owner) {
+      {
         const uint32_t prow_hi = sP + (2 * st) * kPBuf + hl * 128;
         const uint32_t prow_lo = prow_hi + kPBuf;
 #pragma unroll
-        for (int c = 0; c < kT / 8; ++c) {
+        for (int j = 0; j < kSplitCols / 8; ++j) {
+          const int c = k0 / 8 + j;
           const uint32_t off = static_cast<uint32_t>((c ^ (hl & 7)) << 4);
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_hi + off),
-                       "r"(hi[4 * c]), "r"(hi[4 * c + 1]), "r"(hi[4 * c + 2]), "r"(hi[4 * c + 3])
+                       "r"(hi[4 * j]), "r"(hi[4 * j + 1]), "r"(hi[4 * j + 2]), "r"(hi[4 * j + 3])
                        : "memory");
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_lo + off),
-                       "r"(lo[4 * c]), "r"(lo[4 * c + 1]), "r"(lo[4 * c + 2]), "r"(lo[4 * c + 3])
+                       "r"(lo[4 * j]), "r"(lo[4 * j + 1]), "r"(lo[4 * j + 2]), "r"(lo[4 * j + 3])
                        : "memory");
         }
       }
