@@ -256,16 +256,34 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
     const int gt = threadIdx.x - (5 + 2 * grp) * 32;
     int* const gidx = tidx + grp * kT;
+    // Positions of tile t's rows (thread gt < kT holds one), loaded and the
+    // rows prefetched into L2 a tile ahead of their copy.
+    auto load_pos = [&](int t) -> int {
+      if (gt >= kT || t >= n_tiles) return -1;
+      const int slot = slot_lo + t * kT + gt;
+      return slot < slot_hi ? __ldg(idx_row + slot) : -1;
+    };
+    auto prefetch_row = [&](int pos) {
+      if (pos >= 0) {
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                         P.kv + static_cast<size_t>(kv0 + pos) * kLatent),
+                     "r"(kLatent * 2)
+                     : "memory");
+      }
+    };
+    int pos_cur = load_pos(grp);
+    int pos_nxt = load_pos(grp + 2);
+    prefetch_row(pos_cur);
     bool ok = true;
     for (int t = grp; t < n_tiles && ok; t += 2) {
+      prefetch_row(pos_nxt);
       const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
-      if (gt < kT) {
-        const int slot = slot_lo + t * kT + gt;
-        gidx[gt] = slot < slot_hi ? __ldg(idx_row + slot) : -1;
-      }
+      if (gt < kT) gidx[gt] = pos_cur;
       named_bar_sync(2 + grp, kGroupThreads);
+      pos_cur = pos_nxt;
+      pos_nxt = load_pos(t + 4);
       const uint32_t stage = sKV + grp * kKVStage;
       for (int item = gt; item < kT * kBoxes; item += kGroupThreads) {
         const int i = item / kBoxes, bx = item - i * kBoxes;
