@@ -29,7 +29,10 @@
  *    except the h_* fields of dsa_batch, which are HOST mirrors used to plan
  *    the launch without a device sync.  The library allocates nothing, keeps
  *    no state between calls and is re-entrant; calls on different streams
- *    must use different workspaces.
+ *    must use different workspaces.  A workspace must be zero-filled (e.g.
+ *    cudaMemset) before its first use: its first 256 bytes are a control
+ *    block holding the kernels' error word, which calls leave zero unless a
+ *    kernel-side failure sets it, and dsa_check_device_status clears.
  *  - Asynchrony: all work is enqueued on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream).  Nothing synchronises except
  *    dsa_check_device_status.

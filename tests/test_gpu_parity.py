@@ -317,3 +317,22 @@ def test_standalone_calls_between_layer_calls_leave_it_unchanged():
         assert np.array_equal(a, b)
     assert np.array_equal(idx.cpu().numpy(), first[2])
     bd.check_device_status(dw.ws)
+
+
+@pytest.mark.parametrize("make", [_hist_batch, lambda: synth.prefill(1024, 16, 256, seed=100),
+                                  lambda: synth.custom([5000, 777, 128, 129, 2], [1] * 5, 64, 128,
+                                                       seed=102)])
+def test_workspace_control_block_is_zero_after_calls(make):
+    """Calls leave the workspace's control block (the kernels' error word)
+    zero, so the next call and dsa_check_device_status start clean."""
+    wl = make()
+    dw = bd.DeviceWorkload(wl)
+    for _ in range(2):
+        dw.forward()
+        torch.cuda.synchronize()
+        assert not dw.ws[:256].any().item()
+    ld = _up4(wl.ctx_lens.max())
+    scores = torch.zeros(wl.Nq, ld, device="cuda")
+    bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws)
+    torch.cuda.synchronize()
+    assert not dw.ws[:256].any().item()
