@@ -21,6 +21,7 @@ import faulthandler
 import json
 import math
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -219,11 +220,44 @@ def indexer_causal_flops(wl):
 
 def launches_per_layer(wl, sms=148):
     """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
-    sequences with queries), the top-k selection, the sparse attention and,
-    when few rows split the selected set over CTAs, the merge of the slices."""
-    seqs = int((np.diff(wl.q_offsets) > 0).sum())
+    sequences with queries); the top-k selection, which is two kernels (filter
+    and emit) when few long single-query rows take the histogram path, else
+    one; the sparse attention and, when few rows split the selected set over
+    CTAs, the merge of the slices."""
+    nq = np.diff(wl.q_offsets)
+    seqs = int((nq > 0).sum())
+    max_len = int(wl.ctx_lens.max()) if wl.B else 0
+    chunks = max(1, 2 * 148 // max(1, wl.Nq))  # as the library plans it
+    per = -(-max_len // chunks)
+    chunk = min(max(512, -(-per // 512) * 512), 8192)
+    hist = (0 < wl.Nq <= 148 and max_len >= 8192 and max_len >= 4 * wl.top_k
+            and int(nq.max()) <= 1 and -(-max_len // chunk) <= 512)
     few_rows = wl.Nq * ((wl.H + 63) // 64) < sms
-    return (seqs + 63) // 64 + 1 + 1 + (1 if few_rows and wl.top_k > 16 else 0)
+    return (seqs + 63) // 64 + (2 if hist else 1) + 1 + (1 if few_rows and wl.top_k > 16 else 0)
+
+
+def profiled_traffic(profile="profiles/decode_b4_128k_layer.md"):
+    """DRAM bytes per indexer launch from the committed ncu summary, or None
+    once the kernel's sources differ from the ones the counters were taken on."""
+    import hashlib
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), profile)
+    try:
+        text = open(path).read()
+        traffic = int(re.search(r"traffic_bytes:\s*(\d+)", text).group(1))
+        pins = re.search(r"source_sha256_prefix:\s*(.+)", text).group(1).split()
+    except (OSError, AttributeError, ValueError):
+        return None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "dsa_lightning_indexer_b200",
+                        "csrc")
+    for pin in pins:
+        name, _, prefix = pin.partition("=")
+        try:
+            digest = hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest()
+        except OSError:
+            return None
+        if not digest.startswith(prefix):
+            return None
+    return traffic
 
 
 def run_ours(args):
@@ -331,7 +365,7 @@ def run_ours(args):
                        "dsa_layer_forward"),
         "roofline": None if args.no_kernel_times else {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": None, "peak_source": peaks["source"],
+                     "traffic": profiled_traffic(), "peak_source": peaks["source"],
                      "algorithmic_bytes_per_launch": kb},
         "layer_roofline": {"algorithmic_bytes_per_step": db["total"],
                            "achieved_gbs": db["total"] / (ms_step * 1e-3) / 1e9,
