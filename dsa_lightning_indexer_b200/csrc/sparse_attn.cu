@@ -340,6 +340,17 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams P) {
   const int r = blockIdx.x, h = blockIdx.y;
   const size_t rec = static_cast<size_t>(r) * P.H + h;
   const size_t stride = static_cast<size_t>(P.Nq) * P.H;
+  // Every slice's part of this thread's 4 value dims is requested up front
+  // (up to kBatch slices), so the loads overlap the weights' computation.
+  constexpr int kBatch = 32;
+  const int dv = threadIdx.x * 4;
+  const float* const po = P.part_o + rec * kValue + dv;
+  float4 x[kBatch];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    x[j] = j < P.n_split ? __ldcg(reinterpret_cast<const float4*>(po + j * stride * kValue))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   if (threadIdx.x < 32) {
     float m[kMaxSplit / 32], l[kMaxSplit / 32];
     float M = -INFINITY;
@@ -370,17 +381,22 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(const AttnParams P) {
     }
   }
   __syncthreads();
-  const int dv = threadIdx.x * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* const po = P.part_o + rec * kValue + dv;
-#pragma unroll 8
-  for (int sp = 0; sp < P.n_split; ++sp) {
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j) {
+    const float w = j < P.n_split ? wgt[j] : 0.f;
+    acc.x = fmaf(w, x[j].x, acc.x);
+    acc.y = fmaf(w, x[j].y, acc.y);
+    acc.z = fmaf(w, x[j].z, acc.z);
+    acc.w = fmaf(w, x[j].w, acc.w);
+  }
+  for (int sp = kBatch; sp < P.n_split; ++sp) {
     const float w = wgt[sp];
-    const float4 x = __ldcg(reinterpret_cast<const float4*>(po + sp * stride * kValue));
-    acc.x = fmaf(w, x.x, acc.x);
-    acc.y = fmaf(w, x.y, acc.y);
-    acc.z = fmaf(w, x.z, acc.z);
-    acc.w = fmaf(w, x.w, acc.w);
+    const float4 y = __ldcg(reinterpret_cast<const float4*>(po + sp * stride * kValue));
+    acc.x = fmaf(w, y.x, acc.x);
+    acc.y = fmaf(w, y.y, acc.y);
+    acc.z = fmaf(w, y.z, acc.z);
+    acc.w = fmaf(w, y.w, acc.w);
   }
   const float inv = inv_total;
   *reinterpret_cast<float4*>(P.out + rec * kValue + dv) =

@@ -46,6 +46,7 @@ constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
 
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kBoxes * kQBox;
+constexpr int kOffStage = kOffQ;  // output staging [64][512] fp32 over Q and the gather stages
 constexpr int kOffP = kOffKV + 2 * kKVStage;           // [stage][hi, lo]
 constexpr int kOffBar = kOffP + 4 * kPBuf;
 constexpr int kNumBars = 14;
@@ -56,6 +57,7 @@ constexpr int kOffM = kOffAlpha + kHB * 4;              // [64] float
 constexpr int kOffL = kOffM + kHB * 4;                  // [64] float
 constexpr int kSmemUsed = kOffL + kHB * 4;
 constexpr int kSmemTc = kSmemUsed + 1024;               // alignment slack
+static_assert(kOffStage + kHB * kValue * 4 <= kOffP, "output staging overlaps the P buffers");
 static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
@@ -169,13 +171,34 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
   return res != 0;
 }
 
-__device__ __forceinline__ int owner_seq_tc(const int32_t* q_offsets, int B, int r) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (q_offsets[mid] <= r) lo = mid; else hi = mid - 1;
+// Sequence facts of query row r, looked up by each warp with all of its
+// loads in flight at once (lane l checks sequences l, l + 32, ...): the
+// sequence's first cache row and the row's causal length p + 1.
+struct RowSeq {
+  long long kv0;
+  int len;
+};
+
+__device__ __forceinline__ RowSeq row_seq_warp(const int32_t* q_offsets, const int64_t* kv_offsets,
+                                               const int32_t* ctx_lens, int B, int r) {
+  long long kv0 = 0;
+  int len = 0, hit = 0;
+  for (int b = threadIdx.x & 31; b < B; b += 32) {
+    const int q0 = __ldg(q_offsets + b), q1 = __ldg(q_offsets + b + 1);
+    const long long k0 = __ldg(kv_offsets + b);
+    const int L = __ldg(ctx_lens + b);
+    if (r >= q0 && r < q1) {
+      kv0 = k0;
+      len = L - (q1 - q0) + (r - q0) + 1;
+      hit = 1;
+    }
   }
-  return lo;
+  const unsigned m = __ballot_sync(0xffffffffu, hit);
+  const int src = m ? __ffs(m) - 1 : 0;
+  RowSeq rs;
+  rs.kv0 = __shfl_sync(0xffffffffu, kv0, src);
+  rs.len = __shfl_sync(0xffffffffu, len, src);
+  return rs;
 }
 
 __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
@@ -235,15 +258,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  const int b = owner_seq_tc(P.q_offsets, P.B, r);
-  const long long kv0 = P.kv_offsets[b];
+  const RowSeq rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
+  const long long kv0 = rs.kv0;
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
-  int n_slots = P.top_k;
-  if (P.idx_prefix) {  // slots past min(top_k, p+1) hold -1: skip their tiles
-    const int q0 = P.q_offsets[b];
-    const int pos = P.ctx_lens[b] - (P.q_offsets[b + 1] - q0) + (r - q0);
-    n_slots = min(P.top_k, pos + 1);
-  }
+  // With idx_prefix, slots past min(top_k, p+1) hold -1: skip their tiles.
+  const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
   // This CTA's slice of the slots.
   const int slot_lo = sp * P.split_len;
   const int slot_hi = min(n_slots, slot_lo + P.split_len);
@@ -516,34 +535,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     named_bar_sync(1, kSoftThreads);
     if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     tc_fence_after();
-    if (ok && P.n_split == 1) {
-#pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-        const int dv = 128 * blk + 32 * q + lane;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int hh = 32 * half + j;
-            const int h = h0 + hh;
-            if (h < P.H) {
-              const float L = l_s[hh];
-              P.out[(static_cast<size_t>(r) * P.H + h) * kValue + dv] =
-                  L > 0.f ? __uint_as_float(o[j]) / L : 0.f;
-            }
-          }
-        }
-      }
-      if (P.lse && owner && h0 + hl < P.H) {
-        P.lse[static_cast<size_t>(r) * P.H + h0 + hl] =
-            l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
-      }
-    } else if (ok) {
-      // One slice of the set: unnormalised O and (max, sum) for the merge.
-      const size_t rec = (static_cast<size_t>(sp) * P.Nq + r) * P.H;
+    // The Q block and the gather stages are free once the last product has
+    // completed (or, with no tile, once Q has landed): the 64 heads' rows of
+    // the result are staged there, [head][512] fp32, and leave in one bulk
+    // copy, contiguous in out (and in the slice partials) for the block.
+    if (ok && n_tiles == 0) ok = mbar_wait(b_qfull, 0, P.err);
+    const bool good = !named_bar_or(1, kSoftThreads, !ok);
+    if (good) {
+      const bool split = P.n_split > 1;
+      float* const stg = reinterpret_cast<float*>(bp + kOffStage);
 #pragma unroll 1
       for (int blk = 0; blk < 4; ++blk) {
         const int dv = 128 * blk + 32 * q + lane;
@@ -559,12 +559,37 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int h = h0 + 32 * half + j;
-            if (h < P.H) P.part_o[(rec + h) * kValue + dv] = __uint_as_float(o[j]);
+            const int hh = 32 * half + j;
+            float v = __uint_as_float(o[j]);
+            if (!split) {
+              const float L = l_s[hh];
+              v = L > 0.f ? v / L : 0.f;
+            }
+            stg[hh * kValue + dv] = v;
           }
         }
       }
-      if (owner && h0 + hl < P.H) P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
+      fence_proxy_async_smem();
+      named_bar_sync(1, kSoftThreads);
+      const int nh = min(kHB, P.H - h0);
+      const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
+                               : static_cast<size_t>(r) * P.H;
+      if (threadIdx.x == 0) {
+        float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
+        asm volatile(
+            "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
+            "cp.async.bulk.commit_group;\n\t"
+            "cp.async.bulk.wait_group 0;" ::"l"(dst),
+            "r"(smem_u32(stg)), "r"(static_cast<uint32_t>(nh * kValue * 4))
+            : "memory");
+      }
+      if (owner && h0 + hl < P.H) {
+        if (split) {
+          P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
+        } else if (P.lse) {
+          P.lse[rec + h0 + hl] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
+        }
+      }
     }
   }
 
