@@ -57,6 +57,7 @@ cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t st
 
 // How the attention launch covers (query row, head block, slice of the set).
 struct AttnPlan {
+  int decode;       // 1: single-tile tcgen05 kernel, slices of 64 slots (few rows)
   int tc;           // 1: tcgen05 kernel (many rows, 64 heads per CTA, no slices)
   int hb;           // heads per CTA: 16, 32, 48 or 64
   int head_blocks;  // ceil(H / hb)
@@ -89,6 +90,8 @@ struct AttnArgs {
   AttnPlan plan;
 };
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_attn_decode(const AttnArgs& a, cudaStream_t stream);
+int attn_decode_slots();  // selected slots per CTA of the single-tile kernel
 // Merges the slices of a split launch (plan.n_split > 1) into out and lse.
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);

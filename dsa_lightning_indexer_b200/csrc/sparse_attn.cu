@@ -426,12 +426,23 @@ AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms) {
   // tcgen05 kernel: 64 heads per CTA (one CTA per SM).  With few rows the
   // selected set is sliced so the GPU fills; slices hold whole 16-slot groups.
   AttnPlan p;
+  p.decode = 0;
   p.tc = 1;
   p.hb = kHeadsPerCta;
   p.head_blocks = (H + kHeadsPerCta - 1) / kHeadsPerCta;
   p.n_split = 1;
   p.split_len = top_k;
   const long long base = static_cast<long long>(Nq) * p.head_blocks;
+  // Few rows: one tile of selected slots per CTA, as long as that takes at
+  // most two waves of one CTA per SM.
+  const int slots = attn_decode_slots();
+  const int n_dec = (top_k + slots - 1) / slots;
+  if (base > 0 && base < num_sms && n_dec <= kMaxSplit && base * n_dec <= 2LL * num_sms) {
+    p.decode = 1;
+    p.n_split = n_dec;
+    p.split_len = slots;
+    return p;
+  }
   if (base > 0 && base < num_sms) {
     const int want = static_cast<int>(num_sms / base);
     const int n = std::min(std::min(want, kMaxSplit), (top_k + 15) / 16);
@@ -446,6 +457,7 @@ AttnPlan attn_plan(int Nq, int H, int top_k, int num_sms) {
 
 AttnPlan attn_plan_core(int Nq, int H, int top_k, int num_sms) {
   AttnPlan p;
+  p.decode = 0;
   p.tc = 0;
   p.hb = std::min(kHeadsPerCta, (H + 15) / 16 * 16);
   p.head_blocks = (H + p.hb - 1) / p.hb;
@@ -474,6 +486,7 @@ size_t attn_partial_bytes(int Nq, int H, const AttnPlan& p) {
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   if (a.Nq == 0) return cudaSuccess;
+  if (a.plan.decode) return launch_sparse_attn_decode(a, stream);
   if (a.plan.tc) return launch_sparse_attn_tc(a, stream);
   AttnParams P;
   P.q_offsets = a.q_offsets;

@@ -24,11 +24,12 @@
 // warps 5-6 and 7-8 gather even and odd tiles with 16-byte cp.async.
 #include <algorithm>
 
-#include "dsa_common.cuh"
-#include "dsa_internal.h"
+#include "attn_tc_common.cuh"
 
 namespace dsa {
 namespace {
+
+using namespace attn_tc;
 
 constexpr int kT = 48;                    // gathered rows per tile
 constexpr int kHB = 64;                   // heads per CTA
@@ -40,8 +41,6 @@ constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 
 constexpr int kThreadsTc = 288;
 constexpr int kSoftThreads = 128;
 constexpr int kGroupThreads = 64;         // one gather group
-constexpr float kLog2eTc = 1.4426950408889634f;
-constexpr float kLn2Tc = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
 
 constexpr int kOffQ = 0;
@@ -67,144 +66,8 @@ constexpr uint32_t kColO = 128;   // O^T blocks at 128, 192, 256, 320
 // kind::f16 instruction descriptors (bf16 in, fp32 accumulate).
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, kT);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
-
-struct TcParams {
-  const int32_t* q_offsets;
-  const int64_t* kv_offsets;
-  const int32_t* ctx_lens;
-  const __nv_bfloat16* kv;
-  const int32_t* idx;
-  float* out;
-  float* lse;
-  unsigned* err;
-  float* part_o;        // [n_split][Nq][H][512] unnormalised slice outputs (n_split > 1)
-  float2* part_ml;      // [n_split][Nq][H] (running max in log2 units, row sum)
-  int B, Nq, H, top_k;
-  int n_split, split_len;  // slices of the selected set, slots per slice
-  int idx_prefix;       // valid entries are the first min(top_k, p+1) slots
-  float scale_log2;
-};
-
-// MN-major operand in the 128-byte swizzle layout: 64-element chunks along
-// M/N `lbo` bytes apart, groups of 8 K-rows 1024 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo) {
-  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;
-  d |= static_cast<uint64_t>(1u) << 46;
-  d |= static_cast<uint64_t>(2u) << 61;
-  return d;
-}
-
-// 16x32bx2 shape: threads 0-15 read TMEM lanes base..base+15 at the given
-// column, threads 16-31 the same lanes kSplitCols columns further.  With the
-// M = 64 accumulator layout (head row 16q + j at lane 32q + j) the two half
-// warps split each head row's tile of logits between them.
-constexpr int kSplitCols = kT / 2;
-static_assert(kSplitCols == 24, "the logit loads below cover 16 + 8 columns per half warp");
-__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16], %17;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr), "n"(kSplitCols));
-}
-
-__device__ __forceinline__ void tmem_ld_16x32bx2_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], %9;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr), "n"(kSplitCols));
-}
-
-// 2^x on the special-function unit (relative error about 2^-22); 2^-inf = 0.
-__device__ __forceinline__ float exp2_fast(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async16_tc(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// OR of `pred` over the `threads` threads meeting at named barrier `id`.
-__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
-  uint32_t res;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(res)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
-      : "memory");
-  return res != 0;
-}
-
-// Sequence facts of query row r, looked up by each warp with all of its
-// loads in flight at once (lane l checks sequences l, l + 32, ...): the
-// sequence's first cache row and the row's causal length p + 1.
-struct RowSeq {
-  long long kv0;
-  int len;
-};
-
-__device__ __forceinline__ RowSeq row_seq_warp(const int32_t* q_offsets, const int64_t* kv_offsets,
-                                               const int32_t* ctx_lens, int B, int r) {
-  long long kv0 = 0;
-  int len = 0, hit = 0;
-  for (int b = threadIdx.x & 31; b < B; b += 32) {
-    const int q0 = __ldg(q_offsets + b), q1 = __ldg(q_offsets + b + 1);
-    const long long k0 = __ldg(kv_offsets + b);
-    const int L = __ldg(ctx_lens + b);
-    if (r >= q0 && r < q1) {
-      kv0 = k0;
-      len = L - (q1 - q0) + (r - q0) + 1;
-      hit = 1;
-    }
-  }
-  const unsigned m = __ballot_sync(0xffffffffu, hit);
-  const int src = m ? __ffs(m) - 1 : 0;
-  RowSeq rs;
-  rs.kv0 = __shfl_sync(0xffffffffu, kv0, src);
-  rs.len = __shfl_sync(0xffffffffu, len, src);
-  return rs;
-}
-
-__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
+constexpr int kSplitCols = kT / 2;  // logits per half warp (16 + 8 columns)
+static_assert(kSplitCols == 24, "the logit loads cover 16 + 8 columns per half warp");
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
     sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const TcParams P) {
@@ -439,8 +302,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       // This thread's half of its head row: keys k0 .. k0 + 23 of the tile.
       uint32_t va[16], vb[8];
       const uint32_t sa = tmem + lane_base + kColS + 64u * st;
-      tmem_ld_16x32bx2_x16(sa, va);
-      tmem_ld_16x32bx2_x8(sa + 16u, vb);
+      tmem_ld_16x32bx2_x16<kSplitCols>(sa, va);
+      tmem_ld_16x32bx2_x8<kSplitCols>(sa + 16u, vb);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(b_sempty(st));
@@ -576,18 +439,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                                : static_cast<size_t>(r) * P.H;
       if (threadIdx.x == 0) {
         float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
-        asm volatile(
-            "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
-            "cp.async.bulk.commit_group;\n\t"
-            "cp.async.bulk.wait_group 0;" ::"l"(dst),
-            "r"(smem_u32(stg)), "r"(static_cast<uint32_t>(nh * kValue * 4))
-            : "memory");
+        bulk_store_wait(dst, smem_u32(stg), static_cast<uint32_t>(nh * kValue * 4));
       }
       if (owner && h0 + hl < P.H) {
         if (split) {
           P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
         } else if (P.lse) {
-          P.lse[rec + h0 + hl] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2Tc : -INFINITY;
+          P.lse[rec + h0 + hl] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         }
       }
     }
@@ -639,7 +497,7 @@ cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   P.Nq = a.Nq;
   P.H = a.H;
   P.top_k = a.top_k;
-  P.scale_log2 = a.scale * kLog2eTc;
+  P.scale_log2 = a.scale * kLog2e;
   const int head_blocks = (a.H + kHB - 1) / kHB;
   e = launch_pdl(sparse_attn_tc_kernel, dim3(a.Nq, head_blocks, a.plan.n_split),
                  dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, P);
