@@ -101,20 +101,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
 
+  const int slot_lo = sp * P.split_len;
+  // The gather warps request their slot entries before the row lookup
+  // returns (the entries past the row's causal length are masked below).
+  int pos_raw = -1;
+  if (warp >= 5) {
+    const int slot = slot_lo + (threadIdx.x - 160);
+    if (threadIdx.x - 160 < kTD && slot < min(P.top_k, slot_lo + P.split_len)) {
+      pos_raw = __ldg(P.idx + static_cast<size_t>(r) * P.top_k + slot);
+    }
+  }
   const RowSeq rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
   const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
-  const int slot_lo = sp * P.split_len;
   const bool work = slot_lo < n_slots;  // block-uniform
 
   if (warp >= 5) {
     // ------------------------------------------------------------ gather --
     const int g = threadIdx.x - 160;  // 0..127
     if (work) {
-      if (g < kTD) {
-        const int slot = slot_lo + g;
-        const int slot_hi = min(n_slots, slot_lo + P.split_len);
-        tidx[g] = slot < slot_hi ? __ldg(P.idx + static_cast<size_t>(r) * P.top_k + slot) : -1;
-      }
+      if (g < kTD) tidx[g] = slot_lo + g < n_slots ? pos_raw : -1;
       named_bar_sync(2, kGatherThreads);
       // Each thread copies whole 128-byte box rows: eight 16-byte pieces with
       // the swizzle applied.
@@ -260,11 +265,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (good) {
       const bool split = P.n_split > 1;
       float* const stg = reinterpret_cast<float*>(bp + kOffStage);
+      const int nh = min(kHB, P.H - h0);
+      const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
+                               : static_cast<size_t>(r) * P.H;
+      float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
+      // Heads 0-31, then 32-63: each half leaves in its own bulk copy while
+      // the next half is staged.
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-        const int dv = 128 * blk + 32 * q + lane;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          const int dv = 128 * blk + 32 * q + lane;
           uint32_t o[32];
           if (work) {
             tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
@@ -284,16 +295,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             stg[hh * kValue + dv] = v;
           }
         }
+        fence_proxy_async_smem();
+        named_bar_sync(1, kSoftThreads);
+        const int n_half = min(32, nh - 32 * half);
+        if (threadIdx.x == 0 && n_half > 0) {
+          bulk_store_issue(dst + static_cast<size_t>(32 * half) * kValue,
+                           smem_u32(stg + 32 * half * kValue),
+                           static_cast<uint32_t>(n_half * kValue * 4));
+        }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, kSoftThreads);
-      const int nh = min(kHB, P.H - h0);
-      const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
-                               : static_cast<size_t>(r) * P.H;
-      if (threadIdx.x == 0) {
-        bulk_store_wait((split ? P.part_o : P.out) + (rec + h0) * kValue, smem_u32(stg),
-                        static_cast<uint32_t>(nh * kValue * 4));
-      }
+      if (threadIdx.x == 0) bulk_wait_all();
       if (owner && h0 + hl < P.H) {
         if (split) {
           P.part_ml[rec + h0 + hl] = make_float2(m, l);

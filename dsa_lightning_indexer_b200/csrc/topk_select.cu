@@ -735,6 +735,34 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_emit_kernel(const HistParam
   for (int i = tid + 2 * kHThreads; i + n_cand_own < m; i += kHThreads) {
     fin[n_cand_own + i] = __ldcg(cg + i);
   }
+  __syncthreads();
+  if (m <= 64) {  // the usual case: one warp sorts two positions per lane with shuffles
+    if (tid < 32) {
+      int v0 = tid < m ? fin[tid] : 0x7FFFFFFF;
+      int v1 = tid + 32 < m ? fin[tid + 32] : 0x7FFFFFFF;
+#pragma unroll
+      for (int sz = 2; sz <= 64; sz <<= 1) {  // ascending bitonic network over 64 slots
+#pragma unroll
+        for (int stride = sz >> 1; stride > 0; stride >>= 1) {
+          if (stride == 32) {  // slots tid and tid + 32 of this lane (sz = 64: ascending)
+            const int lo_v = min(v0, v1), hi_v = max(v0, v1);
+            v0 = lo_v;
+            v1 = hi_v;
+          } else {
+            const bool lower = (tid & stride) == 0;
+            const int p0 = __shfl_xor_sync(0xffffffffu, v0, stride);
+            const int p1 = __shfl_xor_sync(0xffffffffu, v1, stride);
+            const bool up0 = (tid & sz) == 0, up1 = ((tid + 32) & sz) == 0;
+            v0 = (lower == up0) ? min(v0, p0) : max(v0, p0);
+            v1 = (lower == up1) ? min(v1, p1) : max(v1, p1);
+          }
+        }
+      }
+      if (tid < m && offset + tid < k) R.out[offset + tid] = v0;
+      if (tid + 32 < m && offset + tid + 32 < k) R.out[offset + tid + 32] = v1;
+    }
+    return;
+  }
   int size = 1;
   while (size < m) size <<= 1;
   for (int i = m + tid; i < size; i += kHThreads) fin[i] = 0x7FFFFFFF;
