@@ -164,6 +164,17 @@ def glue_projection(seed, n_in=DV, H=64) -> np.ndarray:
     return normal_bf16(seed, 0, T_PROJ, (n_in, H * D), std=1.0 / math.sqrt(n_in))
 
 
+def chain_query(out: np.ndarray, proj: np.ndarray) -> np.ndarray:
+    """Next stacked layer's main query from this layer's output [Nq, H, 512]:
+    the mean over heads, RMS-normalised and rounded to bf16, times the fixed
+    projection [512, H*576], rounded to bf16 -> [Nq, H, 576] bit patterns."""
+    m = np.asarray(out, dtype=np.float64).mean(axis=1)
+    m = m / np.sqrt((m * m).mean(axis=1, keepdims=True) + 1e-6)
+    x = bf16_to_f32(bf16_bits(m.astype(np.float32)))
+    q = x @ bf16_to_f32(proj)
+    return bf16_bits(q).reshape(out.shape[0], -1, D)
+
+
 # The five workloads the layer is specified on.
 def tiny_prefill(top_k: int) -> Workload:
     """Prefill, 1 sequence of 1024 tokens, 16 heads; run at top_k 256 and 2048. Seed 0."""

@@ -336,3 +336,24 @@ def test_workspace_control_block_is_zero_after_calls(make):
     bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws)
     torch.cuda.synchronize()
     assert not dw.ws[:256].any().item()
+
+
+def test_ragged_stacked_layers_sampled_rows():
+    """The ragged serving batch (32 contexts log-uniform in [1024, 131072],
+    some below top_k): layer 0, then layer 1 whose main query is chained from
+    layer 0's output through the fixed projection.  Sampled rows of each layer
+    (the two shortest, the median, the longest) against the oracle on the same
+    inputs.  Two of the 24 stacked layers: each layer's inputs take the host
+    about 17 s to draw."""
+    proj = synth.glue_projection(4)
+    q = None
+    for layer in range(2):
+        wl = synth.ragged_layer(layer)
+        if q is not None:
+            wl.q = q
+        order = np.argsort(wl.ctx_lens)
+        rows = sorted({int(order[0]), int(order[1]), int(order[len(order) // 2]), int(order[-1])})
+        assert wl.ctx_lens[order[0]] < wl.top_k  # the top_k >= context path is exercised
+        out, _ = _layer_check(wl, rows=rows)
+        q = synth.chain_query(out, proj)
+        assert q.shape == wl.q.shape
