@@ -39,8 +39,7 @@ namespace {
 constexpr int kKeysPerTile = 128;
 constexpr int kKTileBytes = kKeysPerTile * kIdxDim * 2;  // 32 KB
 constexpr int kKBoxBytes = kKTileBytes / 2;              // 128 rows x 64 dims
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kEpiThreads = 128;  // one epilogue set: a warp per TMEM lane quadrant
 
 struct SeqItems {
   long long kv_off;
@@ -61,6 +60,10 @@ struct IdxParams {
 template <int QT>
 struct Cfg {
   static constexpr int N = 32 * QT;
+  // Epilogue sets: with 4 or 8 queries per item the read-out of a tile takes
+  // longer than its MMAs, so two sets of four warps split the queries.
+  static constexpr int kEpiSets = QT >= 4 ? 2 : 1;
+  static constexpr int kThreads = 64 + kEpiSets * kEpiThreads;
   static constexpr int kQBufs = QT <= 4 ? 2 : 1;
   // K ring depth: deep for decode (HBM streaming), shallower when Q is large.
   static constexpr int kStages = QT == 1 ? 5 : (QT == 2 ? 6 : 4);
@@ -110,7 +113,7 @@ __device__ __forceinline__ int snake_item(int j) {
 }
 
 template <int QT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     indexer_score_kernel(const __grid_constant__ CUtensorMap kmap,
                          const __grid_constant__ CUtensorMap qmap,
                          const __grid_constant__ IdxParams P) {
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(qfull(i), 1);
       mbar_init(qempty(i), 1);
       mbar_init(tfull(i), 1);
-      mbar_init(tempty(i), kEpiThreads);
+      mbar_init(tempty(i), C::kEpiSets * kEpiThreads);
     }
     fence_mbar_init();
   }
@@ -254,7 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127
+    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 in the first set
+    const int jset = (warp - 2) >> 2;                    // this warp's epilogue set
     const bool do_hist = (QT == 1) && P.hist != nullptr;
     if (do_hist) {
       for (int i = et; i < kHistBins; i += kEpiThreads) shist[i] = 0;
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int key = kt * kKeysPerTile + quad * 32 + lane;
 #pragma unroll 1
-        for (int jq = 0; jq < QT; ++jq) {
+        for (int jq = jset; jq < QT; jq += C::kEpiSets) {
           if (jq >= v.nrow) break;
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + lane_base + static_cast<uint32_t>(acc * C::N + jq * 32), r);
@@ -400,7 +404,7 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.n_items = items;
     if (items == 0) continue;
     const int grid = std::min(items, a.num_sms);
-    e = launch_pdl(indexer_score_kernel<QT>, dim3(grid), dim3(kThreads), C::kSmemBytes, stream, 0,
+    e = launch_pdl(indexer_score_kernel<QT>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, 0,
                    kmap, qmap, P);
     if (e != cudaSuccess) return e;
   }
