@@ -61,8 +61,8 @@ template <int QT>
 struct Cfg {
   static constexpr int N = 32 * QT;
   // Epilogue sets: with 4 or 8 queries per item the read-out of a tile takes
-  // longer than its MMAs, so two sets of four warps split the queries.
-  static constexpr int kEpiSets = QT >= 4 ? 2 : 1;
+  // longer than its MMAs, so two or four sets of four warps split the queries.
+  static constexpr int kEpiSets = QT >= 8 ? 4 : (QT >= 4 ? 2 : 1);
   static constexpr int kThreads = 64 + kEpiSets * kEpiThreads;
   static constexpr int kQBufs = QT <= 4 ? 2 : 1;
   // K ring depth: deep for decode (HBM streaming), shallower when Q is large.
