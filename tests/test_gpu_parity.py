@@ -154,6 +154,10 @@ ATTN = {
     "decode_h64_split": lambda: synth.custom([3000, 2100, 64], [1, 1, 1], 64, 2048, seed=112),
     "decode_h128": lambda: synth.custom([2500], [1], 128, 1024, seed=113),
     "mixed_h1": lambda: synth.custom([90, 40], [5, 40], 1, 32, seed=114),
+    # 12 rows: too many one-tile slices for two waves, so the many-row kernel
+    # runs with slices of the selected set and the merge
+    "decode_12rows_split": lambda: synth.custom([2200 + 150 * i for i in range(12)], [1] * 12, 64,
+                                                2048, seed=116),
 }
 
 
