@@ -124,7 +124,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Each thread copies whole 128-byte box rows: eight 16-byte pieces with
       // the swizzle applied.
       for (int item = g; item < kTD * kBoxes; item += kGatherThreads) {
-        const int i = item / kBoxes, bx = item - i * kBoxes;
+        // Rows fastest: a warp's lanes take consecutive rows of one box, so
+        // the swizzled 16-byte pieces of one instruction spread over all
+        // eight bank groups of shared memory.
+        const int bx = item / kTD, i = item - bx * kTD;
         const int pos = tidx[i];
         const uint32_t drow = sKV + bx * kKVBox + i * 128;
         const uint32_t x = static_cast<uint32_t>(i & 7);

@@ -168,7 +168,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       pos_nxt = load_pos(t + 4);
       const uint32_t stage = sKV + grp * kKVStage;
       for (int item = gt; item < kT * kBoxes; item += kGroupThreads) {
-        const int i = item / kBoxes, bx = item - i * kBoxes;
+        // Rows fastest: a warp's lanes take consecutive rows of one box, so
+        // the swizzled 16-byte pieces of one instruction spread over all
+        // eight bank groups of shared memory.
+        const int bx = item / kT, i = item - bx * kT;
         const int pos = gidx[i];
         const uint32_t drow = stage + bx * kKVBox + i * 128;
         const uint32_t x = static_cast<uint32_t>(i & 7);
