@@ -478,13 +478,13 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_filter_kernel(const HistPar
     keys[j] = s < s_end ? score_key(__ldcg(R.sc + s)) : 0u;
   }
   const int u = kHThreads - 1 - tid;  // thread t reads bins 8u .. 8u+7, u = 511 - t
-  int cb[8];
+  // Two 16-byte loads per thread: every CTA of the row reads this histogram.
+  const int4 h0 = __ldcg(reinterpret_cast<const int4*>(R.gh) + 2 * u);
+  const int4 h1 = __ldcg(reinterpret_cast<const int4*>(R.gh) + 2 * u + 1);
+  const int cb[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
   int tot = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    cb[j] = __ldcg(R.gh + 8 * u + j);
-    tot += cb[j];
-  }
+  for (int j = 0; j < 8; ++j) tot += cb[j];
   __syncthreads();
   const int n = s_n;
   if (R.c == 0 && tid == 0) R.cnt[3] = n;
