@@ -27,6 +27,7 @@ struct TcParams {
   int B, Nq, H, top_k;
   int n_split, split_len;  // slices of the selected set, slots per slice
   int idx_prefix;       // valid entries are the first min(top_k, p+1) slots
+  int batch_ready;      // the batch arrays may be read before the dependent-launch wait
   float scale_log2;
 };
 

@@ -286,6 +286,7 @@ dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.err = err_word(ws);
   a.ctx_lens = batch->ctx_lens;
   a.idx_prefix = false;
+  a.batch_ready = false;
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
 }
@@ -358,6 +359,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   a.err = err_word(ws);
   a.ctx_lens = batch->ctx_lens;
   a.idx_prefix = true;  // produced by dsa_topk: valid positions first, then -1
+  a.batch_ready = true;  // the layer's own kernels never write the batch arrays
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, st));
 }

@@ -87,6 +87,7 @@ struct AttnArgs {
   float* part;        // split partials (workspace); unused when plan.n_split == 1
   unsigned* err;      // workspace error word (bounded waits)
   bool idx_prefix;    // valid entries are the first min(top_k, p+1) slots of each row
+  bool batch_ready;   // no kernel this launch depends on writes the batch arrays
   AttnPlan plan;
 };
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream);

@@ -98,6 +98,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  // Inside the layer the batch arrays are inputs no earlier kernel writes:
+  // look the row up while the previous kernel finishes.
+  RowSeq rs = {};
+  if (P.batch_ready) rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
   pdl_wait();
   pdl_launch_dependents();
 
@@ -111,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pos_raw = __ldg(P.idx + static_cast<size_t>(r) * P.top_k + slot);
     }
   }
-  const RowSeq rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
+  if (!P.batch_ready) rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
   const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
   const bool work = slot_lo < n_slots;  // block-uniform
 
@@ -357,6 +361,7 @@ cudaError_t launch_sparse_attn_decode(const AttnArgs& a, cudaStream_t stream) {
   P.lse = a.lse;
   P.err = a.err;
   P.idx_prefix = a.idx_prefix ? 1 : 0;
+  P.batch_ready = a.batch_ready ? 1 : 0;
   P.n_split = a.plan.n_split;
   P.split_len = a.plan.split_len;
   const size_t n_rec = static_cast<size_t>(a.plan.n_split) * a.Nq * a.H;

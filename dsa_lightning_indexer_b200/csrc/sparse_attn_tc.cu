@@ -491,6 +491,7 @@ cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   P.lse = a.lse;
   P.err = a.err;
   P.idx_prefix = a.idx_prefix ? 1 : 0;
+  P.batch_ready = a.batch_ready ? 1 : 0;
   P.n_split = a.plan.n_split;
   P.split_len = a.plan.split_len;
   const size_t n_rec = static_cast<size_t>(a.plan.n_split) * a.Nq * a.H;
