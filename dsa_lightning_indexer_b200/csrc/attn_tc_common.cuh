@@ -166,6 +166,13 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Waits until all committed bulk copies have finished reading shared memory
+// (their global writes may still be in flight; they complete before the
+// grid does).
+__device__ __forceinline__ void bulk_wait_all_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Writes `bytes` (a multiple of 16) of shared memory at `src` to global `dst`
 // (16-byte aligned) with one bulk copy and waits until it has completed.
 __device__ __forceinline__ void bulk_store_wait(void* dst, uint32_t src, uint32_t bytes) {

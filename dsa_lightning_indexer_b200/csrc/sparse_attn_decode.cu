@@ -73,8 +73,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  b_pfull = bars + 24u, b_odone = bars + 32u;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
-  float* const m_s = reinterpret_cast<float*>(bp + kOffM);
-  float* const l_s = reinterpret_cast<float*>(bp + kOffL);
+  float* const rl_s = reinterpret_cast<float*>(bp + kOffL);  // 1 / row sum per head
 
   const int warp = warp_id_uniform();
   const int lane = lane_id();
@@ -260,8 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (owner) {
-      m_s[hl] = m;
-      l_s[hl] = l;
+      rl_s[hl] = l > 0.f ? 1.f / l : 0.f;
     }
     // ------------------------------------------------------------ output --
     // Q and the tile are free once the products have completed (or, with no
@@ -295,10 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) {
             const int hh = 32 * half + j;
             float v = __uint_as_float(o[j]);
-            if (!split) {
-              const float L = l_s[hh];
-              v = L > 0.f ? v / L : 0.f;
-            }
+            if (!split) v *= rl_s[hh];
             stg[hh * kValue + dv] = v;
           }
         }
@@ -311,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            static_cast<uint32_t>(n_half * kValue * 4));
         }
       }
-      if (threadIdx.x == 0) bulk_wait_all();
+      if (threadIdx.x == 0) bulk_wait_all_read();
       if (owner && h0 + hl < P.H) {
         if (split) {
           P.part_ml[rec + h0 + hl] = make_float2(m, l);

@@ -88,8 +88,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
-  float* const m_s = reinterpret_cast<float*>(bp + kOffM);
-  float* const l_s = reinterpret_cast<float*>(bp + kOffL);
+  float* const rl_s = reinterpret_cast<float*>(bp + kOffL);  // 1 / row sum per head
 
   const int warp = warp_id_uniform();
   const int lane = lane_id();
@@ -394,10 +393,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_arrive(b_pfull(st));
     }
     // ------------------------------------------------------------ output --
-    if (owner) {
-      m_s[hl] = m_run;
-      l_s[hl] = l_run;
-    }
+    if (owner) rl_s[hl] = l_run > 0.f ? 1.f / l_run : 0.f;
     named_bar_sync(1, kSoftThreads);
     if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     tc_fence_after();
@@ -410,11 +406,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     if (good) {
       const bool split = P.n_split > 1;
       float* const stg = reinterpret_cast<float*>(bp + kOffStage);
+      const int nh = min(kHB, P.H - h0);
+      const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
+                               : static_cast<size_t>(r) * P.H;
+      float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
+      // Heads 0-31, then 32-63: each half leaves in its own bulk copy while
+      // the next half is staged.
 #pragma unroll 1
-      for (int blk = 0; blk < 4; ++blk) {
-        const int dv = 128 * blk + 32 * q + lane;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk) {
+          const int dv = 128 * blk + 32 * q + lane;
           uint32_t o[32];
           if (n_tiles > 0) {
             tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
@@ -427,23 +429,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int j = 0; j < 32; ++j) {
             const int hh = 32 * half + j;
             float v = __uint_as_float(o[j]);
-            if (!split) {
-              const float L = l_s[hh];
-              v = L > 0.f ? v / L : 0.f;
-            }
+            if (!split) v *= rl_s[hh];
             stg[hh * kValue + dv] = v;
           }
         }
+        fence_proxy_async_smem();
+        named_bar_sync(1, kSoftThreads);
+        const int n_half = min(32, nh - 32 * half);
+        if (threadIdx.x == 0 && n_half > 0) {
+          bulk_store_issue(dst + static_cast<size_t>(32 * half) * kValue,
+                           smem_u32(stg + 32 * half * kValue),
+                           static_cast<uint32_t>(n_half * kValue * 4));
+        }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, kSoftThreads);
-      const int nh = min(kHB, P.H - h0);
-      const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
-                               : static_cast<size_t>(r) * P.H;
-      if (threadIdx.x == 0) {
-        float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
-        bulk_store_wait(dst, smem_u32(stg), static_cast<uint32_t>(nh * kValue * 4));
-      }
+      // Shared memory must outlive the copies' reads; their writes finish
+      // on their own before the grid completes.
+      if (threadIdx.x == 0) bulk_wait_all_read();
       if (owner && h0 + hl < P.H) {
         if (split) {
           P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
