@@ -443,46 +443,77 @@ def kernel_times(bd, copies, wl, steps, dev):
     return res
 
 
+def _packed(parts, align=256):
+    """Byte offsets of `parts` (name, nbytes) packed into one buffer."""
+    offs, n = {}, 0
+    for name, nbytes in parts:
+        offs[name] = n
+        n += (nbytes + align - 1) // align * align
+    return offs, n
+
+
 def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
     """Decode step through host buffers: the step's new inputs (queries, indexer
-    queries and weights, and the new token's rows of both caches) are copied from
-    pinned host memory into the resident caches, the layer runs, and its output,
-    log-sum-exp and index sets are read back into pinned host memory."""
-    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-    h_q = pin(wl.q.view(np.int16))
-    h_qi = pin(wl.q_idx.view(np.int16))
-    h_w = pin(wl.w)
+    queries and weights, and the new token's rows of both caches) arrive in one
+    copy from pinned host memory, the cache rows are scattered into the
+    resident caches, the layer runs, and its output, log-sum-exp and index sets
+    leave in one copy into pinned host memory.  The step is captured once as a
+    CUDA graph (copies included) and replayed, as a serving loop would."""
     new_rows = [int(wl.kv_offsets[b] + wl.ctx_lens[b] - 1) for b in range(wl.B)]
-    h_krow = pin(wl.k_idx[new_rows].view(np.int16))
-    h_vrow = pin(wl.kv[new_rows].view(np.int16))
-    out, lse, idx = dw.new_outputs()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h_idx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    q16, qi16 = dw.q.view(torch.int16), dw.q_idx.view(torch.int16)
+    host_in = {"q": wl.q, "q_idx": wl.q_idx, "w": wl.w,
+               "krow": wl.k_idx[new_rows], "vrow": wl.kv[new_rows]}
+    offs, n_in = _packed([(k, v.nbytes) for k, v in host_in.items()])
+    h_in = torch.empty(n_in, dtype=torch.uint8).pin_memory()
+    hv = h_in.numpy()
+    for k, v in host_in.items():
+        hv[offs[k]:offs[k] + v.nbytes] = np.ascontiguousarray(v).view(np.uint8).ravel()
+    d_in = torch.empty(n_in, dtype=torch.uint8, device=dev)
+
+    def dview(buf, o, shape, dtype):
+        nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        return buf[o:o + nbytes].view(dtype).view(*shape)
+
+    q = dview(d_in, offs["q"], wl.q.shape, torch.bfloat16)
+    q_idx = dview(d_in, offs["q_idx"], wl.q_idx.shape, torch.bfloat16)
+    w = dview(d_in, offs["w"], wl.w.shape, torch.float32)
+    krow = dview(d_in, offs["krow"], host_in["krow"].shape, torch.int16)
+    vrow = dview(d_in, offs["vrow"], host_in["vrow"].shape, torch.int16)
+    rows = torch.tensor(new_rows, dtype=torch.long, device=dev)
     k16, v16 = dw.k_idx.view(torch.int16), dw.kv.view(torch.int16)
 
-    def step():
-        q16.copy_(h_q, non_blocking=True)
-        qi16.copy_(h_qi, non_blocking=True)
-        dw.w.copy_(h_w, non_blocking=True)
-        for j, r in enumerate(new_rows):
-            k16[r].copy_(h_krow[j], non_blocking=True)
-            v16[r].copy_(h_vrow[j], non_blocking=True)
-        dw.forward(out, lse, idx)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
-        h_idx.copy_(idx, non_blocking=True)
+    Nq, H, top_k = wl.Nq, wl.H, wl.top_k
+    oo, n_out = _packed([("out", Nq * H * 512 * 4), ("lse", Nq * H * 4), ("idx", Nq * top_k * 4)])
+    d_out = torch.empty(n_out, dtype=torch.uint8, device=dev)
+    h_out = torch.empty(n_out, dtype=torch.uint8).pin_memory()
+    out = dview(d_out, oo["out"], (Nq, H, 512), torch.float32)
+    lse = dview(d_out, oo["lse"], (Nq, H), torch.float32)
+    idx = dview(d_out, oo["idx"], (Nq, top_k), torch.int32)
 
-    for _ in range(warmup):
+    def step():
+        d_in.copy_(h_in, non_blocking=True)
+        k16.index_copy_(0, rows, krow)
+        v16.index_copy_(0, rows, vrow)
+        bd.layer_forward(dw.batch, q, q_idx, w, dw.k_idx, dw.kv, top_k, wl.scale,
+                         out, lse, idx, dw.ws)
+        h_out.copy_(d_out, non_blocking=True)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
         step()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step()
+    torch.cuda.current_stream().wait_stream(s)
+    for _ in range(warmup):
+        g.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
-        step()
+        g.replay()
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
@@ -491,11 +522,21 @@ def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     bd.check_device_status(dw.ws)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_qi, h_w, h_krow, h_vrow))
-    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
+    # The replayed step really moved the results: compare with a plain call.
+    ref_out, ref_lse, ref_idx = dw.forward()
+    torch.cuda.synchronize()
+    hb = h_out.numpy()
+    got_idx = hb[oo["idx"]:oo["idx"] + Nq * top_k * 4].view(np.int32).reshape(Nq, top_k)
+    got_out = hb[oo["out"]:oo["out"] + Nq * H * 512 * 4].view(np.float32).reshape(Nq, H, 512)
+    if not (np.array_equal(got_idx, ref_idx.cpu().numpy())
+            and np.allclose(got_out, ref_out.cpu().numpy(), rtol=0.0, atol=1e-5)):
+        raise RuntimeError("e2e: the results read back differ from a direct layer call")
+    del g
     return {"value": wl.Nq * world * steps / (ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": ms / steps}
+            "h2d_bytes_per_step": int(n_in), "d2h_bytes_per_step": int(n_out),
+            "ms_per_step": ms / steps,
+            "method": "CUDA graph per step: one packed H2D copy, cache-row scatter, "
+                      "dsa_layer_forward, one packed D2H copy"}
 
 
 def prefill_bench(bd, dev, peaks, args):
