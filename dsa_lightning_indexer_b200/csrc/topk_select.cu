@@ -12,13 +12,17 @@
 // key > theta plus the first `need` keys == theta, compacting with ballot
 // prefix counts so the output is deterministic and sorted by position.
 //
-// Main kernel: a thread-block cluster of CS CTAs per row (CS = 1 for the many
-// short rows of a prefill, up to 8 for the few long rows of a decode).  Each
-// CTA holds a contiguous slice of the row's keys in shared memory, so the row
-// is read from memory once; per-pass histograms are summed across the cluster
-// through distributed shared memory (plain loads), and each CTA learns how
-// many selections precede its slice from the other CTAs' counts.  Rows longer
-// than 8 slices use the single-CTA kernel that re-reads the row each pass.
+// Launch shapes: many rows that fit one CTA's shared memory (a prefill) take
+// one CTA per row, which finds the bin of the k-th key from a 12-bit
+// histogram built while loading and runs the exact passes over that bin's
+// keys only.  Few long rows (a standalone decode selection) take a
+// thread-block cluster of 2-8 CTAs per row: each CTA holds a contiguous slice
+// of the row's keys in shared memory, so the row is read from memory once;
+// per-pass histograms are summed across the cluster through distributed
+// shared memory (plain loads), and each CTA learns how many selections
+// precede its slice from the other CTAs' counts.  Rows longer than 8 slices
+// use the single-CTA kernel that re-reads the row each pass.  Decode inside
+// the layer call uses the histogram path at the end of this file.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -409,6 +413,183 @@ __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, i
   }
   theta = prefix;
   need = remaining;
+}
+
+// ------------------------------------------------------- one CTA per row --
+// Many rows that each fit one CTA's shared memory (prefill).  Three sweeps
+// over the row's keys instead of one per radix digit:
+//   1. load the scores as keys (16-byte loads) and count them by their top
+//      12 bits; one scan of the 4096 counts gives the bin holding the k-th
+//      largest key and how many keys lie above it;
+//   2. copy the keys of that bin (typically a few hundred) with their
+//      positions to a candidate list, and count per warp chunk the keys
+//      above the bin;
+//      the k-th key theta and the number of keys equal to theta to keep then
+//      come from radix passes over the candidates alone (over the whole row
+//      when the bin holds more than kRowCandMax keys, i.e. heavy ties);
+//   3. emit in position order as the cluster kernel does.
+constexpr int kRowCandMax = 2048;
+
+__device__ __forceinline__ void row_hist_add(int* hist, uint32_t key) {
+  atomicAdd(&hist[key >> kHistShift], 1);
+}
+
+__global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  int* const hist = reinterpret_cast<int*>(smem);                          // [kHistBins]
+  uint32_t* const ckey = reinterpret_cast<uint32_t*>(hist + kHistBins);    // [kRowCandMax]
+  int* const cpos = reinterpret_cast<int*>(ckey + kRowCandMax);            // [kRowCandMax]
+  uint32_t* const keys = reinterpret_cast<uint32_t*>(cpos + kRowCandMax);  // [slice]
+  __shared__ int buf[kHWarps + 1];
+  __shared__ int s_bin, s_above, s_cnt, s_ncand;
+  __shared__ int warp_gt[kHWarps], warp_eq[kHWarps];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int r = blockIdx.x;
+  const int b = owner_seq(P.q_offsets, P.B, r);
+  const int q0 = P.q_offsets[b];
+  const int nq = P.q_offsets[b + 1] - q0;
+  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;  // positions 0..p; n <= slice
+  const int k = P.top_k;
+  int32_t* const out = P.idx + static_cast<size_t>(r) * k;
+  if (n <= k) {  // every causal position is kept
+    for (int i = tid; i < k; i += kHThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+
+  // ---- sweep 1: keys into shared memory, coarse histogram
+  for (int i = tid; i < kHistBins; i += kHThreads) hist[i] = 0;
+  if (tid == 0) s_ncand = 0;
+  if (tid < kHWarps) {
+    warp_gt[tid] = 0;
+    warp_eq[tid] = 0;
+  }
+  __syncthreads();
+  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
+  const int n4 = (reinterpret_cast<uintptr_t>(sc) & 15u) == 0 ? (n & ~3) : 0;
+  for (int i = 4 * tid; i < n4; i += 4 * kHThreads) {
+    const float4 v = *reinterpret_cast<const float4*>(sc + i);
+    const uint4 kk = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
+    *reinterpret_cast<uint4*>(keys + i) = kk;
+    row_hist_add(hist, kk.x);
+    row_hist_add(hist, kk.y);
+    row_hist_add(hist, kk.z);
+    row_hist_add(hist, kk.w);
+  }
+  for (int i = n4 + tid; i < n; i += kHThreads) {
+    const uint32_t key = score_key(sc[i]);
+    keys[i] = key;
+    row_hist_add(hist, key);
+  }
+  __syncthreads();
+  {
+    // Thread t holds bins 8u .. 8u+7 with u = 511 - t, so the exclusive
+    // prefix in thread order counts the keys in higher bins.
+    const int u = kHThreads - 1 - tid;
+    const int4 ha = reinterpret_cast<const int4*>(hist)[2 * u];
+    const int4 hb = reinterpret_cast<const int4*>(hist)[2 * u + 1];
+    const int c[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tot += c[j];
+    int total;
+    int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
+    if (above < k && k <= above + tot) {
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        if (above + c[j] >= k) {
+          s_bin = 8 * u + j;
+          s_above = above;
+          s_cnt = c[j];
+          break;
+        }
+        above += c[j];
+      }
+    }
+  }
+  __syncthreads();
+  const int bin = s_bin;
+  const int want = k - s_above;  // keys to keep from the bin, 1 .. s_cnt
+  const bool compact = s_cnt <= kRowCandMax;
+
+  // ---- sweep 2: candidates of the bin; keys above the bin per warp chunk
+  const int per_warp = ((n + kHWarps - 1) / kHWarps + 31) & ~31;
+  const int w0 = warp * per_warp;
+  const int w1 = min(n, w0 + per_warp);
+  const unsigned lt = (1u << lane) - 1u;
+  if (compact) {
+    int g = 0;
+    for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
+      const bool in = i < w1;
+      const int d = in ? static_cast<int>(keys[i] >> kHistShift) : -1;
+      g += __popc(__ballot_sync(0xffffffffu, d > bin));
+      const unsigned m = __ballot_sync(0xffffffffu, d == bin);
+      if (m != 0u) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&s_ncand, __popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if ((m >> lane) & 1u) {
+          const int j = base + __popc(m & lt);
+          ckey[j] = keys[i];
+          cpos[j] = i;
+        }
+      }
+    }
+    if (lane == 0) atomicAdd(&warp_gt[warp], g);
+  }
+  __syncthreads();
+  uint32_t theta;
+  int need;
+  const uint32_t known = static_cast<uint32_t>(bin) << kHistShift;
+  const uint32_t known_mask = ~((1u << kHistShift) - 1u);
+  if (compact) {
+    smem_select(ckey, s_ncand, want, 0, kHistShift - 1, known, known_mask, hist, buf, theta, need);
+    // Candidates above theta and equal to it, by the warp chunk holding them.
+    const int nc = s_ncand;
+    for (int j = tid; j < nc; j += kHThreads) {
+      const uint32_t key = ckey[j];
+      const int w = cpos[j] / per_warp;
+      if (key > theta) {
+        atomicAdd(&warp_gt[w], 1);
+      } else if (key == theta) {
+        atomicAdd(&warp_eq[w], 1);
+      }
+    }
+  } else {
+    smem_select(keys, n, want, 0, kHistShift - 1, known, known_mask, hist, buf, theta, need);
+    int g = 0, e = 0;
+    for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
+      const bool in = i < w1;
+      const uint32_t key = in ? keys[i] : 0u;
+      g += __popc(__ballot_sync(0xffffffffu, in && key > theta));
+      e += __popc(__ballot_sync(0xffffffffu, in && key == theta));
+    }
+    if (lane == 0) {
+      warp_gt[warp] = g;
+      warp_eq[warp] = e;
+    }
+  }
+  __syncthreads();
+
+  // ---- sweep 3: emit keys > theta and the first `need` keys == theta
+  int eq_acc = 0, sel_acc = 0;
+  for (int w = 0; w < warp; ++w) {
+    sel_acc += warp_gt[w] + min(max(need - eq_acc, 0), warp_eq[w]);
+    eq_acc += warp_eq[w];
+  }
+  for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
+    const bool in = i < w1;
+    const uint32_t key = in ? keys[i] : 0u;
+    const unsigned gm = __ballot_sync(0xffffffffu, in && key > theta);
+    const unsigned em = __ballot_sync(0xffffffffu, in && key == theta);
+    const bool take_eq = ((em >> lane) & 1u) && eq_acc + __popc(em & lt) < need;
+    const unsigned sm = gm | __ballot_sync(0xffffffffu, take_eq);
+    if ((sm >> lane) & 1u) out[sel_acc + __popc(sm & lt)] = i;
+    eq_acc += __popc(em);
+    sel_acc += __popc(sm);
+  }
 }
 
 // Row bookkeeping shared by the two kernels of the histogram path.
@@ -877,6 +1058,15 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
     return launch_pdl(topk_rows_kernel, dim3(a.Nq), dim3(kThreads), 0, stream, 0, P);
   }
   P.slice = static_cast<int>(slice_of(cs));
+  if (cs == 1) {  // many rows, each within one CTA
+    const size_t head = static_cast<size_t>(kHistBins) * sizeof(int) +
+                        static_cast<size_t>(kRowCandMax) * (sizeof(uint32_t) + sizeof(int));
+    cudaError_t e = ensure_smem_limit<topk_row_cta_kernel>(
+        static_cast<int>(head + static_cast<size_t>(kMaxSlice) * sizeof(uint32_t)));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_row_cta_kernel, dim3(static_cast<unsigned>(a.Nq)), dim3(kHThreads),
+                      head + static_cast<size_t>(P.slice) * sizeof(uint32_t), stream, 0, P);
+  }
   const size_t smem = 2 * kBins * sizeof(int) + static_cast<size_t>(P.slice) * sizeof(uint32_t);
   // The limit is raised once, to the largest slice any launch may use.
   cudaError_t e = ensure_smem_limit<topk_cluster_kernel>(
