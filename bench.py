@@ -139,6 +139,22 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def max_over_ranks(x, dist=None, device="cpu"):
+    """The largest `x` over the ranks of the process group, on every rank (`x`
+    itself without a group): a job's device time is its slowest replica's."""
+    if not dist:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, steps, ms_total):
+    """Whole-job throughput: the units every rank processed over `steps`
+    steps, divided by the (max-over-ranks) time of those steps."""
+    return units_per_rank * world * steps / (ms_total / 1e3)
+
+
 # -------------------------------------------------------- reference arm --
 
 def run_reference(args):
@@ -337,16 +353,12 @@ def run_ours(args):
     if dist:
         dist.barrier()
     sampler.stop()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     for c in copies:
         bd.check_device_status(c.ws)
     del graphs
     ms_step = ms / args.steps
-    value = wl.Nq * world * args.steps / (ms / 1e3)
+    value = job_rate(wl.Nq, world, args.steps, ms)
 
     # --- per-kernel times: the same step as three C-ABI calls, events between them
     ktimes = kernel_times(bd, copies, wl, args.steps, dev) if not args.no_kernel_times else {
@@ -516,11 +528,7 @@ def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     bd.check_device_status(dw.ws)
     # The replayed step really moved the results: compare with a plain call.
     ref_out, ref_lse, ref_idx = dw.forward()
@@ -532,7 +540,7 @@ def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
             and np.allclose(got_out, ref_out.cpu().numpy(), rtol=0.0, atol=1e-5)):
         raise RuntimeError("e2e: the results read back differ from a direct layer call")
     del g
-    return {"value": wl.Nq * world * steps / (ms / 1e3), "unit": UNIT,
+    return {"value": job_rate(wl.Nq, world, steps, ms), "unit": UNIT,
             "h2d_bytes_per_step": int(n_in), "d2h_bytes_per_step": int(n_out),
             "ms_per_step": ms / steps,
             "method": "CUDA graph per step: one packed H2D copy, cache-row scatter, "
