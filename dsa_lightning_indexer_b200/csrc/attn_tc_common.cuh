@@ -153,7 +153,7 @@ __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
 }
 
 // Starts a bulk copy of `bytes` (a multiple of 16) of shared memory at `src`
-// to global `dst` (16-byte aligned); bulk_wait_all() waits for all of them.
+// to global `dst` (16-byte aligned).
 __device__ __forceinline__ void bulk_store_issue(void* dst, uint32_t src, uint32_t bytes) {
   asm volatile(
       "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
@@ -162,26 +162,11 @@ __device__ __forceinline__ void bulk_store_issue(void* dst, uint32_t src, uint32
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // Waits until all committed bulk copies have finished reading shared memory
 // (their global writes may still be in flight; they complete before the
 // grid does).
 __device__ __forceinline__ void bulk_wait_all_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Writes `bytes` (a multiple of 16) of shared memory at `src` to global `dst`
-// (16-byte aligned) with one bulk copy and waits until it has completed.
-__device__ __forceinline__ void bulk_store_wait(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile(
-      "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
-      "cp.async.bulk.commit_group;\n\t"
-      "cp.async.bulk.wait_group 0;" ::"l"(dst),
-      "r"(src), "r"(bytes)
-      : "memory");
 }
 
 }  // namespace attn_tc
