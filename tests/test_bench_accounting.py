@@ -1,0 +1,59 @@
+"""The benchmark's roofline arithmetic, checked against figures worked out by
+hand from the layer's definition (no GPU needed): algorithmic bytes of the
+128K decode step and of one indexer launch, causal indexer flops of the 16K
+prefill, and the kernel count of one layer call."""
+import numpy as np
+import pytest
+
+import bench
+from dsa_lightning_indexer_b200 import synth
+
+
+def _layout(lens, nq, H, top_k):
+    """A workload with the given sequence layout and zero-stride tensors (only
+    shapes and offsets matter here)."""
+    lens = np.asarray(lens, np.int64)
+    nq = np.asarray(nq, np.int64)
+    q_off = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    kv_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    Nq, rows = int(q_off[-1]), int(kv_off[-1])
+    z16 = np.uint16(0)
+    return synth.Workload("layout", q_off, kv_off, lens.astype(np.int32),
+                          np.broadcast_to(z16, (Nq, synth.HI, synth.DI)),
+                          np.broadcast_to(np.float32(0), (Nq, synth.HI)),
+                          np.broadcast_to(z16, (rows, synth.DI)),
+                          np.broadcast_to(z16, (Nq, H, synth.D)),
+                          np.broadcast_to(z16, (rows, synth.D)), top_k, synth.softmax_scale())
+
+
+def test_decode_128k_bytes():
+    wl = _layout([131072] * 4, [1] * 4, 64, 2048)
+    # indexer: every cached key's 256 bytes, plus each query's 32x128 bf16 and 32 fp32 weights
+    k1 = 4 * 131072 * 256 + 4 * (8192 + 128)
+    assert bench.indexer_bytes(wl) == k1 == 134_251_008
+    # layer: keys, 2048 gathered 1152-byte latent rows per query, and per query
+    # q (64x576 bf16), q_idx, w, out (64x512 fp32), lse, idx
+    per_q = 64 * 576 * 2 + 32 * 128 * 2 + 32 * 4 + 64 * 512 * 4 + 64 * 4 + 2048 * 4
+    total = 4 * 131072 * 256 + 4 * 2048 * 1152 + 4 * per_q
+    got = bench.decode_bytes(wl)
+    assert got["total"] == total == 144_541_184
+    assert got["total"] / 4 / 1e6 == pytest.approx(36.14, abs=0.01)  # MB per decode token
+
+
+def test_short_contexts_gather_every_row():
+    wl = _layout([1000, 3000], [1, 1], 64, 2048)
+    assert bench.decode_bytes(wl)["kv"] == (1000 + 2048) * 1152
+
+
+def test_prefill_16k_indexer_flops():
+    wl = _layout([16384], [16384], 64, 2048)
+    pairs = 16384 * 16385 // 2  # causal (query, key) pairs, own position included
+    assert bench.indexer_causal_flops(wl) == 2 * 32 * 128 * pairs
+    assert bench.indexer_causal_flops(wl) / 1e12 == pytest.approx(1.0996, abs=1e-4)
+
+
+def test_kernels_per_layer_call():
+    # decode 4 x 128K: indexer, top-k filter + emit, attention, merge of the slices
+    assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 64, 2048)) == 5
+    # prefill 16K: indexer, one top-k kernel, attention
+    assert bench.launches_per_layer(_layout([16384], [16384], 64, 2048)) == 3
