@@ -1,9 +1,12 @@
 """Comparison rules between the CUDA path and the CPU oracle.
 
-Tolerances (the reasoning is written out in the design doc):
-  * index scores: |gpu - ref| <= SCORE_RTOL * (|ref| + rms(ref row)) — fp32
-    tensor-core accumulation of 128 exact bf16 products per head, then an
-    fp32 weighted sum of 32 heads, against a double-precision reference;
+Tolerances:
+  * index scores: |gpu - ref| <= SCORE_RTOL * (|ref| + rms(ref row)).  Each
+    head's dot product sums 128 exact bf16 products in fp32 on the tensor
+    core (relative error below about 128 * 2^-24 = 8e-6 of the sum of the
+    products' magnitudes), then 32 fp32 multiply-adds weight the heads; the
+    reference is computed in double and rounded once, so 2e-5 of the score's
+    magnitude plus the row's rms covers both;
   * selected sets: identical, except for positions whose oracle score lies
     within TIE_RTOL (relative) of the oracle's k-th score; such boundary swaps
     are counted and reported;
