@@ -57,3 +57,24 @@ def test_kernels_per_layer_call():
     assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 64, 2048)) == 5
     # prefill 16K: indexer, one top-k kernel, attention
     assert bench.launches_per_layer(_layout([16384], [16384], 64, 2048)) == 3
+
+
+def test_device_glue_matches_the_chaining_definition():
+    """The bench's glue between stacked ragged layers (torch ops, run here on
+    the CPU) against the workload's host definition of the chained query."""
+    import torch
+    g = np.random.Generator(np.random.PCG64(11))
+    out = g.standard_normal((32, 64, 512)).astype(np.float32) * 0.3
+    proj = synth.glue_projection(4)
+    want = synth.bf16_to_f32(synth.chain_query(out, proj))
+    q = torch.empty(32, 64, synth.D, dtype=torch.bfloat16)
+    bench.glue_step(torch.from_numpy(out),
+                    torch.from_numpy(proj.view(np.int16)).view(torch.bfloat16), q)
+    got = q.float().numpy()
+    assert got.shape == want.shape
+    # fp32 sums in another order may round a few results to the neighbouring
+    # bf16 value (or, for results that cancel to near zero, differ by ~1e-6 of
+    # the unit-scale entries)
+    close = np.abs(got - want) <= 2.0 ** -7 * np.abs(want) + 1e-4
+    assert close.all()
+    assert (got == want).mean() > 0.99
