@@ -389,6 +389,8 @@ def run_ours(args):
     if not args.no_e2e:
         line["e2e"] = e2e_decode(bd, wl, copies[0], args.steps, max(args.warmup, 3), dev, world,
                                  dist)
+    # the oracle beside the GPU numbers, on the host cores of rank 0 at N = 1
+    args.with_oracle = rank == 0 and world == 1 and not args.no_cpu_baseline
     if not args.no_prefill:
         line["prefill"] = prefill_bench(bd, dev, peaks, args)
     if not args.no_other and world == 1:
@@ -397,12 +399,10 @@ def run_ours(args):
         other = {}
         for key, run in (("decode_B8_L32768",
                           lambda: decode_workload_bench(bd, synth.decode_b8_32k(), dev, peaks,
-                                                        50, 3)),
-                         ("ragged_B32", lambda: ragged_bench(bd, dev, peaks, 50, 3))):
-            try:
-                other[key] = run()
-            except Exception as e:  # noqa: BLE001
-                other[key] = {"error": repr(e)}
+                                                        50, 3, args.with_oracle)),
+                         ("ragged_B32", lambda: ragged_bench(bd, dev, peaks, 50, 3,
+                                                             with_oracle=args.with_oracle))):
+            other[key] = _safe(run)
             torch.cuda.empty_cache()
         line["other_workloads"] = other
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -600,15 +600,20 @@ def prefill_bench(bd, dev, peaks, args):
         k2.append(ev[1].elapsed_time(ev[2]))
         k3.append(ev[2].elapsed_time(ev[3]))
     bd.check_device_status(dw.ws)
+    del dw, out, lse, idx, scores
     fl = indexer_causal_flops(wl)
     k1s = float(np.mean(k1)) * 1e-3
     tf = fl / k1s / 1e12
-    return {"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
+    extra = {}
+    if getattr(args, "with_oracle", False):
+        extra["cpu_baseline"] = _safe(lambda: prefill_oracle(wl))
+    return {**{"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
             "steps": n, "indexer_ms": k1s * 1e3, "topk_ms": float(np.mean(k2)),
             "sparse_attn_ms": float(np.mean(k3)),
             "indexer_roofline": {"bound": "tensor", "achieved": tf,
                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                 "frac": tf / peaks["bf16_tflops"], "causal_flops": fl}}
+                                 "frac": tf / peaks["bf16_tflops"], "causal_flops": fl}},
+            **extra}
 
 
 def _graph_of(fn, dev):
@@ -642,22 +647,27 @@ def _time_flushed(g, steps, warmup, dev):
     return float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
 
-def decode_workload_bench(bd, wl, dev, peaks, steps, warmup):
+def decode_workload_bench(bd, wl, dev, peaks, steps, warmup, with_oracle=False):
     """One decode workload's layer step (a CUDA graph of dsa_layer_forward),
-    inputs resident, L2 flushed before every timed step."""
+    inputs resident, L2 flushed before every timed step; with the oracle's
+    time for the same step on the host cores beside it if asked."""
     dw = bd.DeviceWorkload(wl, dev)
     out, lse, idx = dw.new_outputs()
     g = _graph_of(lambda: dw.forward(out, lse, idx), dev)
     ms = _time_flushed(g, steps, warmup, dev)
     bd.check_device_status(dw.ws)
     del g
+    del dw, out, lse, idx
     db = decode_bytes(wl)
     gbs = db["total"] / (ms * 1e-3) / 1e9
-    return {"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
-            "steps": steps, "l2": "flushed by a 256 MB write before each timed step",
-            "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": db["total"],
-                               "achieved_gbs": gbs, "peak": peaks["hbm_gbs"],
-                               "frac": gbs / peaks["hbm_gbs"]}}
+    res = {"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
+           "steps": steps, "l2": "flushed by a 256 MB write before each timed step",
+           "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": db["total"],
+                              "achieved_gbs": gbs, "peak": peaks["hbm_gbs"],
+                              "frac": gbs / peaks["hbm_gbs"]}}
+    if with_oracle:
+        res["cpu_baseline"] = _safe(lambda: oracle_full(wl))
+    return res
 
 
 def glue_step(out, proj, q):
@@ -670,12 +680,12 @@ def glue_step(out, proj, q):
     q.copy_((x @ proj).view(q.shape))
 
 
-def ragged_bench(bd, dev, peaks, steps, warmup, layers=24):
+def ragged_bench(bd, dev, peaks, steps, warmup, layers=24, with_oracle=False):
     """The ragged serving batch (32 sequences, log-uniform contexts in
     [1024, 131072]): one layer's step, and a step of `layers` stacked layers
     with the glue between them."""
     wl = synth.ragged_layer(0)
-    res = decode_workload_bench(bd, wl, dev, peaks, steps, warmup)
+    res = decode_workload_bench(bd, wl, dev, peaks, steps, warmup, with_oracle)
     dw = bd.DeviceWorkload(wl, dev)
     out, lse, idx = dw.new_outputs()
     proj = bd.bf16_tensor(synth.glue_projection(4), dev)
@@ -699,6 +709,62 @@ def ragged_bench(bd, dev, peaks, steps, warmup, layers=24):
                   "through the glue",
         "glue": "head mean, RMS norm, bf16, x [512, 64*576] bf16 projection (torch ops)"}
     return res
+
+
+def _safe(fn):
+    """fn(), or a record of its failure: an optional measurement must not cost
+    the JSON line."""
+    try:
+        return fn()
+    except Exception as e:  # noqa: BLE001
+        return {"error": repr(e)}
+
+
+def oracle_seconds(wl, rows=None):
+    """Wall time of the oracle, as it stands, for the whole layer on `rows`
+    (every query row when None), OpenMP over the host cores; and the core count."""
+    import oracle
+    oracle.build()
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    a = (wl.q_offsets, wl.kv_offsets, wl.ctx_lens)
+    t0 = time.perf_counter()
+    oracle.dsa_layer(*a, wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv, wl.top_k, wl.scale, sample=rows)
+    return time.perf_counter() - t0, threads
+
+
+def oracle_full(wl):
+    """The oracle on every query row of `wl`, as a cpu_baseline object."""
+    dt, threads = oracle_seconds(wl)
+    return {"value": wl.Nq / dt, "unit": UNIT, "cores": min(threads, wl.Nq), "kind": "oracle",
+            "sample": f"every query row ({wl.Nq}), OpenMP over rows, {dt:.1f} s"}
+
+
+def prefill_sample_rows(n_rows, total=512, seed=2):
+    """Seeded query rows of a prefill for the oracle: every t < 64, every t in
+    [2040, 2056] (around top_k), the rest drawn uniformly without repetition."""
+    fixed = np.array([t for t in list(range(64)) + list(range(2040, 2057)) if t < n_rows])
+    rest = np.setdiff1d(np.arange(n_rows), fixed)
+    g = np.random.Generator(np.random.PCG64(seed))
+    pick = g.choice(rest, size=max(0, min(rest.size, total - fixed.size)), replace=False)
+    return np.sort(np.concatenate([fixed, pick])).astype(np.int64)
+
+
+def prefill_oracle(wl, total=512):
+    """The oracle on a seeded sample of a prefill's query rows, with the full
+    run's time extrapolated by each row's work (indexer flops over its causal
+    keys plus attention flops over its selected rows)."""
+    rows = prefill_sample_rows(wl.Nq, total)
+    dt, threads = oracle_seconds(wl, rows)
+    pos = wl.positions()
+    work = (2.0 * synth.HI * synth.DI * (pos + 1)
+            + 2.0 * wl.H * (synth.D + synth.DV) * np.minimum(wl.top_k, pos + 1))
+    full_s = dt * float(work.sum()) / float(work[rows].sum())
+    return {"value": wl.Nq / full_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows.size} seeded query rows (all t < 64, t in [2040, 2056], the rest "
+                      f"uniform) in {dt:.1f} s; value is EXTRAPOLATED to all {wl.Nq} rows "
+                      f"by per-row work",
+            "per_row_ms": dt / rows.size * 1e3, "extrapolated_full_s": full_s}
 
 
 def cpu_baseline(wl):

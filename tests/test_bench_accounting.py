@@ -78,3 +78,18 @@ def test_device_glue_matches_the_chaining_definition():
     close = np.abs(got - want) <= 2.0 ** -7 * np.abs(want) + 1e-4
     assert close.all()
     assert (got == want).mean() > 0.99
+
+
+def test_prefill_oracle_sample_and_extrapolation():
+    rows = bench.prefill_sample_rows(16384)
+    assert rows.size == 512 and np.unique(rows).size == 512
+    assert set(range(64)) | set(range(2040, 2057)) <= set(rows.tolist())
+    assert np.array_equal(rows, bench.prefill_sample_rows(16384))  # seeded
+    # on a small prefill: the extrapolation weights rows by their work, so a
+    # sample of every row extrapolates to its own time
+    wl = synth.prefill(200, 4, 32, seed=9)
+    full = bench.prefill_oracle(wl, total=200)
+    assert full["extrapolated_full_s"] == pytest.approx(full["per_row_ms"] * 200 / 1e3)
+    part = bench.prefill_oracle(wl, total=40)
+    assert part["kind"] == "oracle" and "EXTRAPOLATED" in part["sample"]
+    assert part["value"] > 0
