@@ -397,7 +397,9 @@ def run_ours(args):
         # The other decode workloads of the specification, reported beside the
         # headline (a failure here must not cost the headline line).
         other = {}
-        for key, run in (("decode_B8_L32768",
+        for key, run in (("prefill_T1024_H16", lambda: tiny_prefill_bench(bd, dev, 20, 3,
+                                                                          args.with_oracle)),
+                         ("decode_B8_L32768",
                           lambda: decode_workload_bench(bd, synth.decode_b8_32k(), dev, peaks,
                                                         50, 3, args.with_oracle)),
                          ("ragged_B32", lambda: ragged_bench(bd, dev, peaks, 50, 3,
@@ -670,6 +672,29 @@ def decode_workload_bench(bd, wl, dev, peaks, steps, warmup, with_oracle=False):
     return res
 
 
+def tiny_prefill_bench(bd, dev, steps, warmup, with_oracle=False):
+    """The 1024-token, 16-head prefill at top_k 256 and 2048 (a parity case;
+    timed for completeness), with the oracle on all host cores (and, at
+    top_k 256, on one)."""
+    res = {}
+    for k in (256, 2048):
+        wl = synth.tiny_prefill(k)
+        dw = bd.DeviceWorkload(wl, dev)
+        out, lse, idx = dw.new_outputs()
+        g = _graph_of(lambda: dw.forward(out, lse, idx), dev)
+        ms = _time_flushed(g, steps, warmup, dev)
+        bd.check_device_status(dw.ws)
+        del g, dw, out, lse, idx
+        r = {"workload": wl.name, "tokens_per_s": wl.Nq / (ms * 1e-3), "ms_per_step": ms,
+             "steps": steps, "l2": "flushed by a 256 MB write before each timed step"}
+        if with_oracle:
+            r["cpu_baseline"] = _safe(lambda: oracle_full(wl))
+            if k == 256:  # and once single-threaded
+                r["cpu_baseline_1_thread"] = _safe(lambda: oracle_full(wl, threads=1))
+        res[f"top_k_{k}"] = r
+    return res
+
+
 def glue_step(out, proj, q):
     """The stacked ragged workload's glue on the device: the next layer's
     query from this layer's output -- mean over heads, RMS-normalised,
@@ -720,12 +745,13 @@ def _safe(fn):
         return {"error": repr(e)}
 
 
-def oracle_seconds(wl, rows=None):
+def oracle_seconds(wl, rows=None, threads=None):
     """Wall time of the oracle, as it stands, for the whole layer on `rows`
-    (every query row when None), OpenMP over the host cores; and the core count."""
+    (every query row when None), OpenMP over `threads` host cores (all of
+    them when None); and the thread count."""
     import oracle
     oracle.build()
-    threads = len(os.sched_getaffinity(0))
+    threads = threads or len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
     a = (wl.q_offsets, wl.kv_offsets, wl.ctx_lens)
     t0 = time.perf_counter()
@@ -733,9 +759,9 @@ def oracle_seconds(wl, rows=None):
     return time.perf_counter() - t0, threads
 
 
-def oracle_full(wl):
+def oracle_full(wl, threads=None):
     """The oracle on every query row of `wl`, as a cpu_baseline object."""
-    dt, threads = oracle_seconds(wl)
+    dt, threads = oracle_seconds(wl, threads=threads)
     return {"value": wl.Nq / dt, "unit": UNIT, "cores": min(threads, wl.Nq), "kind": "oracle",
             "sample": f"every query row ({wl.Nq}), OpenMP over rows, {dt:.1f} s"}
 
