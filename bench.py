@@ -139,6 +139,43 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def replica_launch_cmd(argv, n):
+    """Command that runs this script as `n` ranks, one process per GPU, on
+    this node (rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+            os.path.abspath(__file__), *argv]
+
+
+def dry_run(args):
+    """The multi-rank plumbing without a GPU: gloo process group, barrier,
+    max-over-ranks of a rank-dependent time, and the JSON line's rank and
+    rate fields (launcher check)."""
+    import datetime
+    rank, _, world = env_rank()
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        dist.barrier()
+    ms = max_over_ranks(10.0 + rank, dist)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "gpus_flag": args.gpus,
+                          "ms_per_step": ms / max(1, args.steps),
+                          "value": job_rate(4, world, args.steps, ms)}), flush=True)
+    return 0
+
+
 def max_over_ranks(x, dist=None, device="cpu"):
     """The largest `x` over the ranks of the process group, on every rank (`x`
     itself without a group): a job's device time is its slowest replica's."""
@@ -336,27 +373,43 @@ def run_ours(args):
         else:
             step(i)
 
+    # Timed region: every step is replayed with the L2 flushed first (a 256 MB
+    # write, outside the step's events), so no step finds the previous one's
+    # gathered rows, partials or scores in L2; the step's device time is the
+    # sum of the per-step event intervals.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.05)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
-    e0.record()
-    for i in range(args.steps):
+    for i, (a, b) in enumerate(evs):
+        flush.fill_(i & 0xFF)
+        a.record()
         timed_step(i)
-    e1.record()
+        b.record()
     torch.cuda.synchronize()
     t1 = time.perf_counter()
     if dist:
         dist.barrier()
     sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), dist, dev)
+    # For context: the same steps back to back with no flush (two rotating copies).
+    torch.cuda.synchronize()
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record()
+    for i in range(args.steps):
+        timed_step(i)
+    w1.record()
+    torch.cuda.synchronize()
+    ms_warm = max_over_ranks(w0.elapsed_time(w1), dist, dev) / args.steps
     for c in copies:
         bd.check_device_status(c.ws)
-    del graphs
+    del graphs, flush
     ms_step = ms / args.steps
     value = job_rate(wl.Nq, world, args.steps, ms)
 
@@ -374,7 +427,11 @@ def run_ours(args):
         "data": "synthetic",
         "config": dict(config_of(wl, len(copies)),
                        launch="direct calls" if args.no_graph else "CUDA graph replay of "
-                       "dsa_layer_forward"),
+                       "dsa_layer_forward",
+                       l2="flushed by a 256 MB write before every timed step (outside its "
+                          "CUDA events); each step also streams "
+                          f"{indexer_bytes(wl) / 1e6:.0f} MB of indexer keys"),
+        "ms_per_step_back_to_back": ms_warm,
         "roofline": None if args.no_kernel_times else {"bound": "hbm", "kernel": "indexer_score", "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": profiled_traffic(), "peak_source": peaks["source"],
@@ -427,11 +484,15 @@ def kernel_times(bd, copies, wl, steps, dev):
     scores = torch.empty(wl.Nq, ld, dtype=torch.float32, device=dev)
     out, lse, idx = c0.new_outputs()
 
+    # The histogram flag makes the two calls launch exactly the layer's kernels:
+    # the indexer with its score-histogram epilogue, then the filter and emit.
+    flags = bd.FLAG_SCORE_HISTOGRAM
+
     def k1(c):
-        bd.indexer_score(c.batch, c.q_idx, c.w, c.k_idx, scores, ld, c.ws)
+        bd.indexer_score(c.batch, c.q_idx, c.w, c.k_idx, scores, ld, c.ws, flags=flags)
 
     def k2(c):
-        bd.topk(c.batch, scores, ld, c.top_k, idx, c.ws)
+        bd.topk(c.batch, scores, ld, c.top_k, idx, c.ws, flags=flags)
 
     def k3(c):
         bd.sparse_attn(c.batch, c.q, c.kv, idx, c.top_k, c.scale, out, lse, c.ws)
@@ -441,7 +502,7 @@ def kernel_times(bd, copies, wl, steps, dev):
     torch.cuda.synchronize()
     res = {}
     side = torch.cuda.Stream(dev)
-    for name, fn in (("indexer_score_us", k1), ("topk_standalone_us", k2),
+    for name, fn in (("indexer_score_us", k1), ("topk_us", k2),
                      ("sparse_attn_us", k3)):
         g = torch.cuda.CUDAGraph()
         side.wait_stream(torch.cuda.current_stream(dev))
@@ -464,8 +525,9 @@ def kernel_times(bd, copies, wl, steps, dev):
         del g
     res["launches_timed"] = n * reps
     res["method"] = "per-kernel CUDA graphs of 16 launches, CUDA events around replays"
-    res["note"] = ("each C-ABI call alone; the standalone top-k has no indexer histogram and "
-                   "takes the cluster path, the layer's takes the histogram path")
+    res["note"] = ("each C-ABI call alone, with DSA_FLAG_SCORE_HISTOGRAM: the same launches "
+                   "as inside dsa_layer_forward (indexer with its histogram epilogue; "
+                   "top-k filter and emit); inputs alternate between two copies")
     for c in copies:
         bd.check_device_status(c.ws)
     return res
@@ -829,7 +891,19 @@ def main():
                     help="launch each step directly instead of replaying a CUDA graph")
     ap.add_argument("--copies", type=int, default=2,
                     help="rotating copies of the decode inputs (L2 defeat)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="check the multi-rank launch path without a GPU (gloo)")
     args = ap.parse_args()
+    _, _, world = env_rank()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # One process per GPU: run this script again as --gpus ranks.
+        return subprocess.call(replica_launch_cmd(sys.argv[1:], args.gpus))
+    if "WORLD_SIZE" in os.environ and world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU",
+              file=sys.stderr)
+        return 2
+    if args.dry_run:
+        return dry_run(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

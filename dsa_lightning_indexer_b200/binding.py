@@ -28,7 +28,11 @@ class DsaError(RuntimeError):
 
 # status codes (dsa_status)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, \
-    ERR_NOT_SM100 = range(7)
+    ERR_NOT_SM100, ERR_BAD_INDEX = range(8)
+
+# flags
+FLAG_SCORE_HISTOGRAM = 0x1
+FLAG_TEST_STALL = 0x80000000
 
 INDEX_HEADS, INDEX_DIM, LATENT_DIM, VALUE_DIM, MAX_TOPK, MAX_HEADS = 32, 128, 576, 512, 2048, 128
 CONTROL_BYTES = 256
@@ -37,9 +41,9 @@ CONTROL_BYTES = 256
 SIGNATURES = {
     "dsa_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int, ctypes.c_int, ctypes.c_uint32]),
     "dsa_indexer_score": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_size_t,
-                                         _P]),
+                                         ctypes.c_uint32, _P]),
     "dsa_topk": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int, _P, _P, ctypes.c_size_t,
-                                _P]),
+                                ctypes.c_uint32, _P]),
     "dsa_sparse_attn": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, ctypes.c_int,
                                        ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
     "dsa_layer_forward": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
@@ -160,15 +164,15 @@ def alloc_workspace(batch: Batch, H: int, top_k: int, device="cuda") -> torch.Te
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def indexer_score(batch, q_idx, w, k_idx, scores, ld, ws, stream=None):
+def indexer_score(batch, q_idx, w, k_idx, scores, ld, ws, stream=None, flags=0):
     _check(lib.dsa_indexer_score(batch.ref, _bf16(q_idx), _f32(w), _bf16(k_idx), _f32(scores),
-                                 int(ld), _ptr(ws), ws.numel(), _stream(stream)),
+                                 int(ld), _ptr(ws), ws.numel(), int(flags), _stream(stream)),
            "dsa_indexer_score")
 
 
-def topk(batch, scores, ld, top_k, idx, ws, stream=None):
+def topk(batch, scores, ld, top_k, idx, ws, stream=None, flags=0):
     _check(lib.dsa_topk(batch.ref, _f32(scores), int(ld), int(top_k), _i32(idx), _ptr(ws),
-                        ws.numel(), _stream(stream)), "dsa_topk")
+                        ws.numel(), int(flags), _stream(stream)), "dsa_topk")
 
 
 def sparse_attn(batch, q, kv, idx, top_k, scale, out, lse, ws, stream=None):
@@ -186,11 +190,12 @@ def sparse_attn_noalloc(batch, q, kv, idx, top_k, scale, out, lse, stream=None):
            "dsa_sparse_attn_noalloc")
 
 
-def layer_forward(batch, q, q_idx, w, k_idx, kv, top_k, scale, out, lse, idx, ws, stream=None):
+def layer_forward(batch, q, q_idx, w, k_idx, kv, top_k, scale, out, lse, idx, ws, stream=None,
+                  flags=0):
     H = int(q.shape[1])
     _check(lib.dsa_layer_forward(batch.ref, _bf16(q), H, _bf16(q_idx), _f32(w), _bf16(k_idx),
                                  _bf16(kv), int(top_k), float(scale), _f32(out), _f32(lse),
-                                 _i32(idx), _ptr(ws), ws.numel(), 0, _stream(stream)),
+                                 _i32(idx), _ptr(ws), ws.numel(), int(flags), _stream(stream)),
            "dsa_layer_forward")
 
 
@@ -230,11 +235,11 @@ class DeviceWorkload:
         idx = torch.empty(self.batch.Nq, self.top_k, dtype=torch.int32, device=dev)
         return out, lse, idx
 
-    def forward(self, out=None, lse=None, idx=None, stream=None):
+    def forward(self, out=None, lse=None, idx=None, stream=None, flags=0):
         if out is None:
             out, lse, idx = self.new_outputs()
         layer_forward(self.batch, self.q, self.q_idx, self.w, self.k_idx, self.kv,
-                      self.top_k, self.scale, out, lse, idx, self.ws, stream)
+                      self.top_k, self.scale, out, lse, idx, self.ws, stream, flags)
         return out, lse, idx
 
 

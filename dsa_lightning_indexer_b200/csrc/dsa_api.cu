@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/dsa.h"
@@ -26,18 +27,7 @@ EncodeTiledFn get_encode_tiled() {
   return fn;
 }
 
-namespace {
-
-// Split planning uses a fixed SM count so workspace sizes do not depend on
-// which device (or whether any device) is present.
-constexpr int kPlanSms = 148;
-
-struct BatchInfo {
-  int64_t max_len;     // longest context
-  int64_t cache_rows;  // kv_offsets[B]
-};
-
-inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 dsa_status check_batch(const dsa_batch* b, BatchInfo* info) {
   if (!b || b->B < 0 || b->Nq < 0) return DSA_ERR_INVALID_ARG;
@@ -84,48 +74,6 @@ dsa_status check_ptr(const void* p) {
   return aligned16(p) ? DSA_OK : DSA_ERR_UNSUPPORTED;
 }
 
-// Workspace: [control 256 B][scores][top-k histograms and candidate lists]
-// [attention partials]; the middle regions exist for dsa_layer_forward only.
-struct WsLayout {
-  size_t scores_off, scores_bytes, hist_off, hist_bytes, part_off, part_bytes, total;
-  int64_t ld;
-  bool hist_topk;  // selection driven by histograms the indexer builds
-  AttnPlan plan;
-};
-
-// Few long rows with one query per sequence (decode): the indexer builds the
-// score-key histograms and the selection makes one filtering pass.
-bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
-  return b->Nq > 0 && b->Nq <= kPlanSms && info.max_len >= 8192 &&
-         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B) &&
-         topk_hist_supported(b->Nq, info.max_len);
-}
-
-inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bool scores,
-                 bool attn) {
-  WsLayout w;
-  w.ld = static_cast<int64_t>(round_up(static_cast<size_t>(info.max_len), 4));
-  w.scores_off = kControlBytes;
-  w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
-  w.hist_topk = scores && plan_hist_topk(b, info, top_k);
-  w.hist_off = w.scores_off + w.scores_bytes;
-  w.hist_bytes =
-      w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0;
-  w.part_off = w.hist_off + w.hist_bytes;
-  w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
-  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
-  w.total = w.part_off + w.part_bytes;
-  return w;
-}
-
-dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
-  if (!ws || ws_bytes < need) return DSA_ERR_WORKSPACE;
-  if (!aligned16(ws)) return DSA_ERR_UNSUPPORTED;
-  return DSA_OK;
-}
-
 // The current device must be compute capability 10.0 (B200, sm_100a code).
 dsa_status check_device(int* num_sms) {
   int dev = -1;
@@ -154,6 +102,66 @@ dsa_status check_device(int* num_sms) {
     return DSA_OK;
   }
   return DSA_ERR_NOT_SM100;
+}
+
+namespace {
+
+// Split planning uses a fixed SM count so workspace sizes do not depend on
+// which device (or whether any device) is present.
+constexpr int kPlanSms = 148;
+
+// Workspace: [control 256 B][scores][top-k histograms and candidate lists]
+// [attention partials]; the middle regions exist for dsa_layer_forward only.
+struct WsLayout {
+  size_t scores_off, scores_bytes, hist_off, hist_bytes, part_off, part_bytes, total;
+  int64_t ld;
+  bool hist_topk;  // selection driven by histograms the indexer builds
+  AttnPlan plan;
+};
+
+// Few long rows with one query per sequence (decode): the indexer builds the
+// score-key histograms and the selection makes one filtering pass.
+bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
+  return b->Nq > 0 && b->Nq <= kPlanSms && info.max_len >= 8192 &&
+         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B) &&
+         topk_hist_supported(b->Nq, info.max_len);
+}
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace bytes of the standalone calls with DSA_FLAG_SCORE_HISTOGRAM: the
+// control block, then the histogram region (the histograms and counters
+// first, the selection's lists after them).
+size_t standalone_hist_need(const dsa_batch* b, const BatchInfo& info, int top_k) {
+  return kControlBytes + round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256);
+}
+
+WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bool scores,
+                 bool attn) {
+  WsLayout w;
+  w.ld = static_cast<int64_t>(round_up(static_cast<size_t>(info.max_len), 4));
+  w.scores_off = kControlBytes;
+  w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
+  w.hist_topk = scores && plan_hist_topk(b, info, top_k);
+  w.hist_off = w.scores_off + w.scores_bytes;
+  w.hist_bytes =
+      w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0;
+  w.part_off = w.hist_off + w.hist_bytes;
+  w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
+  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
+  w.total = w.part_off + w.part_bytes;
+  // The standalone calls with DSA_FLAG_SCORE_HISTOGRAM keep the histogram
+  // region right after the control block.
+  if (scores && attn && indexer_single_query_items(b->h_q_offsets, b->B)) {
+    w.total = std::max(w.total, standalone_hist_need(b, info, top_k));
+  }
+  return w;
+}
+
+dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || ws_bytes < need) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
 }
 
 inline dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
@@ -186,7 +194,25 @@ IndexerArgs indexer_args(const dsa_batch* b, const BatchInfo& info, const uint16
   a.err = err_word(ws);
   a.num_sms = num_sms;
   a.hist = nullptr;
+  a.test_stall = false;
   return a;
+}
+
+TopkArgs topk_args(const dsa_batch* b, const BatchInfo& info, const float* scores, int64_t ld,
+                   int top_k, int32_t* idx, void* ws, int num_sms) {
+  TopkArgs t;
+  t.B = b->B;
+  t.Nq = b->Nq;
+  t.q_offsets = b->q_offsets;
+  t.ctx_lens = b->ctx_lens;
+  t.scores = scores;
+  t.ld = ld;
+  t.top_k = top_k;
+  t.idx = idx;
+  t.max_len = info.max_len;
+  t.num_sms = num_sms;
+  t.err = err_word(ws);
+  return t;
 }
 
 }  // namespace
@@ -208,47 +234,61 @@ size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t fla
 
 dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,
                              const uint16_t* k_idx, float* scores, int64_t ld_scores, void* ws,
-                             size_t ws_bytes, void* stream) {
+                             size_t ws_bytes, uint32_t flags, void* stream) {
   BatchInfo info;
   DSA_TRY(check_batch(batch, &info));
+  if ((flags & ~DSA_FLAG_SCORE_HISTOGRAM) != 0u) return DSA_ERR_INVALID_ARG;
+  const bool hist = (flags & DSA_FLAG_SCORE_HISTOGRAM) != 0u;
+  if (hist && !indexer_single_query_items(batch->h_q_offsets, batch->B)) {
+    return DSA_ERR_UNSUPPORTED;
+  }
   if (batch->Nq == 0) return DSA_OK;
   DSA_TRY(check_ptr(q_idx));
   DSA_TRY(check_ptr(w));
   DSA_TRY(check_ptr(k_idx));
   DSA_TRY(check_ptr(scores));
   if (ld_scores < info.max_len || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
-  DSA_TRY(check_ws(ws, ws_bytes, kControlBytes));
+  DSA_TRY(check_ws(ws, ws_bytes, hist ? kControlBytes + topk_hist_zero_bytes(batch->Nq)
+                                      : kControlBytes));
   int sms = 0;
   DSA_TRY(check_device(&sms));
-  return cuda_status(launch_indexer_score(
-      indexer_args(batch, info, q_idx, w, k_idx, scores, ld_scores, ws, sms),
-      static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  IndexerArgs ia = indexer_args(batch, info, q_idx, w, k_idx, scores, ld_scores, ws, sms);
+  if (hist) {
+    void* const region = static_cast<uint8_t*>(ws) + kControlBytes;
+    DSA_TRY(cuda_status(cudaMemsetAsync(region, 0, topk_hist_zero_bytes(batch->Nq), st)));
+    ia.hist = static_cast<int*>(region);
+  }
+  return cuda_status(launch_indexer_score(ia, st));
 }
 
 dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scores, int top_k,
-                    int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+                    int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags, void* stream) {
   BatchInfo info;
   DSA_TRY(check_batch(batch, &info));
   DSA_TRY(check_topk(top_k));
+  if ((flags & ~DSA_FLAG_SCORE_HISTOGRAM) != 0u) return DSA_ERR_INVALID_ARG;
   if (batch->Nq == 0) return DSA_OK;
   DSA_TRY(check_ptr(scores));
   DSA_TRY(check_ptr(idx));
   if (ld_scores < info.max_len || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
-  DSA_TRY(check_ws(ws, ws_bytes, kControlBytes));
+  // The histogram path where the fused layer would take it, given the flag.
+  const bool hist = (flags & DSA_FLAG_SCORE_HISTOGRAM) != 0u &&
+                    plan_hist_topk(batch, info, top_k);
+  DSA_TRY(check_ws(ws, ws_bytes,
+                   hist ? standalone_hist_need(batch, info, top_k) : kControlBytes));
   int sms = 0;
   DSA_TRY(check_device(&sms));
-  TopkArgs a;
-  a.B = batch->B;
-  a.Nq = batch->Nq;
-  a.q_offsets = batch->q_offsets;
-  a.ctx_lens = batch->ctx_lens;
-  a.scores = scores;
-  a.ld = ld_scores;
-  a.top_k = top_k;
-  a.idx = idx;
-  a.max_len = info.max_len;
-  a.num_sms = sms;
-  return cuda_status(launch_topk(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const TopkArgs a = topk_args(batch, info, scores, ld_scores, top_k, idx, ws, sms);
+  if (!hist) return cuda_status(launch_topk(a, st));
+  // The filter accumulates into the sub-histograms and counters that follow
+  // the histograms: clear those, so the same histograms serve every call.
+  uint8_t* const region = static_cast<uint8_t*>(ws) + kControlBytes;
+  const size_t hist_bytes = static_cast<size_t>(batch->Nq) * kHistBins * sizeof(int);
+  DSA_TRY(cuda_status(cudaMemsetAsync(region + hist_bytes, 0,
+                                      topk_hist_zero_bytes(batch->Nq) - hist_bytes, st)));
+  return cuda_status(launch_topk_hist(a, region, st));
 }
 
 dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, const uint16_t* kv,
@@ -296,8 +336,8 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
                              const uint16_t* kv, int top_k, float scale, float* out, float* lse,
                              int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags,
                              void* stream) {
-  (void)flags;
   BatchInfo info;
+  if ((flags & ~DSA_FLAG_TEST_STALL) != 0u) return DSA_ERR_INVALID_ARG;
   DSA_TRY(check_batch(batch, &info));
   DSA_TRY(check_heads(H));
   DSA_TRY(check_topk(top_k));
@@ -319,6 +359,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   float* const scores = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.scores_off);
 
   IndexerArgs ia = indexer_args(batch, info, q_idx, w, k_idx, scores, L.ld, ws, sms);
+  ia.test_stall = (flags & DSA_FLAG_TEST_STALL) != 0u;
   void* const hist_region = static_cast<uint8_t*>(ws) + L.hist_off;
   if (L.hist_topk) {
     // The histograms and counters start from zero on every call: no state is
@@ -329,17 +370,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   }
   DSA_TRY(cuda_status(launch_indexer_score(ia, st)));
 
-  TopkArgs t;
-  t.B = batch->B;
-  t.Nq = batch->Nq;
-  t.q_offsets = batch->q_offsets;
-  t.ctx_lens = batch->ctx_lens;
-  t.scores = scores;
-  t.ld = L.ld;
-  t.top_k = top_k;
-  t.idx = idx;
-  t.max_len = info.max_len;
-  t.num_sms = sms;
+  const TopkArgs t = topk_args(batch, info, scores, L.ld, top_k, idx, ws, sms);
   DSA_TRY(cuda_status(L.hist_topk ? launch_topk_hist(t, hist_region, st) : launch_topk(t, st)));
 
   AttnArgs a;
@@ -375,7 +406,7 @@ dsa_status dsa_check_device_status(void* ws, size_t ws_bytes, void* stream) {
   }
   if (host_err != 0) {
     if (cudaMemset(err_word(ws), 0, sizeof(unsigned)) != cudaSuccess) return DSA_ERR_CUDA;
-    return DSA_ERR_DEVICE_TIMEOUT;
+    return (host_err & kErrTimeout) != 0u ? DSA_ERR_DEVICE_TIMEOUT : DSA_ERR_BAD_INDEX;
   }
   return DSA_OK;
 }
@@ -389,6 +420,7 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
     case DSA_ERR_DEVICE_TIMEOUT: return "DSA_ERR_DEVICE_TIMEOUT";
     case DSA_ERR_NOT_SM100: return "DSA_ERR_NOT_SM100";
+    case DSA_ERR_BAD_INDEX: return "DSA_ERR_BAD_INDEX";
   }
   return "DSA_ERR_UNKNOWN";
 }

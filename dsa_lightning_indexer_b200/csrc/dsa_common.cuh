@@ -23,7 +23,8 @@ constexpr int kHistShift = 20;
 constexpr int kHistBins = 1 << (32 - kHistShift);
 
 // Error bits in the workspace control block.
-constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrTimeout = 1u;  // a bounded wait ran out
+constexpr unsigned kErrIndex = 2u;    // an index entry outside [-1, p] was dropped
 
 // First 256 bytes of every workspace.
 struct Control {
@@ -88,6 +89,30 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
       }
     }
   }
+}
+
+// Waits, with the same time limit but whatever the error word says, for the
+// phase of parity `parity` of `bar` to complete.  A CTA that abandoned its
+// loops calls this before it exits, so that no TMA copy or tcgen05 operation
+// it issued is still writing its shared memory or TMEM when they are handed
+// to the next CTA.  Returns false (and sets the timeout bit) if the limit
+// ran out.
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, unsigned* err) {
+  const long long t0 = clock64();
+  for (unsigned it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && clock64() - t0 > kWaitCycles) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// True when an earlier kernel recorded an error in the workspace: the
+// kernels of a call then skip their work until dsa_check_device_status
+// clears the word.  Read after the dependent-launch wait.
+__device__ __forceinline__ bool error_recorded(const unsigned* err) {
+  return err != nullptr && *reinterpret_cast<const volatile unsigned*>(err) != 0u;
 }
 
 // ----------------------------------------------------------------- TMA ----

@@ -9,7 +9,27 @@
 
 #include <atomic>
 
+#include "../../include/dsa.h"
+
 namespace dsa {
+
+// ------------------------------------------------ argument validation ----
+// Shared by every entry point; each returns DSA_OK or the status to report.
+struct BatchInfo {
+  int64_t max_len;     // longest context
+  int64_t cache_rows;  // kv_offsets[B]
+};
+bool aligned16(const void* p);
+// The batch layout (host mirrors) is consistent and within the 32-bit row
+// coordinates of the tensor maps; fills `info`.
+dsa_status check_batch(const dsa_batch* b, BatchInfo* info);
+dsa_status check_topk(int top_k);
+dsa_status check_heads(int H);
+// Non-null and 16-byte aligned.
+dsa_status check_ptr(const void* p);
+// The current device is compute capability 10.0; its SM count (cached per
+// device) goes to `num_sms`.
+dsa_status check_device(int* num_sms);
 
 struct IndexerArgs {
   int B;
@@ -26,6 +46,7 @@ struct IndexerArgs {
   unsigned* err;
   int num_sms;
   int* hist;          // per-row score-key histograms to accumulate, or null
+  bool test_stall;    // test only: the TMA producer issues nothing (every wait runs out)
 };
 // True when the indexer launch for this batch processes one query per item
 // (the only case in which it can build the histograms).
@@ -43,6 +64,7 @@ struct TopkArgs {
   int32_t* idx;
   int64_t max_len;   // longest context in the batch
   int num_sms;
+  unsigned* err;     // workspace error word: the kernels skip their work when it is set
 };
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 // Selection driven by the histograms the indexer built (see IndexerArgs.hist):

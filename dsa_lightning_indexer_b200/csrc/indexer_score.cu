@@ -55,6 +55,7 @@ struct IdxParams {
   long long ld;
   unsigned* err;
   int* hist;  // [Nq][kHistBins] score-key histograms, or null
+  int stall;  // test only: the TMA producer issues nothing, so every wait runs out
 };
 
 template <int QT>
@@ -72,7 +73,7 @@ struct Cfg {
   static constexpr int kQBytes = 2 * kQBoxBytes;
   static constexpr int kTmemCols = 2 * N < 32 ? 32 : 2 * N;
   static constexpr int kSmemData = kQBufs * kQBytes + kStages * kKTileBytes + kHistBytes;
-  static constexpr int kBarBytes = 8 * (2 * kStages + 8) + 16;
+  static constexpr int kBarBytes = 8 * (2 * kStages + 9) + 16;
   static constexpr int kSmemBytes = kSmemData + kBarBytes + 1024;
   static constexpr uint32_t kIdesc = idesc_bf16_f32(128, N);
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -133,8 +134,10 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   auto qempty = [&](int i) { return bars + 8u * (2 * C::kStages + 2 + i); };
   auto tfull = [&](int i) { return bars + 8u * (2 * C::kStages + 4 + i); };
   auto tempty = [&](int i) { return bars + 8u * (2 * C::kStages + 6 + i); };
+  const uint32_t drain = bars + 8u * (2 * C::kStages + 8);  // the MMAs' completion at exit
   uint32_t* const tmem_slot =
-      reinterpret_cast<uint32_t*>(base_ptr + C::kSmemData + 8 * (2 * C::kStages + 8));
+      reinterpret_cast<uint32_t*>(base_ptr + C::kSmemData + 8 * (2 * C::kStages + 9));
+  __shared__ int s_abort;
 
   const int warp = warp_id_uniform();
   const int lane = lane_id();
@@ -150,6 +153,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       mbar_init(tfull(i), 1);
       mbar_init(tempty(i), C::kEpiSets * kEpiThreads);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -167,14 +171,22 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   // Everything above overlapped the previous kernel; from here on memory is shared.
   pdl_wait();
   pdl_launch_dependents();
+  // An error recorded by an earlier kernel: skip the work (every role alike).
+  if (threadIdx.x == 0) s_abort = error_recorded(P.err);
+  __syncthreads();
+  const bool abort = s_abort != 0;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
-    if (lane == 0) {
+    if (lane == 0 && !abort && !P.stall) {
       const uint64_t pol_stream = l2_policy_evict_first();
       const uint64_t pol_keep = l2_policy_evict_last();
       int stage = 0, qb = 0;
       uint32_t sph = 0, qph = 0;
+      // Parity of the last load issued into each K stage and Q buffer (2: none).
+      uint32_t k_last[C::kStages], q_last[2] = {2u, 2u};
+#pragma unroll
+      for (int st = 0; st < C::kStages; ++st) k_last[st] = 2u;
       bool ok = true;
       for (int j = 0; ok; ++j) {
         const int item = snake_item(j);
@@ -184,6 +196,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         ok = mbar_wait(qempty(qb), qph ^ 1u, P.err);
         if (!ok) break;
         mbar_arrive_expect_tx(qfull(qb), C::kQBytes);
+        q_last[qb] = qph;
         const uint32_t qdst = q_smem + qb * C::kQBytes;
         tma_load_2d(qdst, &qmap, qfull(qb), 0, v.row0 * kIdxHeads, pol_keep);
         tma_load_2d(qdst + C::kQBoxBytes, &qmap, qfull(qb), 64, v.row0 * kIdxHeads, pol_keep);
@@ -195,6 +208,10 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           ok = mbar_wait(empty(stage), sph ^ 1u, P.err);
           if (!ok) break;
           mbar_arrive_expect_tx(full(stage), kKTileBytes);
+#pragma unroll
+          for (int st = 0; st < C::kStages; ++st) {
+            if (st == stage) k_last[st] = sph;
+          }
           const uint32_t kdst = k_smem + stage * kKTileBytes;
           const int row = static_cast<int>(v.kv0 + static_cast<long long>(kt) * kKeysPerTile);
           tma_load_2d(kdst, &kmap, full(stage), 0, row, pol_stream);
@@ -205,10 +222,19 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           }
         }
       }
+      // Every load issued has landed before the CTA may exit (immediate
+      // unless the loops were abandoned).
+#pragma unroll
+      for (int st = 0; st < C::kStages; ++st) {
+        if (k_last[st] != 2u) mbar_drain(full(st), k_last[st], P.err);
+      }
+      for (int i = 0; i < 2; ++i) {
+        if (q_last[i] != 2u) mbar_drain(qfull(i), q_last[i], P.err);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    if (lane == 0 && !abort) {
       int stage = 0, qb = 0, acc = 0;
       uint32_t sph = 0, qph = 0, aph = 0;
       bool ok = true;
@@ -252,6 +278,9 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           qph ^= 1u;
         }
       }
+      // Every MMA issued has completed before TMEM and the stages are released.
+      tc_commit(drain);
+      mbar_drain(drain, 0, P.err);
     }
   } else {
     // --------------------------------------------------------- epilogue --
@@ -266,7 +295,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     }
     int acc = 0;
     uint32_t aph = 0;
-    bool ok = true;
+    bool ok = !abort;
     for (int j = 0; ok; ++j) {
       const int item = snake_item(j);
       if (item >= P.n_items) break;
@@ -385,6 +414,7 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.ld = a.ld;
     P.err = a.err;
     P.hist = QT == 1 ? a.hist : nullptr;
+    P.stall = a.test_stall ? 1 : 0;
     int items = 0, n = 0;
     for (; b < a.B && n < kMaxSeqPerLaunch; ++b) {
       const int nq = a.h_q_offsets[b + 1] - a.h_q_offsets[b];

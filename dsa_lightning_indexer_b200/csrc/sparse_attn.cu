@@ -34,6 +34,8 @@ constexpr float kLn2 = 0.6931471805599453f;
 struct AttnParams {
   const int32_t* q_offsets;
   const int64_t* kv_offsets;
+  const int32_t* ctx_lens;
+  unsigned* err;        // error word for dropped index entries, or null
   const __nv_bfloat16* q;
   const __nv_bfloat16* kv;
   const int32_t* idx;
@@ -122,6 +124,9 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
   pdl_launch_dependents();
   const int b = owner_seq(P.q_offsets, P.B, r);
   const long long kv0 = P.kv_offsets[b];
+  // Causal length p + 1 of the row: only positions below it are read.
+  const int row_len = P.ctx_lens[b] - (P.q_offsets[b + 1] - P.q_offsets[b]) +
+                      (r - P.q_offsets[b]) + 1;
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
   const int slot0 = sp * P.split_len;
   const int slot1 = min(slot0 + P.split_len, P.top_k);
@@ -144,7 +149,11 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
     for (int e = tid; e < kTileRows * (kLatent / 8); e += kThreads) {
       const int i = e / (kLatent / 8), ch = e - i * (kLatent / 8);
       const int slot = s0 + i;
-      const int pos = slot < slot1 ? __ldg(idx_row + slot) : -1;
+      int pos = slot < slot1 ? __ldg(idx_row + slot) : -1;
+      if (pos < -1 || pos >= row_len) {  // outside 0..p: skipped (and recorded)
+        if (P.err != nullptr && ch == 0) atomicOr(P.err, kErrIndex);
+        pos = -1;
+      }
       if (ch == 0) tidx[buf * kTileRows + i] = pos;
       if (pos >= 0) {
         cp_async16(smem_u32(dstb + i * kRowPad + ch * 8),
@@ -491,6 +500,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   AttnParams P;
   P.q_offsets = a.q_offsets;
   P.kv_offsets = a.kv_offsets;
+  P.ctx_lens = a.ctx_lens;
+  P.err = a.err;
   P.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   P.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
   P.idx = a.idx;

@@ -44,7 +44,7 @@ constexpr int kOffKV = kOffQ + kBoxes * kQBox;
 constexpr int kOffP = kOffKV + kBoxes * kKVBox;          // [hi, lo]
 constexpr int kOffStage = 0;                             // [64][512] fp32 over Q and the tile
 constexpr int kOffBar = kOffP + 2 * kPBuf;
-constexpr int kNumBars = 5;
+constexpr int kNumBars = 6;
 constexpr int kOffTmem = kOffBar + 8 * kNumBars;
 constexpr int kOffIdx = kOffTmem + 16;                   // [64] int
 constexpr int kOffM = kOffIdx + kTD * 4;                 // [64] float
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = base + kOffQ, sKV = base + kOffKV, sP = base + kOffP;
   const uint32_t bars = base + kOffBar;
   const uint32_t b_qfull = bars, b_kvfull = bars + 8u, b_sfull = bars + 16u,
-                 b_pfull = bars + 24u, b_odone = bars + 32u;
+                 b_pfull = bars + 24u, b_odone = bars + 32u, b_drain = bars + 40u;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const rl_s = reinterpret_cast<float*>(bp + kOffL);  // 1 / row sum per head
@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(b_sfull, 1);
     mbar_init(b_pfull, kSoftThreads);
     mbar_init(b_odone, 1);
+    mbar_init(b_drain, 1);
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -122,7 +123,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ gather --
     const int g = threadIdx.x - 160;  // 0..127
     if (work) {
-      if (g < kTD) tidx[g] = slot_lo + g < n_slots ? pos_raw : -1;
+      if (g < kTD) {
+        // Only positions 0..p of the row are read; any other entry but -1 is
+        // recorded as an error and skipped.
+        int pos = slot_lo + g < n_slots ? pos_raw : -1;
+        if (pos < -1 || pos >= rs.len) {
+          atomicOr(P.err, kErrIndex);
+          pos = -1;
+        }
+        tidx[g] = pos;
+      }
       named_bar_sync(2, kGatherThreads);
       // Each thread copies whole 128-byte box rows: eight 16-byte pieces with
       // the swizzle applied.
@@ -195,6 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit_warp(b_odone);
       }
     }
+    // Nothing this warp issued (the Q load, the MMAs) may still be running
+    // when the CTA exits; immediate unless a wait above was abandoned.
+    tc_commit_warp(b_drain);
+    if (lane == 0) {
+      mbar_drain(b_drain, 0, P.err);
+      mbar_drain(b_qfull, 0, P.err);
+    }
+    __syncwarp();
   } else {
     // ----------------------------------------------------------- softmax --
     const int q = warp;

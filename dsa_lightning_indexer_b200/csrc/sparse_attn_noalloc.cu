@@ -16,10 +16,13 @@
 // their scratch lives differs.
 //
 // The first call on a device looks up the array's device address (once per
-// device, under a lock); make that first call before capturing a stream into
-// a CUDA graph.  All calls share the one array: calls whose work overlaps on
-// the GPU (two streams, or two threads on one device) race on it and must be
-// serialised by the caller.
+// device, under a lock).  Under lazy module loading (the CUDA 12 default) that
+// lookup is also when the module holding the array is loaded, so the 10 MiB
+// are committed then and the lookup can fail in a device whose memory is
+// already full: make the first call at start-up, before memory fills up and
+// before any stream is captured into a CUDA graph.  All calls share the one
+// array: calls whose work overlaps on the GPU (two streams, or two threads on
+// one device) race on it and must be serialised by the caller.
 #include <mutex>
 
 #include "../../include/dsa.h"
@@ -50,14 +53,15 @@ cudaError_t scratch_for_current_device(void** ptr) {
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // leave no sticky error for the caller's next CUDA call
+      return e;
+    }
     g_scratch_ptr[dev] = p;
   }
   *ptr = g_scratch_ptr[dev];
   return cudaSuccess;
 }
-
-bool aligned16_na(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 }  // namespace dsa
@@ -69,45 +73,24 @@ extern "C" DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, co
                                                       const int32_t* idx, int top_k,
                                                       float scale, float* out, float* lse,
                                                       void* stream) {
-  // Same argument rules as dsa_sparse_attn.
-  if (!batch || batch->B < 0 || batch->Nq < 0) return DSA_ERR_INVALID_ARG;
-  if (batch->B == 0) return batch->Nq == 0 ? DSA_OK : DSA_ERR_INVALID_ARG;
-  if (!batch->q_offsets || !batch->kv_offsets || !batch->ctx_lens || !batch->h_q_offsets ||
-      !batch->h_kv_offsets || !batch->h_ctx_lens) {
-    return DSA_ERR_INVALID_ARG;
+  // Same argument rules as dsa_sparse_attn (the same validation helpers).
+  BatchInfo info;
+  dsa_status st = check_batch(batch, &info);
+  if (st == DSA_OK) st = check_heads(H);
+  if (st == DSA_OK) st = check_topk(top_k);
+  if (st != DSA_OK || batch->Nq == 0) return st;
+  const void* ptrs[] = {q, kv, idx, out};
+  for (const void* p : ptrs) {
+    if ((st = check_ptr(p)) != DSA_OK) return st;
   }
-  if (batch->h_q_offsets[0] != 0 || batch->h_q_offsets[batch->B] != batch->Nq ||
-      batch->h_kv_offsets[0] < 0) {
-    return DSA_ERR_INVALID_ARG;
-  }
-  for (int i = 0; i < batch->B; ++i) {
-    const int64_t nq = static_cast<int64_t>(batch->h_q_offsets[i + 1]) - batch->h_q_offsets[i];
-    const int64_t cap = batch->h_kv_offsets[i + 1] - batch->h_kv_offsets[i];
-    const int64_t L = batch->h_ctx_lens[i];
-    if (nq < 0 || cap < 0 || L < 0 || nq > L || L > cap) return DSA_ERR_INVALID_ARG;
-  }
-  if (H < 1 || top_k < 1) return DSA_ERR_INVALID_ARG;
-  if (H > kMaxHeads || top_k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
-  if (batch->Nq == 0) return DSA_OK;
-  if (!q || !kv || !idx || !out) return DSA_ERR_INVALID_ARG;
-  if (!aligned16_na(q) || !aligned16_na(kv) || !aligned16_na(idx) || !aligned16_na(out) ||
-      (lse && !aligned16_na(lse))) {
-    return DSA_ERR_UNSUPPORTED;
-  }
+  if (lse && (st = check_ptr(lse)) != DSA_OK) return st;
   if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((st = check_device(&sms)) != DSA_OK) return st;
 
-  // The CUDA-core kernels and their split plan.
-  const AttnPlan plan = attn_plan_core(batch->Nq, H, top_k, 148);
+  // The CUDA-core kernels and their split plan for this device's SM count.
+  const AttnPlan plan = attn_plan_core(batch->Nq, H, top_k, sms);
   if (attn_partial_bytes(batch->Nq, H, plan) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
-
-  int dev = 0, major = 0, minor = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return DSA_ERR_NOT_SM100;
-  }
-  if (major != 10 || minor != 0) return DSA_ERR_NOT_SM100;
   void* scratch = nullptr;
   if (scratch_for_current_device(&scratch) != cudaSuccess) return DSA_ERR_CUDA;
 

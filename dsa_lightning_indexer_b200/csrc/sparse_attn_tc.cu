@@ -48,7 +48,7 @@ constexpr int kOffKV = kOffQ + kBoxes * kQBox;
 constexpr int kOffStage = kOffQ;  // output staging [64][512] fp32 over Q and the gather stages
 constexpr int kOffP = kOffKV + 2 * kKVStage;           // [stage][hi, lo]
 constexpr int kOffBar = kOffP + 4 * kPBuf;
-constexpr int kNumBars = 14;
+constexpr int kNumBars = 15;
 constexpr int kOffTmem = kOffBar + 8 * kNumBars;
 constexpr int kOffIdx = kOffTmem + 16;                  // [2][kT] int
 constexpr int kOffAlpha = kOffIdx + 2 * kT * 4;         // [64] float
@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   auto b_pfull = [&](int s) { return bars + 8u * (9 + s); };
   auto b_pempty = [&](int s) { return bars + 8u * (11 + s); };
   const uint32_t b_odone = bars + 8u * 13;
+  const uint32_t b_drain = bars + 8u * 14;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_init(b_pempty(s), 1);
     }
     mbar_init(b_odone, 1);
+    mbar_init(b_drain, 1);
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -142,7 +144,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto load_pos = [&](int t) -> int {
       if (gt >= kT || t >= n_tiles) return -1;
       const int slot = slot_lo + t * kT + gt;
-      return slot < slot_hi ? __ldg(idx_row + slot) : -1;
+      if (slot >= slot_hi) return -1;
+      const int pos = __ldg(idx_row + slot);
+      // Only positions 0..p of the row are read; any other entry but -1 is
+      // recorded as an error and skipped.
+      if (pos < -1 || pos >= rs.len) {
+        atomicOr(P.err, kErrIndex);
+        return -1;
+      }
+      return pos;
     };
     auto prefetch_row = [&](int pos) {
       if (pos >= 0) {
@@ -287,6 +297,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tc_fence_after();
       issue_pv(n_tiles - 1);
     }
+    // Nothing this warp issued (the Q load, the MMAs) may still be running
+    // when the CTA exits; immediate unless a wait above was abandoned.
+    tc_commit_warp(b_drain);
+    if (lane == 0) {
+      mbar_drain(b_drain, 0, P.err);
+      mbar_drain(b_qfull, 0, P.err);
+    }
+    __syncwarp();
   } else {
     // ----------------------------------------------------------- softmax --
     const int q = warp;                          // TMEM lane quadrant

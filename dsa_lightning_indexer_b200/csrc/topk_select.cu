@@ -53,6 +53,7 @@ struct TopkParams {
   int B;
   int top_k;
   int slice;  // keys per CTA (cluster kernel)
+  const unsigned* err;  // an earlier kernel's error: skip the work
 };
 
 // Largest b in [0, B) with q_offsets[b] <= r: the sequence that owns row r.
@@ -183,6 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_rows_kernel(const TopkParams
   __shared__ int buf[kWarps + 1];
   pdl_wait();
   pdl_launch_dependents();
+  if (error_recorded(P.err)) return;  // nothing in this kernel sets it: uniform
   const int r = blockIdx.x;
   const int b = owner_seq(P.q_offsets, P.B, r);
   const int q0 = P.q_offsets[b];
@@ -212,6 +214,7 @@ __global__ void __launch_bounds__(kCThreads) topk_cluster_kernel(const TopkParam
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
+  if (error_recorded(P.err)) return;  // the same for every CTA of the cluster
   const int r = blockIdx.x / CS;
   const int b = owner_seq(P.q_offsets, P.B, r);
   const int q0 = P.q_offsets[b];
@@ -366,6 +369,7 @@ struct HistParams {
   int* cand_pos;        // [Nq][kCandMax] their positions
   int* chunk_gt;        // [Nq][chunks][top_k] positions above the bin, per chunk
   int* chunk_ngt;       // [Nq][chunks] how many
+  const unsigned* err;  // an earlier kernel's error: skip the work
 };
 
 // Finds, among `n` shared-memory keys, the `want`-th largest key theta and how
@@ -447,6 +451,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
   pdl_launch_dependents();
+  if (error_recorded(P.err)) return;
   const int r = blockIdx.x;
   const int b = owner_seq(P.q_offsets, P.B, r);
   const int q0 = P.q_offsets[b];
@@ -639,6 +644,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_filter_kernel(const HistPar
 
   pdl_wait();
   pdl_launch_dependents();
+  if (error_recorded(P.err)) return;
   const int tid = threadIdx.x, lane = tid & 31;
   const HistRow R = hist_row(P);
   const int k = P.top_k;
@@ -775,6 +781,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_emit_kernel(const HistParam
 
   pdl_wait();
   pdl_launch_dependents();
+  if (error_recorded(P.err)) return;
   const int tid = threadIdx.x;
   const HistRow R = hist_row(P);
   const int k = P.top_k;
@@ -1008,6 +1015,7 @@ cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t st
   P.idx = a.idx;
   P.B = a.B;
   P.top_k = a.top_k;
+  P.err = a.err;
   P.chunks = topk_hist_chunks(a.Nq, a.max_len, &P.chunk);
   uint8_t* p = static_cast<uint8_t*>(ws_region);
   P.hist = reinterpret_cast<int*>(p);
@@ -1043,6 +1051,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   P.B = a.B;
   P.top_k = a.top_k;
   P.slice = 0;
+  P.err = a.err;
   const long long n_max = a.max_len;
   auto slice_of = [&](int cs) { return static_cast<long long>((n_max + cs - 1) / cs + 127) / 128 * 128; };
   // Cluster size: enough CTAs for the row to fit, more while the GPU has idle

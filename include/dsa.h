@@ -29,18 +29,25 @@
  *    except the h_* fields of dsa_batch, which are HOST mirrors used to plan
  *    the launch without a device sync.  The library allocates nothing, keeps
  *    no state between calls and is re-entrant; calls on different streams
- *    must use different workspaces.  A workspace must be zero-filled (e.g.
- *    cudaMemset) before its first use: its first 256 bytes are a control
- *    block holding the kernels' error word, which calls leave zero unless a
- *    kernel-side failure sets it, and dsa_check_device_status clears.
+ *    must use different workspaces.  The one exception is
+ *    dsa_sparse_attn_noalloc, which keeps its scratch in a static device
+ *    array shared by all of its calls (see its declaration: calls of it
+ *    that may overlap on the GPU must be serialised).  A workspace must be
+ *    zero-filled (e.g. cudaMemset) before its first use: its first 256
+ *    bytes are a control block holding the kernels' error word, which calls
+ *    leave zero unless a kernel-side failure sets it, and
+ *    dsa_check_device_status clears.
  *  - Asynchrony: all work is enqueued on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream).  Nothing synchronises except
  *    dsa_check_device_status.
  *  - Errors: every call validates all arguments before it launches anything;
  *    on any error it returns a non-OK status and writes nothing.  No C++
  *    exception crosses this boundary.  Kernel-side failures (a bounded wait
- *    that ran out) set an error word in the workspace, read back by
- *    dsa_check_device_status.
+ *    that ran out, an index entry outside 0..p) set an error word in the
+ *    workspace, read back and cleared by dsa_check_device_status.  The error
+ *    word is sticky: while it is set, the kernels of later calls on the same
+ *    workspace skip their work, and the outputs of the failing call and of
+ *    those later calls are undefined.
  *  - Alignment: every tensor pointer must be 16-byte aligned.
  *  - Fixed shapes: indexer 32 heads x 128, latent row 576, value width 512,
  *    1 <= top_k <= 2048, 1 <= H <= 128.  Other values give
@@ -76,8 +83,19 @@ typedef enum {
   DSA_ERR_WORKSPACE = 3,      /* ws NULL or smaller than the call needs */
   DSA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
   DSA_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait ran out (device side) */
-  DSA_ERR_NOT_SM100 = 6       /* current device is not compute capability 10.0 */
+  DSA_ERR_NOT_SM100 = 6,      /* current device is not compute capability 10.0 */
+  DSA_ERR_BAD_INDEX = 7       /* an index entry outside -1..p was skipped (device side) */
 } dsa_status;
+
+/* Flags (bitwise OR); every bit not listed here is reserved and must be 0. */
+/* dsa_indexer_score and dsa_topk: build, then use, the per-row histogram of
+ * the scores that the fused layer builds (see those calls). */
+#define DSA_FLAG_SCORE_HISTOGRAM 0x1u
+/* dsa_layer_forward, for tests of the timeout path only: the indexer's TMA
+ * producer issues no load, so every wait of the indexer runs out after its
+ * time limit (about a second); the call then leaves DSA_ERR_DEVICE_TIMEOUT in
+ * the workspace, and its outputs are undefined. */
+#define DSA_FLAG_TEST_STALL 0x80000000u
 
 /*
  * A batch of sequences.  Sequence b owns
@@ -119,11 +137,18 @@ DSA_API size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint
  *   scores  [Nq, ld_scores] fp32 out: scores[r, s] for s = 0..p(r);
  *                                entries past p(r) are left untouched.
  *   ld_scores >= max_b ctx_lens[b], a multiple of 4.
+ *   ws      workspace: at least 256 bytes; with DSA_FLAG_SCORE_HISTOGRAM, at
+ *           least dsa_workspace_size(batch, 1, 1, 0) bytes.
+ *   flags   0, or DSA_FLAG_SCORE_HISTOGRAM: also count every score of each
+ *           row into a 4096-bin histogram of its top 12 order-preserving key
+ *           bits, kept in the workspace for a following dsa_topk with the
+ *           same flag (as the fused layer does for decode).  Needs at most
+ *           one query per sequence (else DSA_ERR_UNSUPPORTED).
  * Runs on tcgen05 tensor cores (bf16 products, fp32 accumulation).
  */
 DSA_API dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,
                              const uint16_t* k_idx, float* scores, int64_t ld_scores, void* ws,
-                             size_t ws_bytes, void* stream);
+                             size_t ws_bytes, uint32_t flags, void* stream);
 
 /*
  * Step 2, top-k selection (aiaulis.com paragraphs 2-3: attention only for the
@@ -134,9 +159,16 @@ DSA_API dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_i
  *          lower position, written in ascending position order, followed by
  *          top_k - n entries of -1.  Positions are sequence-relative.
  *   -0.0 and +0.0 are the same score.  NaN scores are not supported.
+ *   ws     workspace: at least 256 bytes; with DSA_FLAG_SCORE_HISTOGRAM, at
+ *          least dsa_workspace_size(batch, 1, top_k, 0) bytes.
+ *   flags  0, or DSA_FLAG_SCORE_HISTOGRAM: the histograms that the preceding
+ *          dsa_indexer_score call with that flag left in this workspace, for
+ *          these same scores, drive the selection (one filtering pass over
+ *          each row) wherever few long rows make that path pay; the result
+ *          is the same either way.
  */
 DSA_API dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scores, int top_k,
-                    int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+                    int32_t* idx, void* ws, size_t ws_bytes, uint32_t flags, void* stream);
 
 /*
  * Step 3, attention over the selected rows only (aiaulis.com paragraph 2;
@@ -144,7 +176,11 @@ DSA_API dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t
  *   q    [Nq, H, 576] bf16     attention queries
  *   kv   [rows, 576]  bf16     shared latent cache; V = first 512 entries
  *   idx  [Nq, top_k]  int32    sequence-relative positions, -1 = unused slot;
- *                              every other entry must satisfy 0 <= idx <= p(r)
+ *                              every other entry must satisfy 0 <= idx <= p(r):
+ *                              an entry outside -1..p(r) is checked on the
+ *                              device, skipped (no memory is read for it) and
+ *                              reported as DSA_ERR_BAD_INDEX by
+ *                              dsa_check_device_status
  *   out  [Nq, H, 512] fp32     out: softmax_s(scale * q.kv[s]) weighted sum of
  *                              kv[s, :512] over the listed s
  *   lse  [Nq, H] fp32 or NULL  out: natural-log log-sum-exp of the logits
@@ -157,8 +193,8 @@ DSA_API dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, in
 /*
  * The whole DSA layer: dsa_indexer_score -> dsa_topk -> dsa_sparse_attn,
  * with the scores kept in the workspace.  Arguments as above; `idx` receives
- * the selected index sets, `out`/`lse` the attention output.  `flags` is
- * reserved, pass 0.
+ * the selected index sets, `out`/`lse` the attention output.  `flags` is 0
+ * (or DSA_FLAG_TEST_STALL, in tests of the timeout path only).
  */
 DSA_API dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
                              const uint16_t* q_idx, const float* w, const uint16_t* k_idx,
@@ -180,11 +216,16 @@ DSA_API dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, 
  * returns DSA_ERR_WORKSPACE and runs nothing (no shape within the fixed limits
  * needs more than about 9.3 MiB).  It allocates nothing and calls no
  * allocating routine.  The first call on each device looks up the array's
- * address; make it before capturing a stream into a CUDA graph.  Calls share
+ * address, which under lazy module loading (the CUDA 12 default) also loads
+ * the module and commits the array's memory: make that first call at
+ * start-up, before device memory fills up and before capturing a stream into
+ * a CUDA graph (a failed lookup returns DSA_ERR_CUDA).  Calls share
  * the array: calls that may overlap on the GPU (different streams) race and
  * must be serialised by the caller.  It always runs the CUDA-core attention
  * kernels, so results agree with dsa_sparse_attn within the library's
- * tolerances (not bit for bit).
+ * tolerances (not bit for bit).  Index entries outside -1..p(r) are skipped
+ * as in dsa_sparse_attn, but with no workspace there is no error word to
+ * report them in.
  */
 DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, const uint16_t* q, int H,
                                            const uint16_t* kv, const int32_t* idx, int top_k,
@@ -192,8 +233,9 @@ DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, const uint16_
 
 /* Synchronises `stream`, then reads and clears the device error word that the
  * kernels of earlier calls on this workspace may have set.  Returns DSA_OK,
- * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the stream itself reports an
- * error. */
+ * DSA_ERR_DEVICE_TIMEOUT (a bounded wait ran out; takes precedence),
+ * DSA_ERR_BAD_INDEX (an index entry outside -1..p was skipped), or
+ * DSA_ERR_CUDA if the stream itself reports an error. */
 DSA_API dsa_status dsa_check_device_status(void* ws, size_t ws_bytes, void* stream);
 
 /* Static, human-readable name of a status code. */

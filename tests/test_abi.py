@@ -36,8 +36,8 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     names = ["DSA_OK", "DSA_ERR_INVALID_ARG", "DSA_ERR_UNSUPPORTED", "DSA_ERR_WORKSPACE",
-             "DSA_ERR_CUDA", "DSA_ERR_DEVICE_TIMEOUT", "DSA_ERR_NOT_SM100"]
-    assert [bd.status_string(i) for i in range(7)] == names
+             "DSA_ERR_CUDA", "DSA_ERR_DEVICE_TIMEOUT", "DSA_ERR_NOT_SM100", "DSA_ERR_BAD_INDEX"]
+    assert [bd.status_string(i) for i in range(8)] == names
     assert bd.status_string(99) == "DSA_ERR_UNKNOWN"
 
 
@@ -57,8 +57,8 @@ class FakeBatch:
         return ctypes.byref(self.c)
 
 
-def _topk(b, top_k=16, scores=FAKE, ld=64, idx=FAKE, ws=FAKE, ws_bytes=1 << 20):
-    return bd.lib.dsa_topk(b.ref, scores, ld, top_k, idx, ws, ws_bytes, None)
+def _topk(b, top_k=16, scores=FAKE, ld=64, idx=FAKE, ws=FAKE, ws_bytes=1 << 20, flags=0):
+    return bd.lib.dsa_topk(b.ref, scores, ld, top_k, idx, ws, ws_bytes, flags, None)
 
 
 def _attn(b, H=16, top_k=16, q=FAKE, kv=FAKE, idx=FAKE, scale=0.04, out=FAKE, lse=None,
@@ -82,7 +82,7 @@ def test_batch_validation():
         assert bd.lib.dsa_workspace_size(b.ref, 16, 16, 0) == 0
         assert _topk(b) == bd.ERR_INVALID_ARG
         assert _attn(b) == bd.ERR_INVALID_ARG
-    assert bd.lib.dsa_topk(None, FAKE, 64, 16, FAKE, FAKE, 1 << 20, None) == bd.ERR_INVALID_ARG
+    assert bd.lib.dsa_topk(None, FAKE, 64, 16, FAKE, FAKE, 1 << 20, 0, None) == bd.ERR_INVALID_ARG
 
 
 def test_shape_and_pointer_validation():
@@ -100,7 +100,7 @@ def test_shape_and_pointer_validation():
     assert _attn(b, scale=float("nan")) == bd.ERR_INVALID_ARG
     assert _attn(b, lse=FAKE + 8) == bd.ERR_UNSUPPORTED
     assert _attn(b, ws_bytes=16) == bd.ERR_WORKSPACE
-    st = bd.lib.dsa_indexer_score(b.ref, FAKE, FAKE, FAKE, FAKE, 60, FAKE, 1 << 20, None)
+    st = bd.lib.dsa_indexer_score(b.ref, FAKE, FAKE, FAKE, FAKE, 60, FAKE, 1 << 20, 0, None)
     assert st == bd.ERR_INVALID_ARG
     st = bd.lib.dsa_layer_forward(b.ref, FAKE, 16, FAKE, FAKE, FAKE, FAKE, 16, 0.04, FAKE,
                                   None, None, FAKE, 1 << 30, 0, None)
@@ -126,3 +126,38 @@ def test_workspace_grows_with_the_problem():
 def test_valid_call_without_a_b200_is_refused():
     b = FakeBatch([0, 1], [0, 64], [64])
     assert _topk(b) == bd.ERR_NOT_SM100
+
+
+def test_flag_validation():
+    b = FakeBatch([0, 1], [0, 64], [64])
+    multi = FakeBatch([0, 2], [0, 64], [64])                    # two queries in one sequence
+    hist, stall = bd.FLAG_SCORE_HISTOGRAM, bd.FLAG_TEST_STALL
+
+    def score(batch, flags):
+        return bd.lib.dsa_indexer_score(batch.ref, FAKE, FAKE, FAKE, FAKE, 64, FAKE, 1 << 20,
+                                        flags, None)
+
+    def layer(flags):
+        return bd.lib.dsa_layer_forward(b.ref, FAKE, 16, FAKE, FAKE, FAKE, FAKE, 16, 0.04, FAKE,
+                                        None, FAKE, FAKE, 1 << 30, flags, None)
+    assert score(b, 0x2) == bd.ERR_INVALID_ARG                 # reserved bit
+    assert score(b, stall) == bd.ERR_INVALID_ARG               # a layer-only flag
+    assert score(multi, hist) == bd.ERR_UNSUPPORTED            # histogram: one query per sequence
+    assert _topk(b, flags=0x4) == bd.ERR_INVALID_ARG
+    assert _topk(b, flags=stall) == bd.ERR_INVALID_ARG
+    assert layer(hist) == bd.ERR_INVALID_ARG                   # the layer builds it itself
+    assert layer(0x10) == bd.ERR_INVALID_ARG
+    # workspace checks come before the device check: too small for the histograms
+    assert bd.lib.dsa_indexer_score(b.ref, FAKE, FAKE, FAKE, FAKE, 64, FAKE, 300, hist,
+                                    None) == bd.ERR_WORKSPACE
+
+
+def test_workspace_covers_the_standalone_histogram_region():
+    # a decode batch long enough for the histogram-driven selection
+    b = FakeBatch([0, 1, 2], [0, 40000, 60000], [40000, 20000])
+    size = bd.lib.dsa_workspace_size(b.ref, 16, 2048, 0)
+    hist_zero = 2 * (4096 + 2048 + 4) * 4
+    assert size >= 256 + hist_zero
+    st = bd.lib.dsa_topk(b.ref, FAKE, 40000, 2048, FAKE, FAKE, 256 + hist_zero,
+                         bd.FLAG_SCORE_HISTOGRAM, None)
+    assert st == bd.ERR_WORKSPACE                              # needs the lists too

@@ -78,3 +78,34 @@ def test_packed_buffers_are_aligned_and_disjoint():
     assert all(o % 256 == 0 for o in offs.values())
     assert offs == {"a": 0, "b": 256, "c": 512, "d": 768, "e": 768}
     assert total == 768 + 512
+
+
+def test_gpus_flag_launches_one_rank_per_gpu():
+    """`bench.py --gpus 2` without WORLD_SIZE re-runs itself as two ranks
+    (torch.distributed.run, rendezvous on 127.0.0.1); the line reports both."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--steps", "5", "--dry-run"], env=env, capture_output=True,
+                         text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["gpus_flag"] == 2
+    assert line["ms_per_step"] == pytest.approx(11.0 / 5)   # the slower rank's time
+    assert line["value"] == pytest.approx(4 * 2 * 5 / 0.011)
+
+
+def test_gpus_flag_must_match_the_launch():
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                          "--dry-run"], env=env, capture_output=True, text=True, timeout=120)
+    assert out.returncode == 2 and "WORLD_SIZE=3" in out.stderr

@@ -1,17 +1,18 @@
-"""dsa_sparse_attn_noalloc against dsa_sparse_attn (needs a B200).
+"""dsa_sparse_attn_noalloc against the oracle and dsa_sparse_attn (needs a B200).
 
 The no-allocation entry point is for callers that cannot call cudaMalloc when
 they run the layer (a fixed memory pool, a runtime that only hands kernels
 its own tensors).  It keeps its scratch in a static device array instead of
-a caller workspace.  Its results must agree with the workspace entry point on
-the same inputs, on two calls in a row (the array keeps the previous call's
-contents, which must not leak into the next result).
+a caller workspace, and that array keeps whatever the previous call left in
+it.  So before each checked call another call with a different split (more
+rows, 128 heads, other inputs) fills most of the array; if a checked call
+read any slot it did not write itself, it would pick up the filler's values.
+Each checked call is compared with the CPU oracle directly, and with the
+workspace entry point on the same inputs, on two calls in a row.
 
 This file is named to be collected last, so a run that stops at the first
 failure has already run every other test.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -38,24 +39,43 @@ CASES = {
 }
 
 
+def _filler():
+    """18 decode rows x 128 heads with random index sets: a split whose
+    partials cover about 9.5 MiB of the 10 MiB array."""
+    wl = synth.custom([2100 + 37 * i for i in range(18)], [1] * 18, 128, 2048, seed=152)
+    g = np.random.Generator(np.random.PCG64(153))
+    idx = np.stack([np.sort(g.choice(int(L), size=2048, replace=False)) for L in wl.ctx_lens])
+    dw = bd.DeviceWorkload(wl)
+    return dw, torch.from_numpy(idx.astype(np.int32)).cuda()
+
+
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_noalloc_matches_workspace_entry_point(name):
+def test_noalloc_matches_oracle_and_workspace_entry_point(name):
     wl = CASES[name]()
     _, idx_np, _, _ = oracle.dsa_layer(*_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q, wl.kv,
                                        wl.top_k, wl.scale)
+    ora_out, ora_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, idx_np, wl.scale)
     dw = bd.DeviceWorkload(wl)
     idx = torch.from_numpy(idx_np).cuda()
     ref_out = torch.empty(wl.Nq, wl.H, 512, device="cuda")
     ref_lse = torch.empty(wl.Nq, wl.H, device="cuda")
     bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, ref_out, ref_lse, dw.ws)
     ref_out, ref_lse = ref_out.cpu().numpy(), ref_lse.cpu().numpy()
+
+    fill, fill_idx = _filler()
+    fill_out = torch.empty(fill.batch.Nq, fill.H, 512, device="cuda")
+    fill_lse = torch.empty(fill.batch.Nq, fill.H, device="cuda")
     runs = []
     for _ in range(2):
+        bd.sparse_attn_noalloc(fill.batch, fill.q, fill.kv, fill_idx, 2048, fill.scale,
+                               fill_out, fill_lse)
         out = torch.full((wl.Nq, wl.H, 512), float("nan"), device="cuda")
         lse = torch.full((wl.Nq, wl.H), float("nan"), device="cuda")
         bd.sparse_attn_noalloc(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, out, lse)
         torch.cuda.synchronize()
         runs.append((out.cpu().numpy(), lse.cpu().numpy()))
+    assert torch.isfinite(fill_out).all().item()
     for out, lse in runs:
-        parity.check_attention(out, lse, ref_out, ref_lse.astype(np.float64))
+        parity.check_attention(out, lse, ora_out, ora_lse)                       # the oracle
+        parity.check_attention(out, lse, ref_out, ref_lse.astype(np.float64))    # workspace call
     assert np.array_equal(runs[0][0], runs[1][0]) and np.array_equal(runs[0][1], runs[1][1])
