@@ -273,10 +273,12 @@ def indexer_causal_flops(wl):
 
 def launches_per_layer(wl, sms=148):
     """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
-    sequences with queries); the top-k selection, which is two kernels (filter
-    and emit) when few long single-query rows take the histogram path, else
-    one; the sparse attention and, when few rows split the selected set over
-    CTAs, the merge of the slices."""
+    sequences with queries), then either the fused decode tail (selection,
+    attention and merge in one kernel: few long single-query rows, at most 64
+    heads), or the top-k selection -- two kernels (filter and emit) when the
+    indexer's histograms drive it, else one -- followed by the sparse
+    attention and, when few rows split the selected set over CTAs, the merge
+    of the slices."""
     nq = np.diff(wl.q_offsets)
     seqs = int((nq > 0).sum())
     max_len = int(wl.ctx_lens.max()) if wl.B else 0
@@ -285,6 +287,11 @@ def launches_per_layer(wl, sms=148):
     chunk = min(max(512, -(-per // 512) * 512), 8192)
     hist = (0 < wl.Nq <= 148 and max_len >= 8192 and max_len >= 4 * wl.top_k
             and int(nq.max()) <= 1 and -(-max_len // chunk) <= 512)
+    C = 148 // max(1, wl.Nq)
+    fused = (hist and wl.H <= 64 and wl.Nq <= 16 and C >= 8
+             and (-(-max_len // C) + 31) // 32 <= 512)
+    if fused:
+        return (seqs + 63) // 64 + 1
     few_rows = wl.Nq * ((wl.H + 63) // 64) < sms
     return (seqs + 63) // 64 + (2 if hist else 1) + 1 + (1 if few_rows and wl.top_k > 16 else 0)
 
@@ -543,86 +550,124 @@ def _packed(parts, align=256):
 
 
 def e2e_decode(bd, wl, dw, steps, warmup, dev, world, dist):
-    """Decode step through host buffers: the step's new inputs (queries, indexer
-    queries and weights, and the new token's rows of both caches) arrive in one
-    copy from pinned host memory, the cache rows are scattered into the
-    resident caches, the layer runs, and its output, log-sum-exp and index sets
-    leave in one copy into pinned host memory.  The step is captured once as a
-    CUDA graph (copies included) and replayed, as a serving loop would."""
+    """Decode steps through host buffers, as a serving loop overlaps them: each
+    step's new inputs (queries, indexer queries and weights, and the new
+    token's rows of both caches) arrive in one copy from pinned host memory,
+    the cache rows are scattered into the resident caches, the layer runs,
+    and its output, log-sum-exp and index sets leave in one copy into pinned
+    host memory.  Two buffer sets alternate, and the uploads and downloads run
+    on their own streams, so one step's copies overlap the neighbouring
+    steps' compute (the scatter and the layer stay in order on the compute
+    stream).  G steps are captured as one CUDA graph and replayed."""
     new_rows = [int(wl.kv_offsets[b] + wl.ctx_lens[b] - 1) for b in range(wl.B)]
     host_in = {"q": wl.q, "q_idx": wl.q_idx, "w": wl.w,
                "krow": wl.k_idx[new_rows], "vrow": wl.kv[new_rows]}
     offs, n_in = _packed([(k, v.nbytes) for k, v in host_in.items()])
-    h_in = torch.empty(n_in, dtype=torch.uint8).pin_memory()
-    hv = h_in.numpy()
-    for k, v in host_in.items():
-        hv[offs[k]:offs[k] + v.nbytes] = np.ascontiguousarray(v).view(np.uint8).ravel()
-    d_in = torch.empty(n_in, dtype=torch.uint8, device=dev)
+    Nq, H, top_k = wl.Nq, wl.H, wl.top_k
+    oo, n_out = _packed([("out", Nq * H * 512 * 4), ("lse", Nq * H * 4), ("idx", Nq * top_k * 4)])
 
     def dview(buf, o, shape, dtype):
         nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
         return buf[o:o + nbytes].view(dtype).view(*shape)
 
-    q = dview(d_in, offs["q"], wl.q.shape, torch.bfloat16)
-    q_idx = dview(d_in, offs["q_idx"], wl.q_idx.shape, torch.bfloat16)
-    w = dview(d_in, offs["w"], wl.w.shape, torch.float32)
-    krow = dview(d_in, offs["krow"], host_in["krow"].shape, torch.int16)
-    vrow = dview(d_in, offs["vrow"], host_in["vrow"].shape, torch.int16)
+    sets = []
+    for _ in range(2):
+        h_in = torch.empty(n_in, dtype=torch.uint8).pin_memory()
+        hv = h_in.numpy()
+        for k, v in host_in.items():
+            hv[offs[k]:offs[k] + v.nbytes] = np.ascontiguousarray(v).view(np.uint8).ravel()
+        d_in = torch.empty(n_in, dtype=torch.uint8, device=dev)
+        d_out = torch.empty(n_out, dtype=torch.uint8, device=dev)
+        sets.append({
+            "h_in": h_in, "d_in": d_in, "d_out": d_out,
+            "h_out": torch.empty(n_out, dtype=torch.uint8).pin_memory(),
+            "q": dview(d_in, offs["q"], wl.q.shape, torch.bfloat16),
+            "q_idx": dview(d_in, offs["q_idx"], wl.q_idx.shape, torch.bfloat16),
+            "w": dview(d_in, offs["w"], wl.w.shape, torch.float32),
+            "krow": dview(d_in, offs["krow"], host_in["krow"].shape, torch.int16),
+            "vrow": dview(d_in, offs["vrow"], host_in["vrow"].shape, torch.int16),
+            "out": dview(d_out, oo["out"], (Nq, H, 512), torch.float32),
+            "lse": dview(d_out, oo["lse"], (Nq, H), torch.float32),
+            "idx": dview(d_out, oo["idx"], (Nq, top_k), torch.int32),
+        })
     rows = torch.tensor(new_rows, dtype=torch.long, device=dev)
     k16, v16 = dw.k_idx.view(torch.int16), dw.kv.view(torch.int16)
+    s_comp, s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("up", "comp", "down")}
+    G = max(g for g in range(1, 9) if steps % g == 0)  # steps per captured graph
 
-    Nq, H, top_k = wl.Nq, wl.H, wl.top_k
-    oo, n_out = _packed([("out", Nq * H * 512 * 4), ("lse", Nq * H * 4), ("idx", Nq * top_k * 4)])
-    d_out = torch.empty(n_out, dtype=torch.uint8, device=dev)
-    h_out = torch.empty(n_out, dtype=torch.uint8).pin_memory()
-    out = dview(d_out, oo["out"], (Nq, H, 512), torch.float32)
-    lse = dview(d_out, oo["lse"], (Nq, H), torch.float32)
-    idx = dview(d_out, oo["idx"], (Nq, top_k), torch.int32)
+    def enqueue(i, first):
+        b = i & 1
+        st = sets[b]
+        with torch.cuda.stream(s_up):
+            if not first:
+                s_up.wait_event(ev["comp"][b])   # the layer that read this buffer is done
+            st["d_in"].copy_(st["h_in"], non_blocking=True)
+            ev["up"][b].record(s_up)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev["up"][b])
+            if not first:
+                s_comp.wait_event(ev["down"][b])  # this output buffer has been read out
+            k16.index_copy_(0, rows, st["krow"])
+            v16.index_copy_(0, rows, st["vrow"])
+            bd.layer_forward(dw.batch, st["q"], st["q_idx"], st["w"], dw.k_idx, dw.kv, top_k,
+                             wl.scale, st["out"], st["lse"], st["idx"], dw.ws)
+            ev["comp"][b].record(s_comp)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev["comp"][b])
+            st["h_out"].copy_(st["d_out"], non_blocking=True)
+            ev["down"][b].record(s_down)
 
-    def step():
-        d_in.copy_(h_in, non_blocking=True)
-        k16.index_copy_(0, rows, krow)
-        v16.index_copy_(0, rows, vrow)
-        bd.layer_forward(dw.batch, q, q_idx, w, dw.k_idx, dw.kv, top_k, wl.scale,
-                         out, lse, idx, dw.ws)
-        h_out.copy_(d_out, non_blocking=True)
+    cur = torch.cuda.current_stream(dev)
 
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        step()
+    def capture():
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
-            step()
-    torch.cuda.current_stream().wait_stream(s)
-    for _ in range(warmup):
+        for s_ in (s_comp, s_up, s_down):
+            s_.wait_stream(cur)
+        with torch.cuda.graph(g, stream=s_comp):
+            s_up.wait_stream(s_comp)
+            s_down.wait_stream(s_comp)
+            for i in range(G):
+                enqueue(i, first=i < 2)
+            s_comp.wait_stream(s_up)
+            s_comp.wait_stream(s_down)
+        cur.wait_stream(s_comp)
+        return g
+
+    for i in range(2):  # eager warm-up (lazy initialisation before capture)
+        enqueue(i, first=True)
+    torch.cuda.synchronize()
+    g = capture()
+    for _ in range(max(1, warmup // G + 1)):
         g.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(steps):
+    for _ in range(steps // G):
         g.replay()
     e1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     bd.check_device_status(dw.ws)
-    # The replayed step really moved the results: compare with a plain call.
+    # The replayed steps really moved the results: compare with a plain call.
     ref_out, ref_lse, ref_idx = dw.forward()
     torch.cuda.synchronize()
-    hb = h_out.numpy()
-    got_idx = hb[oo["idx"]:oo["idx"] + Nq * top_k * 4].view(np.int32).reshape(Nq, top_k)
-    got_out = hb[oo["out"]:oo["out"] + Nq * H * 512 * 4].view(np.float32).reshape(Nq, H, 512)
-    if not (np.array_equal(got_idx, ref_idx.cpu().numpy())
-            and np.allclose(got_out, ref_out.cpu().numpy(), rtol=0.0, atol=1e-5)):
-        raise RuntimeError("e2e: the results read back differ from a direct layer call")
+    for st in sets:
+        hb = st["h_out"].numpy()
+        got_idx = hb[oo["idx"]:oo["idx"] + Nq * top_k * 4].view(np.int32).reshape(Nq, top_k)
+        got_out = hb[oo["out"]:oo["out"] + Nq * H * 512 * 4].view(np.float32).reshape(Nq, H, 512)
+        if not (np.array_equal(got_idx, ref_idx.cpu().numpy())
+                and np.allclose(got_out, ref_out.cpu().numpy(), rtol=0.0, atol=1e-5)):
+            raise RuntimeError("e2e: the results read back differ from a direct layer call")
     del g
     return {"value": job_rate(wl.Nq, world, steps, ms), "unit": UNIT,
             "h2d_bytes_per_step": int(n_in), "d2h_bytes_per_step": int(n_out),
-            "ms_per_step": ms / steps,
-            "method": "CUDA graph per step: one packed H2D copy, cache-row scatter, "
-                      "dsa_layer_forward, one packed D2H copy"}
+            "ms_per_step": ms / steps, "steps_per_graph": G,
+            "method": "two buffer sets; per step one packed H2D copy (upload stream), cache-row "
+                      "scatter and dsa_layer_forward (compute stream), one packed D2H copy "
+                      "(download stream); G steps per CUDA graph, replayed"}
 
 
 def prefill_bench(bd, dev, peaks, args):
@@ -758,43 +803,61 @@ def tiny_prefill_bench(bd, dev, steps, warmup, with_oracle=False):
 
 
 def glue_step(out, proj, q):
-    """The stacked ragged workload's glue on the device: the next layer's
-    query from this layer's output -- mean over heads, RMS-normalised,
+    """The stacked ragged workload's glue on the device, in fp32: the next
+    layer's query from this layer's output -- mean over heads, RMS-normalised,
     rounded to bf16, times the fixed bf16 projection, rounded to bf16."""
-    m = out.double().mean(dim=1)
+    m = out.mean(dim=1)
     m = m * torch.rsqrt((m * m).mean(dim=1, keepdim=True) + 1e-6)
-    x = m.float().to(torch.bfloat16)
-    q.copy_((x @ proj).view(q.shape))
+    q.copy_((m.to(torch.bfloat16) @ proj).view(q.shape))
 
 
 def ragged_bench(bd, dev, peaks, steps, warmup, layers=24, with_oracle=False):
     """The ragged serving batch (32 sequences, log-uniform contexts in
-    [1024, 131072]): one layer's step, and a step of `layers` stacked layers
-    with the glue between them."""
-    wl = synth.ragged_layer(0)
-    res = decode_workload_bench(bd, wl, dev, peaks, steps, warmup, with_oracle)
-    dw = bd.DeviceWorkload(wl, dev)
-    out, lse, idx = dw.new_outputs()
+    [1024, 131072]): one layer's step, and a step of `layers` stacked layers,
+    each with its own seeded caches and indexer inputs, with the glue between
+    them (the last layer's output feeds the first layer's query of the next
+    step)."""
+    wl0 = synth.ragged_layer(0)
+    res = decode_workload_bench(bd, wl0, dev, peaks, steps, warmup, with_oracle)
+    t0 = time.perf_counter()
+    dws, layer_bytes = [], 0
+    for layer in range(layers):
+        wl = wl0 if layer == 0 else synth.ragged_layer(layer)
+        dw = bd.DeviceWorkload(wl, dev)
+        dw.wl = None  # the host arrays are not needed once the inputs are on the device
+        layer_bytes += decode_bytes(wl)["total"]
+        if layer > 0:
+            del dw.ws  # one workspace serves every layer (same batch, calls in order)
+        dws.append(dw)
+        del wl
+    draw_s = time.perf_counter() - t0
+    ws = dws[0].ws
+    out, lse, idx = dws[0].new_outputs()
     proj = bd.bf16_tensor(synth.glue_projection(4), dev)
 
     def stack():
-        for _ in range(layers):
-            dw.forward(out, lse, idx)
-            glue_step(out, proj, dw.q)
+        for layer, dw in enumerate(dws):
+            bd.layer_forward(dw.batch, dw.q, dw.q_idx, dw.w, dw.k_idx, dw.kv, dw.top_k,
+                             dw.scale, out, lse, idx, ws)
+            glue_step(out, proj, dws[(layer + 1) % layers].q)
 
     g = _graph_of(stack, dev)
     n = max(3, steps // 10)
     ms = _time_flushed(g, n, min(warmup, 3), dev)
-    bd.check_device_status(dw.ws)
-    del g
+    bd.check_device_status(ws)
+    del g, dws, ws, out, lse, idx
+    gbs = layer_bytes / (ms * 1e-3) / 1e9
     res["stack"] = {
         "layers": layers, "ms_per_step": ms, "steps": n,
-        "tokens_per_s": wl.Nq / (ms * 1e-3),
+        "tokens_per_s": wl0.Nq / (ms * 1e-3),
         "ms_per_layer_with_glue": ms / layers,
-        "inputs": "layer 0's caches and indexer inputs serve every layer (drawing all "
-                  "24 layers' inputs takes the host minutes); the main query chains "
-                  "through the glue",
-        "glue": "head mean, RMS norm, bf16, x [512, 64*576] bf16 projection (torch ops)"}
+        "inputs": f"{layers} layers, each with its own seeded caches, indexer inputs and "
+                  f"weights (drawn in {draw_s:.0f} s); the main query chains through the glue",
+        "glue": "head mean, RMS norm, bf16, x [512, 64*576] bf16 projection (torch ops, fp32)",
+        "layer_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": layer_bytes,
+                           "achieved_gbs": gbs, "peak": peaks["hbm_gbs"],
+                           "frac": gbs / peaks["hbm_gbs"],
+                           "note": "layers' algorithmic bytes only; glue time included"}}
     return res
 
 

@@ -115,7 +115,8 @@ constexpr int kPlanSms = 148;
 struct WsLayout {
   size_t scores_off, scores_bytes, hist_off, hist_bytes, part_off, part_bytes, total;
   int64_t ld;
-  bool hist_topk;  // selection driven by histograms the indexer builds
+  bool hist_topk;   // selection driven by histograms the indexer builds
+  bool fused_tail;  // ... and everything after the indexer in one kernel
   AttnPlan plan;
 };
 
@@ -143,12 +144,15 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.scores_off = kControlBytes;
   w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
   w.hist_topk = scores && plan_hist_topk(b, info, top_k);
+  w.fused_tail = w.hist_topk && attn && decode_tail_supported(b->Nq, H, info.max_len, kPlanSms);
   w.hist_off = w.scores_off + w.scores_bytes;
   w.hist_bytes =
-      w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0;
+      w.fused_tail
+          ? round_up(decode_tail_ws_bytes(b->Nq, decode_tail_chunks(b->Nq, kPlanSms)), 256)
+          : (w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0);
   w.part_off = w.hist_off + w.hist_bytes;
   w.plan = attn_plan(b->Nq, H, top_k, kPlanSms);
-  w.part_bytes = attn ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
+  w.part_bytes = attn && !w.fused_tail ? round_up(attn_partial_bytes(b->Nq, H, w.plan), 256) : 0;
   w.total = w.part_off + w.part_bytes;
   // The standalone calls with DSA_FLAG_SCORE_HISTOGRAM keep the histogram
   // region right after the control block.
@@ -364,11 +368,34 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   if (L.hist_topk) {
     // The histograms and counters start from zero on every call: no state is
     // carried in the workspace from one call to the next.
-    DSA_TRY(cuda_status(
-        cudaMemsetAsync(hist_region, 0, topk_hist_zero_bytes(batch->Nq), st)));
+    DSA_TRY(cuda_status(cudaMemsetAsync(
+        hist_region, 0,
+        L.fused_tail ? decode_tail_zero_bytes(batch->Nq) : topk_hist_zero_bytes(batch->Nq), st)));
     ia.hist = static_cast<int*>(hist_region);
   }
   DSA_TRY(cuda_status(launch_indexer_score(ia, st)));
+  if (L.fused_tail) {
+    DecodeTailArgs d;
+    d.B = batch->B;
+    d.Nq = batch->Nq;
+    d.H = H;
+    d.top_k = top_k;
+    d.q_offsets = batch->q_offsets;
+    d.kv_offsets = batch->kv_offsets;
+    d.ctx_lens = batch->ctx_lens;
+    d.q = q;
+    d.kv = kv;
+    d.scores = scores;
+    d.ld = L.ld;
+    d.ws_region = hist_region;
+    d.idx = idx;
+    d.out = out;
+    d.lse = lse;
+    d.err = err_word(ws);
+    d.scale = scale;
+    d.num_sms = std::min(sms, kPlanSms);  // the workspace holds kPlanSms / Nq chunks
+    return cuda_status(launch_decode_tail(d, st));
+  }
 
   const TopkArgs t = topk_args(batch, info, scores, L.ld, top_k, idx, ws, sms);
   DSA_TRY(cuda_status(L.hist_topk ? launch_topk_hist(t, hist_region, st) : launch_topk(t, st)));

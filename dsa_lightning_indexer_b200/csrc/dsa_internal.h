@@ -77,6 +77,33 @@ int topk_hist_chunks(int Nq, int64_t max_len, int* chunk_len);
 bool topk_hist_supported(int Nq, int64_t max_len);
 cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t stream);
 
+// The decode layer after the indexer as one cooperative kernel (selection
+// from the indexer's histograms, attention, merge): few long rows with one
+// query per sequence and at most 64 heads.
+struct DecodeTailArgs {
+  int B, Nq, H, top_k;
+  const int32_t* q_offsets;   // device
+  const int64_t* kv_offsets;  // device
+  const int32_t* ctx_lens;    // device
+  const uint16_t* q;
+  const uint16_t* kv;
+  const float* scores;
+  int64_t ld;
+  void* ws_region;   // decode_tail_ws_bytes; its first decode_tail_zero_bytes zeroed
+                     // before the indexer builds the histograms at its start
+  int32_t* idx;
+  float* out;
+  float* lse;
+  unsigned* err;
+  float scale;
+  int num_sms;       // SMs the launch may fill (one CTA per SM)
+};
+int decode_tail_chunks(int Nq, int num_sms);
+bool decode_tail_supported(int Nq, int H, int64_t max_len, int num_sms);
+size_t decode_tail_zero_bytes(int Nq);
+size_t decode_tail_ws_bytes(int Nq, int C);
+cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream);
+
 // How the attention launch covers (query row, head block, slice of the set).
 struct AttnPlan {
   int decode;       // 1: single-tile tcgen05 kernel, slices of 64 slots (few rows)

@@ -5,9 +5,13 @@ layer's arithmetic.  Tests, the benchmark and the smoke check take their inputs
 from here, and the same host arrays feed both the CUDA library and the CPU
 oracle.
 
-Every tensor comes from numpy's PCG64 seeded with SeedSequence([seed, layer,
-tensor_id]); normal draws are made in float32 and rounded to bfloat16 with
-round-to-nearest-even.  bf16 tensors are held as their uint16 bit patterns.
+Normal tensors are drawn in float32 with numpy's PCG64, in consecutive blocks
+of BLOCK elements (row-major order), block i from SeedSequence([seed, layer,
+tensor_id, i]); the blocks are drawn in parallel threads, and the values do
+not depend on the thread count.  Other draws (weights, lengths, directions)
+come from one PCG64 seeded with SeedSequence([seed, layer, tensor_id]).
+Values are rounded to bfloat16 with round-to-nearest-even; bf16 tensors are
+held as their uint16 bit patterns.
 
 The shapes follow the released Kimi-K3.1-Pro configuration (llama.cpp b12180
 news, devotd.net configuration table): indexer of 32 heads x 128, no RoPE,
@@ -18,6 +22,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -30,9 +36,16 @@ DV = 512      # value width (leading part of the latent row)
 T_QIDX, T_W, T_KIDX, T_Q, T_KV, T_DIRS, T_ASSIGN, T_LENS, T_PROJ = range(9)
 
 
+BLOCK = 1 << 22  # elements per independently seeded block of a normal tensor
+
+
 def bf16_bits(x: np.ndarray) -> np.ndarray:
     """float32 -> bfloat16 bit pattern (uint16), round to nearest even."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.size >= (1 << 16):  # the same rounding, multi-threaded, for big tensors
+        import torch
+        return torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    u = x.view(np.uint32)
     r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
 
@@ -47,12 +60,29 @@ def rng(seed: int, layer: int, tensor_id: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, layer, tensor_id])))
 
 
-def normal_bf16(seed, layer, tid, shape, std=1.0) -> np.ndarray:
-    g = rng(seed, layer, tid)
-    x = g.standard_normal(size=shape, dtype=np.float32)
+def normal_f32(seed, layer, tid, shape, std=1.0) -> np.ndarray:
+    """N(0, std^2) float32 draws of `shape`, in seeded blocks of BLOCK elements."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    nblk = max(1, (n + BLOCK - 1) // BLOCK)
+
+    def fill(i):
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, layer, tid, i])))
+        a, b = i * BLOCK, min(n, (i + 1) * BLOCK)
+        g.standard_normal(size=b - a, dtype=np.float32, out=out[a:b])
+
+    if nblk == 1:
+        fill(0)
+    else:
+        with ThreadPoolExecutor(min(nblk, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(nblk)))
     if std != 1.0:
-        x *= np.float32(std)
-    return bf16_bits(x)
+        out *= np.float32(std)
+    return out.reshape(shape)
+
+
+def normal_bf16(seed, layer, tid, shape, std=1.0) -> np.ndarray:
+    return bf16_bits(normal_f32(seed, layer, tid, shape, std))
 
 
 @dataclasses.dataclass
@@ -118,7 +148,7 @@ def _assemble(name, seed, layer, nq_per_seq, lens, H, top_k, planted=False, caps
         dirs = g.standard_normal(size=(64, DI), dtype=np.float32)
         dirs /= np.linalg.norm(dirs, axis=1, keepdims=True)
         assign = rng(seed, layer, T_ASSIGN).integers(0, 64, size=rows)
-        base = rng(seed, layer, T_KIDX).standard_normal(size=(rows, DI), dtype=np.float32)
+        base = normal_f32(seed, layer, T_KIDX, (rows, DI))
         base += np.float32(3.0) * dirs[assign]
         k_idx = bf16_bits(base)
     else:
