@@ -60,6 +60,8 @@ def _load():
                                                 P, i64]
         lib.oracle_dsa_layer.argtypes = [i32, P, P, P, i32, i32, P, P, P, i32, i32, i32, P, P,
                                          i32, dbl, P, i64, P, P, P, P, i64]
+        lib.oracle_indexer_project.argtypes = [i32, P, P, P, i32, i32, i64, i64, P, P, P, P, P,
+                                               P, P, P, P, i64]
         _lib = lib
     return _lib
 
@@ -185,3 +187,33 @@ def dsa_layer(q_offsets, kv_offsets, ctx_lens, q_idx, w, k_idx, q, kv, top_k, sc
                              _ptr(k_idx), H, D, Dv, _ptr(q), _ptr(kv), int(top_k), float(scale),
                              _ptr(scores), ld, _ptr(idx), _ptr(out), _ptr(lse), _ptr(s), ns)
     return scores, idx, out, lse
+
+
+def indexer_project(q_offsets, kv_offsets, ctx_lens, x, c_q, w_q_b, w_k, w_proj, k_idx,
+                    sample=None):
+    """The indexer's input step for every (sampled) query row: returns
+    (q_idx [Nq, Hi, Di] bf16 bits, k_idx with the new tokens' rows written,
+    w [Nq, Hi] float32).  x [Nq, d_model] and c_q [Nq, d_q] are bf16 bits;
+    weights are [out, in] bf16 bits: w_q_b [Hi*Di, d_q], w_k [Di, d_model],
+    w_proj [Hi, d_model].  k_idx is copied, not modified."""
+    B, qo, ko, cl = _batch(q_offsets, kv_offsets, ctx_lens)
+    x = _c(x, np.uint16)
+    c_q = _c(c_q, np.uint16)
+    w_q_b = _c(w_q_b, np.uint16)
+    w_k = _c(w_k, np.uint16)
+    w_proj = _c(w_proj, np.uint16)
+    k_out = np.array(k_idx, dtype=np.uint16, copy=True, order="C")
+    Nq, d_model = x.shape
+    d_q = c_q.shape[1]
+    Di = w_k.shape[0]
+    Hi = w_proj.shape[0]
+    assert c_q.shape[0] == Nq and w_q_b.shape == (Hi * Di, d_q)
+    assert w_k.shape == (Di, d_model) and w_proj.shape == (Hi, d_model)
+    assert k_out.shape[1] == Di
+    q_idx = np.zeros((Nq, Hi, Di), dtype=np.uint16)
+    w = np.full((Nq, Hi), np.nan, dtype=np.float32)
+    s, ns = _sample(sample)
+    _load().oracle_indexer_project(B, _ptr(qo), _ptr(ko), _ptr(cl), Hi, Di, int(d_model),
+                                   int(d_q), _ptr(x), _ptr(c_q), _ptr(w_q_b), _ptr(w_k),
+                                   _ptr(w_proj), _ptr(q_idx), _ptr(k_out), _ptr(w), _ptr(s), ns)
+    return q_idx, k_out, w

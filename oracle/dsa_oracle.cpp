@@ -27,6 +27,15 @@
 //     attention (aiaulis.com paragraph 7; aiunderstanding.org "What happened";
 //     devotd.net section 4).  oracle_full_causal_attn states that case with no
 //     indexer code at all.
+//   * The indexer's input step: the three indexer tensors named on the pages
+//     (q_b, k and the head-weight projection; aiunderstanding.org "What
+//     happened"; devotd.net section 3 -- kept out of quantization, so bf16
+//     here) are plain linear maps of each new token: q_idx = c_q . W_q_b^T
+//     from the token's query latent c_q, k = x . W_k^T and w = x . W_proj^T
+//     from its hidden state x; k is appended to the indexer key cache at the
+//     token's own row (devotd.net section 2: the indexer keeps a key cache).
+//     The pages give no widths for x and c_q, and no normalisation or
+//     scaling; none is applied.
 //
 // Conventions shared with the header of the product library (restated here,
 // not included): sequence b owns query rows [q_off[b], q_off[b+1]) and cache
@@ -157,6 +166,25 @@ void attend_row(const Row& r, int H, int D, int Dv, const uint16_t* q, const uin
   }
 }
 
+// bf16 bit pattern of a double, rounded to nearest even through fp32 (the
+// precision in which a projection's sum is formed before it is stored).
+uint16_t double_to_bf16(double v) {
+  const float f = static_cast<float>(v);
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof u);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return static_cast<uint16_t>((u >> 16) | 0x40u);  // NaN
+  u += 0x7FFFu + ((u >> 16) & 1u);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+// sum_j a[j] * W[f, j] in double for one output feature f; W is [n_out, n_in].
+double linear_one(const uint16_t* a, const uint16_t* W, int64_t n_in, int64_t f) {
+  double acc = 0.0;
+  const uint16_t* wf = W + f * n_in;
+  for (int64_t j = 0; j < n_in; ++j) acc += bf16_to_double(a[j]) * bf16_to_double(wf[j]);
+  return acc;
+}
+
 }  // namespace
 
 extern "C" {
@@ -263,6 +291,45 @@ void oracle_dsa_layer(int B, const int32_t* q_off, const int64_t* kv_off,
     }
     attend_row(r, H, D, Dv, q, kv, pos.data(), static_cast<int64_t>(pos.size()), scale, out,
                lse);
+  }
+}
+
+// The indexer's input step for every (sampled) query row t (a new token of
+// sequence b at position p): q_idx[t] = c_q[t] . W_q_b^T (Hi*Di outputs, bf16),
+// k = x[t] . W_k^T (Di outputs, bf16) written to cache row kv_off[b] + p of
+// k_idx, w[t] = x[t] . W_proj^T (Hi outputs, fp32).  Weights are [out, in].
+void oracle_indexer_project(int B, const int32_t* q_off, const int64_t* kv_off,
+                            const int32_t* ctx_lens, int Hi, int Di, int64_t d_model,
+                            int64_t d_q, const uint16_t* x, const uint16_t* c_q,
+                            const uint16_t* w_q_b, const uint16_t* w_k, const uint16_t* w_proj,
+                            uint16_t* q_idx, uint16_t* k_idx, float* w, const int64_t* sample,
+                            int64_t n_sample) {
+  const std::vector<Row> rows = plan_rows(B, q_off, kv_off, ctx_lens, sample, n_sample);
+  const int64_t n = static_cast<int64_t>(rows.size());
+  const int64_t nq_out = static_cast<int64_t>(Hi) * Di;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t i = 0; i < n; ++i) {
+    const Row& r = rows[i];
+    const uint16_t* xr = x + r.row * d_model;
+    const uint16_t* cr = c_q + r.row * d_q;
+    for (int64_t f = 0; f < nq_out; ++f) {
+      q_idx[r.row * nq_out + f] = double_to_bf16(linear_one(cr, w_q_b, d_q, f));
+    }
+    const int64_t cache_row = (g_fault == 6) ? r.kv0 + r.pos + 1 : r.kv0 + r.pos;  // fault 6
+    for (int64_t f = 0; f < Di; ++f) {
+      double v = 0.0;
+      if (g_fault == 7) {  // fault 7: the key map read transposed (W_k taken as [in, out])
+        for (int64_t j = 0; j < d_model; ++j) {
+          v += bf16_to_double(xr[j]) * bf16_to_double(w_k[j * Di + f]);
+        }
+      } else {
+        v = linear_one(xr, w_k, d_model, f);
+      }
+      k_idx[cache_row * Di + f] = double_to_bf16(v);
+    }
+    for (int h = 0; h < Hi; ++h) {
+      w[r.row * Hi + h] = static_cast<float>(linear_one(xr, w_proj, d_model, h));
+    }
   }
 }
 

@@ -300,4 +300,77 @@ def pin_single_row_returns_its_value():
         assert np.abs(lse[r] - logit).max() < 1e-5 * max(1.0, np.abs(logit).max())
 
 
+
+
+# --------------------------------------------------- indexer input step ----
+
+def pin_projection_worked_example():
+    g = json.load(open(os.path.join(GOLDEN, "indexer_projection_worked_example.json")))
+    qo, ko, cl = _one_seq(3, 2)
+    sentinel = _bf16(np.full((3, g["Di"]), 7.0, np.float32))
+    q_idx, k_out, w = oracle.indexer_project(
+        qo, ko, cl, _bf16(g["x"]), _bf16(g["c_q"]), _bf16(g["w_q_b"]), _bf16(g["w_k"]),
+        _bf16(g["w_proj"]), sentinel)
+    assert np.array_equal(_f(q_idx), np.array(g["q_idx"], np.float64))
+    for row, vals in g["k_rows"].items():
+        assert np.array_equal(_f(k_out[int(row)]), np.array(vals, np.float64))
+    assert np.array_equal(k_out[0], sentinel[0])           # earlier token untouched
+    assert np.array_equal(w.astype(np.float64), np.array(g["w"], np.float64))
+
+
+def pin_projection_identity_weights_copy_their_inputs():
+    # unit rows pick input entries exactly: q_idx = c_q, k = x[:, :Di], w = x[:, 5:5+Hi]
+    Hi, Di, d_model = 3, 4, 16
+    d_q = Hi * Di
+    g = np.random.Generator(np.random.PCG64(21))
+    qo = np.array([0, 2, 3], np.int32)
+    ko = np.array([0, 6, 10], np.int64)
+    cl = np.array([5, 4], np.int32)
+    x = _bf16(g.standard_normal((3, d_model)))
+    c_q = _bf16(g.standard_normal((3, d_q)))
+    w_q_b = _bf16(np.eye(d_q))
+    w_k = _bf16(np.eye(Di, d_model))
+    w_proj = _bf16(np.eye(Hi, d_model, k=5))
+    k0 = np.zeros((10, Di), np.uint16)
+    q_idx, k_out, w = oracle.indexer_project(qo, ko, cl, x, c_q, w_q_b, w_k, w_proj, k0)
+    assert np.array_equal(q_idx.reshape(3, d_q), c_q)
+    # new tokens: sequence 0 positions 3, 4 (rows 3, 4); sequence 1 position 3 (row 6 + 3)
+    for t, row in enumerate([3, 4, 9]):
+        assert np.array_equal(k_out[row], x[t, :Di]), (t, row)
+    assert np.array_equal(w, _f(x[:, 5:5 + Hi]).astype(np.float32))
+    written = {3, 4, 9}
+    for row in range(10):
+        if row not in written:
+            assert not k_out[row].any(), row
+
+
+def pin_projection_matches_float64_matmul():
+    # the general case is a matmul: compare with torch's float64 product, rounded
+    # to bf16 through fp32 as the step stores it
+    Hi, Di, d_model, d_q = 4, 8, 96, 40
+    g = np.random.Generator(np.random.PCG64(22))
+    qo = np.array([0, 3, 3, 5], np.int32)
+    ko = np.array([0, 7, 9, 15], np.int64)
+    cl = np.array([6, 2, 5], np.int32)
+    Nq, rows = 5, 15
+    x = _bf16(g.standard_normal((Nq, d_model)))
+    c_q = _bf16(g.standard_normal((Nq, d_q)))
+    w_q_b = _bf16(g.standard_normal((Hi * Di, d_q)) * 0.2)
+    w_k = _bf16(g.standard_normal((Di, d_model)) * 0.1)
+    w_proj = _bf16(g.standard_normal((Hi, d_model)) * 0.1)
+    k0 = _bf16(g.standard_normal((rows, Di)))
+    q_idx, k_out, w = oracle.indexer_project(qo, ko, cl, x, c_q, w_q_b, w_k, w_proj, k0)
+    T = lambda a: torch.from_numpy(_f(a))  # noqa: E731
+    want_q = (T(c_q) @ T(w_q_b).T).numpy().astype(np.float32)
+    want_k = (T(x) @ T(w_k).T).numpy().astype(np.float32)
+    want_w = (T(x) @ T(w_proj).T).numpy()
+    assert np.array_equal(q_idx.reshape(Nq, -1), synth.bf16_bits(want_q))
+    # new tokens' cache rows: the last nq_b positions of each sequence
+    new_rows = [3, 4, 5, 12, 13]
+    assert np.array_equal(k_out[new_rows], synth.bf16_bits(want_k))
+    others = [r for r in range(rows) if r not in new_rows]
+    assert np.array_equal(k_out[others], k0[others])
+    assert np.allclose(w.astype(np.float64), want_w, rtol=1e-6, atol=1e-7)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -11,6 +11,8 @@ FAULTS = {
     3: "causal window excludes the query's own position",
     4: "softmax scale dropped",
     5: "V taken from the tail of the latent row instead of its head",
+    6: "indexer key written one cache row past the new token's position",
+    7: "indexer key map read transposed",
 }
 
 
