@@ -51,6 +51,10 @@ SIGNATURES = {
                                          ctypes.c_uint32, _P]),
     "dsa_sparse_attn_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, ctypes.c_int,
                                                ctypes.c_float, _P, _P, _P]),
+    "dsa_indexer_project_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int64,
+                                                             ctypes.c_int64]),
+    "dsa_indexer_project": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _P,
+                                           _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "dsa_check_device_status": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "dsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
@@ -197,6 +201,22 @@ def layer_forward(batch, q, q_idx, w, k_idx, kv, top_k, scale, out, lse, idx, ws
                                  _bf16(kv), int(top_k), float(scale), _f32(out), _f32(lse),
                                  _i32(idx), _ptr(ws), ws.numel(), int(flags), _stream(stream)),
            "dsa_layer_forward")
+
+
+def indexer_project_workspace(batch, d_model, d_q, device="cuda"):
+    """A zero-filled workspace for dsa_indexer_project on this batch."""
+    n = int(lib.dsa_indexer_project_workspace_size(batch.ref, int(d_model), int(d_q)))
+    if n == 0:
+        raise DsaError(ERR_INVALID_ARG, "dsa_indexer_project_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def indexer_project(batch, x, c_q, w_q_b, w_k, w_proj, q_idx, k_idx, w, ws, stream=None):
+    """The indexer's input step: q_idx, w out; the new tokens' k rows into k_idx."""
+    _check(lib.dsa_indexer_project(batch.ref, _bf16(x), int(x.shape[1]), _bf16(c_q),
+                                   int(c_q.shape[1]), _bf16(w_q_b), _bf16(w_k), _bf16(w_proj),
+                                   _bf16(q_idx), _bf16(k_idx), _f32(w), _ptr(ws), ws.numel(),
+                                   _stream(stream)), "dsa_indexer_project")
 
 
 def check_device_status(ws, stream=None):

@@ -422,6 +422,63 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   return cuda_status(launch_sparse_attn(a, st));
 }
 
+namespace {
+inline bool projection_width_ok(int64_t d) { return d >= 64 && d <= 65536 && d % 64 == 0; }
+}  // namespace
+
+size_t dsa_indexer_project_workspace_size(const dsa_batch* batch, int64_t d_model, int64_t d_q) {
+  BatchInfo info;
+  if (check_batch(batch, &info) != DSA_OK || !projection_width_ok(d_model) ||
+      !projection_width_ok(d_q)) {
+    return 0;
+  }
+  return kControlBytes + project_ws_bytes(batch->Nq, static_cast<int>(d_q),
+                                          static_cast<int>(d_model), kPlanSms);
+}
+
+dsa_status dsa_indexer_project(const dsa_batch* batch, const uint16_t* x, int64_t d_model,
+                               const uint16_t* c_q, int64_t d_q, const uint16_t* w_q_b,
+                               const uint16_t* w_k, const uint16_t* w_proj, uint16_t* q_idx,
+                               uint16_t* k_idx, float* w, void* ws, size_t ws_bytes,
+                               void* stream) {
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  if (!projection_width_ok(d_model) || !projection_width_ok(d_q)) return DSA_ERR_UNSUPPORTED;
+  if (batch->Nq == 0) return DSA_OK;
+  const void* ptrs[] = {x, c_q, w_q_b, w_k, w_proj, q_idx, k_idx, w};
+  for (const void* p : ptrs) DSA_TRY(check_ptr(p));
+  // Split planning uses kPlanSms, so the workspace size does not depend on the device.
+  const size_t need = kControlBytes + project_ws_bytes(batch->Nq, static_cast<int>(d_q),
+                                                       static_cast<int>(d_model), kPlanSms);
+  DSA_TRY(check_ws(ws, ws_bytes, need));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProjectArgs a;
+  a.B = batch->B;
+  a.T = batch->Nq;
+  a.q_offsets = batch->q_offsets;
+  a.kv_offsets = batch->kv_offsets;
+  a.ctx_lens = batch->ctx_lens;
+  a.x = x;
+  a.c_q = c_q;
+  a.w_q_b = w_q_b;
+  a.w_k = w_k;
+  a.w_proj = w_proj;
+  a.d_model = static_cast<int>(d_model);
+  a.d_q = static_cast<int>(d_q);
+  a.q_idx = q_idx;
+  a.k_cache = k_idx;
+  a.w = w;
+  a.ws_region = static_cast<uint8_t*>(ws) + kControlBytes;
+  a.err = err_word(ws);
+  a.num_sms = kPlanSms;
+  // The split-K tickets start from zero on every call.
+  DSA_TRY(cuda_status(cudaMemsetAsync(a.ws_region, 0,
+                                      project_zero_bytes(a.T, a.d_q, a.d_model, kPlanSms), st)));
+  return cuda_status(launch_indexer_project(a, st));
+}
+
 dsa_status dsa_check_device_status(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < kControlBytes) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

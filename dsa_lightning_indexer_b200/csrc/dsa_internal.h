@@ -104,6 +104,30 @@ size_t decode_tail_zero_bytes(int Nq);
 size_t decode_tail_ws_bytes(int Nq, int C);
 cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream);
 
+// The indexer's input step (projections of the new tokens, k appended to the
+// indexer key cache) as one tcgen05 GEMM over the concatenated features.
+struct ProjectArgs {
+  int B, T;                   // sequences, new tokens (query rows)
+  const int32_t* q_offsets;   // device
+  const int64_t* kv_offsets;  // device
+  const int32_t* ctx_lens;    // device
+  const uint16_t* x;          // [T][d_model]
+  const uint16_t* c_q;        // [T][d_q]
+  const uint16_t* w_q_b;      // [4096][d_q]
+  const uint16_t* w_k;        // [128][d_model]
+  const uint16_t* w_proj;     // [32][d_model]
+  int d_model, d_q;           // multiples of 64
+  uint16_t* q_idx;            // [T][4096]
+  uint16_t* k_cache;          // [rows][128]
+  float* w;                   // [T][32]
+  void* ws_region;            // project_ws_bytes; its first project_zero_bytes zeroed
+  unsigned* err;
+  int num_sms;
+};
+size_t project_ws_bytes(int T, int d_q, int d_model, int num_sms);
+size_t project_zero_bytes(int T, int d_q, int d_model, int num_sms);
+cudaError_t launch_indexer_project(const ProjectArgs& a, cudaStream_t stream);
+
 // How the attention launch covers (query row, head block, slice of the set).
 struct AttnPlan {
   int decode;       // 1: single-tile tcgen05 kernel, slices of 64 slots (few rows)

@@ -203,6 +203,33 @@ DSA_API dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, 
                              void* stream);
 
 /*
+ * The indexer's input step for the new tokens of a batch (aiunderstanding.org
+ * "What happened": the indexer's q_b, k and projection tensors are kept out
+ * of quantization; devotd.net section 2: a DSA layer keeps an indexer key
+ * cache).  The pages give no widths and no normalisation; the three maps are
+ * taken as plain linear maps.  For every query row t (the j-th new token of
+ * sequence b, at position p = ctx_lens[b] - nq_b + j):
+ *   q_idx[t] = c_q[t] . w_q_b^T     [Nq, 32, 128] bf16 out
+ *   k        = x[t]   . w_k^T       written to k_idx row kv_offsets[b] + p (bf16)
+ *   w[t]     = x[t]   . w_proj^T    [Nq, 32] fp32 out
+ * Inputs, bf16: x [Nq, d_model] (hidden states), c_q [Nq, d_q] (query
+ * latents); weights [out, in]: w_q_b [4096, d_q], w_k [128, d_model],
+ * w_proj [32, d_model].  d_model and d_q are multiples of 64 in [64, 65536].
+ * Rows of k_idx other than the new tokens' are not touched.  Products are
+ * exact, sums fp32, outputs rounded to bf16 (to nearest even) except w.
+ * Runs as one tcgen05 GEMM; the workspace holds split-K partials
+ * (dsa_indexer_project_workspace_size bytes, zero-filled before first use
+ * like every workspace).
+ */
+DSA_API size_t dsa_indexer_project_workspace_size(const dsa_batch* batch, int64_t d_model,
+                                                  int64_t d_q);
+DSA_API dsa_status dsa_indexer_project(const dsa_batch* batch, const uint16_t* x, int64_t d_model,
+                                       const uint16_t* c_q, int64_t d_q, const uint16_t* w_q_b,
+                                       const uint16_t* w_k, const uint16_t* w_proj,
+                                       uint16_t* q_idx, uint16_t* k_idx, float* w, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/*
  * dsa_sparse_attn without a workspace, for callers that cannot allocate
  * device memory when they run the layer (a fixed pre-sized memory pool, a
  * runtime that hands kernels only the tensors it owns, a plugin host that

@@ -24,7 +24,8 @@ def test_header_declares_the_boundary():
     assert declared_symbols() == sorted([
         "dsa_workspace_size", "dsa_indexer_score", "dsa_topk", "dsa_sparse_attn",
         "dsa_layer_forward", "dsa_check_device_status", "dsa_status_string",
-        "dsa_sparse_attn_noalloc"])
+        "dsa_sparse_attn_noalloc", "dsa_indexer_project_workspace_size",
+        "dsa_indexer_project"])
 
 
 def test_library_exports_every_declared_symbol():
