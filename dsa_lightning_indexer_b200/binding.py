@@ -33,6 +33,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOU
 # flags
 FLAG_SCORE_HISTOGRAM = 0x1
 FLAG_TEST_STALL = 0x80000000
+FLAG_MASKED_ROUTE = 0x2
 
 INDEX_HEADS, INDEX_DIM, LATENT_DIM, VALUE_DIM, MAX_TOPK, MAX_HEADS = 32, 128, 576, 512, 2048, 128
 CONTROL_BYTES = 256
@@ -49,6 +50,8 @@ SIGNATURES = {
     "dsa_layer_forward": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int,
                                          ctypes.c_float, _P, _P, _P, _P, ctypes.c_size_t,
                                          ctypes.c_uint32, _P]),
+    "dsa_masked_attn": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, ctypes.c_int,
+                                       ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
     "dsa_sparse_attn_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _P, _P, ctypes.c_int,
                                                ctypes.c_float, _P, _P, _P]),
     "dsa_indexer_project_workspace_size": (ctypes.c_size_t, [_P, ctypes.c_int64,
@@ -156,13 +159,14 @@ def _stream(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
 
 
-def workspace_size(batch: Batch, H: int, top_k: int) -> int:
-    return int(lib.dsa_workspace_size(batch.ref, int(H), int(top_k), 0))
+def workspace_size(batch: Batch, H: int, top_k: int, flags: int = 0) -> int:
+    return int(lib.dsa_workspace_size(batch.ref, int(H), int(top_k), int(flags)))
 
 
-def alloc_workspace(batch: Batch, H: int, top_k: int, device="cuda") -> torch.Tensor:
-    """A zero-filled workspace large enough for every call on this batch."""
-    n = workspace_size(batch, H, top_k)
+def alloc_workspace(batch: Batch, H: int, top_k: int, device="cuda", flags=0) -> torch.Tensor:
+    """A zero-filled workspace large enough for every call on this batch
+    (with FLAG_MASKED_ROUTE, for dsa_masked_attn too)."""
+    n = workspace_size(batch, H, top_k, flags)
     if n == 0:
         raise DsaError(ERR_INVALID_ARG, "dsa_workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)
@@ -184,6 +188,14 @@ def sparse_attn(batch, q, kv, idx, top_k, scale, out, lse, ws, stream=None):
     _check(lib.dsa_sparse_attn(batch.ref, _bf16(q), H, _bf16(kv), _i32(idx), int(top_k),
                                float(scale), _f32(out), _f32(lse), _ptr(ws), ws.numel(),
                                _stream(stream)), "dsa_sparse_attn")
+
+
+def masked_attn(batch, q, kv, idx, top_k, scale, out, lse, ws, stream=None):
+    """Attention over the listed rows computed as a mask over the whole cache."""
+    H = int(q.shape[1])
+    _check(lib.dsa_masked_attn(batch.ref, _bf16(q), H, _bf16(kv), _i32(idx), int(top_k),
+                               float(scale), _f32(out), _f32(lse), _ptr(ws), ws.numel(),
+                               _stream(stream)), "dsa_masked_attn")
 
 
 def sparse_attn_noalloc(batch, q, kv, idx, top_k, scale, out, lse, stream=None):

@@ -130,6 +130,12 @@ bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// dsa_masked_attn: the control block and the chunks' partial results.
+size_t masked_ws_need(const dsa_batch* b, const BatchInfo& info, int H) {
+  const AttnPlan p = masked_attn_plan(b->Nq, H, info.max_len, kPlanSms);
+  return kControlBytes + round_up(attn_partial_bytes(b->Nq, H, p), 256);
+}
+
 // Workspace bytes of the standalone calls with DSA_FLAG_SCORE_HISTOGRAM: the
 // control block, then the histogram region (the histograms and counters
 // first, the selection's lists after them).
@@ -227,13 +233,16 @@ using namespace dsa;
 extern "C" {
 
 size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t flags) {
-  (void)flags;
   BatchInfo info;
   if (check_batch(batch, &info) != DSA_OK || check_heads(H) != DSA_OK ||
-      check_topk(top_k) != DSA_OK) {
+      check_topk(top_k) != DSA_OK || (flags & ~DSA_FLAG_MASKED_ROUTE) != 0u) {
     return 0;
   }
-  return plan_ws(batch, info, H, top_k, true, true).total;
+  size_t total = plan_ws(batch, info, H, top_k, true, true).total;
+  if ((flags & DSA_FLAG_MASKED_ROUTE) != 0u) {
+    total = std::max(total, masked_ws_need(batch, info, H));
+  }
+  return total;
 }
 
 dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,
@@ -331,8 +340,50 @@ dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.ctx_lens = batch->ctx_lens;
   a.idx_prefix = false;
   a.batch_ready = false;
+  a.cache_rows = info.cache_rows;
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, static_cast<cudaStream_t>(stream)));
+}
+
+dsa_status dsa_masked_attn(const dsa_batch* batch, const uint16_t* q, int H, const uint16_t* kv,
+                           const int32_t* idx, int top_k, float scale, float* out, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+  BatchInfo info;
+  DSA_TRY(check_batch(batch, &info));
+  DSA_TRY(check_heads(H));
+  DSA_TRY(check_topk(top_k));
+  if (batch->Nq == 0) return DSA_OK;
+  DSA_TRY(check_ptr(q));
+  DSA_TRY(check_ptr(kv));
+  DSA_TRY(check_ptr(idx));
+  DSA_TRY(check_ptr(out));
+  if (lse) DSA_TRY(check_ptr(lse));
+  if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  if (!masked_attn_supported(info.max_len)) return DSA_ERR_UNSUPPORTED;
+  DSA_TRY(check_ws(ws, ws_bytes, masked_ws_need(batch, info, H)));
+  int sms = 0;
+  DSA_TRY(check_device(&sms));
+  AttnArgs a;
+  a.B = batch->B;
+  a.Nq = batch->Nq;
+  a.q_offsets = batch->q_offsets;
+  a.kv_offsets = batch->kv_offsets;
+  a.ctx_lens = batch->ctx_lens;
+  a.q = q;
+  a.H = H;
+  a.kv = kv;
+  a.idx = idx;
+  a.top_k = top_k;
+  a.scale = scale;
+  a.out = out;
+  a.lse = lse;
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kControlBytes);
+  a.err = err_word(ws);
+  a.idx_prefix = false;
+  a.batch_ready = false;
+  a.cache_rows = info.cache_rows;
+  a.plan = masked_attn_plan(batch->Nq, H, info.max_len, kPlanSms);
+  return cuda_status(launch_masked_attn(a, static_cast<cudaStream_t>(stream)));
 }
 
 dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
@@ -418,6 +469,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   a.ctx_lens = batch->ctx_lens;
   a.idx_prefix = true;  // produced by dsa_topk: valid positions first, then -1
   a.batch_ready = true;  // the layer's own kernels never write the batch arrays
+  a.cache_rows = info.cache_rows;
   a.plan = L.plan;
   return cuda_status(launch_sparse_attn(a, st));
 }

@@ -161,6 +161,7 @@ struct AttnArgs {
   unsigned* err;      // workspace error word (bounded waits)
   bool idx_prefix;    // valid entries are the first min(top_k, p+1) slots of each row
   bool batch_ready;   // no kernel this launch depends on writes the batch arrays
+  int64_t cache_rows; // rows of kv (the masked route's tensor map)
   AttnPlan plan;
 };
 cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream);
@@ -169,6 +170,11 @@ int attn_decode_slots();  // selected slots per CTA of the single-tile kernel
 // Merges the slices of a split launch (plan.n_split > 1) into out and lse.
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+// The mask-over-the-whole-cache route (comparison): chunks of the causal
+// positions per CTA, every cached row streamed, unlisted rows masked.
+AttnPlan masked_attn_plan(int Nq, int H, int64_t max_len, int num_sms);
+bool masked_attn_supported(int64_t max_len);
+cudaError_t launch_masked_attn(const AttnArgs& a, cudaStream_t stream);
 
 // Raises a kernel's dynamic shared-memory limit to `bytes`, once per device
 // (the attribute call is not free, and launches may be captured in a graph).

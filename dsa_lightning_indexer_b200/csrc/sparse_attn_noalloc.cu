@@ -112,6 +112,7 @@ extern "C" DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, co
   a.err = nullptr;  // the CUDA-core kernels never wait on a barrier
   a.idx_prefix = false;
   a.batch_ready = false;
+  a.cache_rows = info.cache_rows;
   a.plan = plan;
   return launch_sparse_attn(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK
                                                                                    : DSA_ERR_CUDA;

@@ -22,6 +22,16 @@
 // Warp roles (288 threads): warps 0-3 softmax and output (TMEM quadrants
 // 0-3), warp 4 TMEM allocation, the Q load (TMA) and single-thread MMA issue,
 // warps 5-6 and 7-8 gather even and odd tiles with 16-byte cp.async.
+//
+// The same kernel, instantiated with kMasked, is the mask-over-the-whole-
+// cache route the pages describe for llama.cpp (aiaulis.com paragraph 4;
+// devotd.net section 2: the selection becomes a mask so that the existing
+// sparse flash attention is reused): a CTA owns a chunk of the row's causal
+// positions instead of a slice of its index set, streams every cached row of
+// the chunk with TMA tile loads, and masks the logits of the rows that the
+// index set does not list (a bitmap of the chunk built from it).  It reads
+// the whole latent cache; it is kept as the measured comparison to the
+// gather.
 #include <algorithm>
 
 #include "attn_tc_common.cuh"
@@ -54,7 +64,9 @@ constexpr int kOffIdx = kOffTmem + 16;                  // [2][kT] int
 constexpr int kOffAlpha = kOffIdx + 2 * kT * 4;         // [64] float
 constexpr int kOffM = kOffAlpha + kHB * 4;              // [64] float
 constexpr int kOffL = kOffM + kHB * 4;                  // [64] float
-constexpr int kSmemUsed = kOffL + kHB * 4;
+constexpr int kOffMask = kOffL + kHB * 4;               // masked route: chunk bitmap
+constexpr int kMaskWords = 1024;                        // positions per chunk <= 32768
+constexpr int kSmemUsed = kOffMask + kMaskWords * 4;
 constexpr int kSmemTc = kSmemUsed + 1024;               // alignment slack
 static_assert(kOffStage + kHB * kValue * 4 <= kOffP, "output staging overlaps the P buffers");
 static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
@@ -69,8 +81,10 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-ma
 constexpr int kSplitCols = kT / 2;  // logits per half warp (16 + 8 columns)
 static_assert(kSplitCols == 24, "the logit loads cover 16 + 8 columns per half warp");
 
+template <bool kMasked>
 __global__ void __launch_bounds__(kThreadsTc, 1)
-    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const TcParams P) {
+    sparse_attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                          const __grid_constant__ CUtensorMap kvmap, const TcParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -90,6 +104,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
   float* const rl_s = reinterpret_cast<float*>(bp + kOffL);  // 1 / row sum per head
+  uint32_t* const mask = reinterpret_cast<uint32_t*>(bp + kOffMask);
 
   const int warp = warp_id_uniform();
   const int lane = lane_id();
@@ -100,7 +115,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(b_kvfull(s), kGroupThreads);
+      mbar_init(b_kvfull(s), kMasked ? 1 : kGroupThreads);
       mbar_init(b_kvempty(s), 1);
       mbar_init(b_sfull(s), 1);
       mbar_init(b_sempty(s), kSoftThreads);
@@ -127,12 +142,62 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
   // With idx_prefix, slots past min(top_k, p+1) hold -1: skip their tiles.
   const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
-  // This CTA's slice of the slots.
+  // This CTA's slice of the slots (of the causal positions, masked route).
   const int slot_lo = sp * P.split_len;
-  const int slot_hi = min(n_slots, slot_lo + P.split_len);
+  const int slot_hi = min(kMasked ? rs.len : n_slots, slot_lo + P.split_len);
   const int n_tiles = slot_hi > slot_lo ? (slot_hi - slot_lo + kT - 1) / kT : 0;
+  if (kMasked) {
+    // Bitmap of the chunk's positions that the index set lists.
+    const int nwords = (P.split_len + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += kThreadsTc) mask[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < P.top_k; i += kThreadsTc) {
+      const int pos = __ldg(idx_row + i);
+      if (pos < -1 || pos >= rs.len) {  // outside 0..p: skipped and recorded
+        atomicOr(P.err, kErrIndex);
+      } else if (pos >= slot_lo && pos < slot_hi) {
+        atomicOr(&mask[(pos - slot_lo) >> 5], 1u << ((pos - slot_lo) & 31));
+      }
+    }
+    __syncthreads();
+  }
 
-  if (warp >= 5) {
+  if (kMasked && warp >= 5) {
+    // ----------------------------------------- whole-cache tiles (masked) --
+    // Each group stages its tiles' positions (-1 where the mask drops the row)
+    // and one thread loads all rows of the tile with TMA.
+    const int grp = (warp - 5) >> 1;
+    const int gt = threadIdx.x - (5 + 2 * grp) * 32;
+    int* const gidx = tidx + grp * kT;
+    const uint64_t pol = l2_policy_evict_first();
+    bool ok = true;
+    int last_t = -1;  // the last tile this group loaded
+    for (int t = grp; t < n_tiles && ok; t += 2) {
+      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
+      if (!ok) break;
+      if (gt < kT) {
+        const int rel = t * kT + gt;
+        const int pos = slot_lo + rel;
+        const bool on = pos < slot_hi && ((mask[rel >> 5] >> (rel & 31)) & 1u);
+        gidx[gt] = on ? pos : -1;
+      }
+      named_bar_sync(2 + grp, kGroupThreads);
+      if (gt == 0) {
+        const uint32_t stage = sKV + grp * kKVStage;
+        mbar_arrive_expect_tx(b_kvfull(grp), kKVStage);
+        const int row = static_cast<int>(kv0 + slot_lo + t * kT);
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          tma_load_2d(stage + bx * kKVBox, &kvmap, b_kvfull(grp), 64 * bx, row, pol);
+        }
+        last_t = t;
+      }
+    }
+    // The loads this group issued land before the CTA may exit.
+    if (gt == 0 && last_t >= 0) {
+      mbar_drain(b_kvfull(grp), static_cast<uint32_t>((last_t >> 1) & 1), P.err);
+    }
+  } else if (warp >= 5) {
     // ------------------------------------------------------------ gather --
     // Each thread copies whole 128-byte box rows (eight 16-byte pieces with
     // the swizzle applied), after the group has staged the tile's positions.
@@ -481,24 +546,38 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
 }
 
-}  // namespace
 
-cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+template <bool kMasked>
+cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   if (a.Nq == 0) return cudaSuccess;
   EncodeTiledFn fn = get_encode_tiled();
   if (!fn) return cudaErrorInvalidValue;
-  CUtensorMap qmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLatent),
-                              static_cast<cuuint64_t>(a.Nq) * a.H};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLatent) * 2};
-  const cuuint32_t box[2] = {64, kHB};
+  CUtensorMap qmap, kvmap;
   const cuuint32_t estr[2] = {1, 1};
-  if (fn(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides,
-         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
-    return cudaErrorInvalidValue;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLatent),
+                                static_cast<cuuint64_t>(a.Nq) * a.H};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLatent) * 2};
+    const cuuint32_t box[2] = {64, kHB};
+    if (fn(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.q), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      return cudaErrorInvalidValue;
+    }
   }
-  cudaError_t e = ensure_smem_limit<sparse_attn_tc_kernel>(kSmemTc);
+  kvmap = qmap;  // unused by the gather instantiation
+  if (kMasked) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kLatent),
+                                static_cast<cuuint64_t>(a.cache_rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kLatent) * 2};
+    const cuuint32_t box[2] = {64, kT};
+    if (fn(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.kv), dims,
+           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      return cudaErrorInvalidValue;
+    }
+  }
+  cudaError_t e = ensure_smem_limit<sparse_attn_tc_kernel<kMasked>>(kSmemTc);
   if (e != cudaSuccess) return e;
   TcParams P;
   P.q_offsets = a.q_offsets;
@@ -522,10 +601,44 @@ cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
   P.top_k = a.top_k;
   P.scale_log2 = a.scale * kLog2e;
   const int head_blocks = (a.H + kHB - 1) / kHB;
-  e = launch_pdl(sparse_attn_tc_kernel, dim3(a.Nq, head_blocks, a.plan.n_split),
-                 dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, P);
+  e = launch_pdl(sparse_attn_tc_kernel<kMasked>, dim3(a.Nq, head_blocks, a.plan.n_split),
+                 dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, kvmap, P);
   if (e != cudaSuccess || a.plan.n_split == 1) return e;
   return launch_attn_merge(a, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_sparse_attn_tc(const AttnArgs& a, cudaStream_t stream) {
+  return launch_tc<false>(a, stream);
+}
+
+AttnPlan masked_attn_plan(int Nq, int H, int64_t max_len, int num_sms) {
+  AttnPlan p;
+  p.decode = 0;
+  p.tc = 1;
+  p.hb = kHB;
+  p.head_blocks = (H + kHB - 1) / kHB;
+  // Chunks of the causal positions: about one wave of CTAs, at most
+  // kMaskWords * 32 positions each, whole tiles.
+  const long long base = static_cast<long long>(Nq) * p.head_blocks;
+  int n = static_cast<int>(std::max<long long>(1, num_sms / std::max<long long>(1, base)));
+  n = std::max(n, static_cast<int>((max_len + kMaskWords * 32 - 1) / (kMaskWords * 32)));
+  n = std::min(n, 64);
+  int per = static_cast<int>((max_len + n - 1) / n);
+  per = (per + kT - 1) / kT * kT;
+  p.split_len = std::max(per, kT);
+  p.n_split = static_cast<int>((max_len + p.split_len - 1) / p.split_len);
+  if (p.n_split < 1) p.n_split = 1;
+  return p;
+}
+
+bool masked_attn_supported(int64_t max_len) {
+  return max_len <= static_cast<int64_t>(64) * kMaskWords * 32;
+}
+
+cudaError_t launch_masked_attn(const AttnArgs& a, cudaStream_t stream) {
+  return launch_tc<true>(a, stream);
 }
 
 }  // namespace dsa

@@ -96,6 +96,8 @@ typedef enum {
  * time limit (about a second); the call then leaves DSA_ERR_DEVICE_TIMEOUT in
  * the workspace, and its outputs are undefined. */
 #define DSA_FLAG_TEST_STALL 0x80000000u
+/* dsa_workspace_size: the size also covers dsa_masked_attn on the batch. */
+#define DSA_FLAG_MASKED_ROUTE 0x2u
 
 /*
  * A batch of sequences.  Sequence b owns
@@ -123,8 +125,9 @@ typedef struct {
 } dsa_batch;
 
 /* Bytes of workspace that dsa_layer_forward needs for this batch; it is also
- * enough for every other call on the same batch, H and top_k.  Returns 0 for
- * an invalid batch.  `flags` is reserved, pass 0. */
+ * enough for every other call on the same batch, H and top_k (with
+ * DSA_FLAG_MASKED_ROUTE in `flags`, for dsa_masked_attn too; otherwise pass
+ * 0).  Returns 0 for an invalid batch or flag. */
 DSA_API size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t flags);
 
 /*
@@ -189,6 +192,22 @@ DSA_API dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t
 DSA_API dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, const uint16_t* kv,
                            const int32_t* idx, int top_k, float scale, float* out, float* lse,
                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Step 3 the way the pages describe llama.cpp doing it, kept as a measured
+ * comparison (aiaulis.com paragraph 4; devotd.net section 2: the selection
+ * is applied as a mask over the whole cache so that the existing sparse
+ * flash attention can be reused; off that path the cost is full-cache
+ * attention).  Same arguments, result and error rules as dsa_sparse_attn
+ * (results agree within the library's tolerances), but it reads every cached
+ * row 0..p of each query and masks the logits of the rows idx does not list,
+ * instead of gathering only the listed rows.  Needs the workspace size that
+ * dsa_workspace_size reports with DSA_FLAG_MASKED_ROUTE; contexts up to 2^21.
+ */
+DSA_API dsa_status dsa_masked_attn(const dsa_batch* batch, const uint16_t* q, int H,
+                                   const uint16_t* kv, const int32_t* idx, int top_k, float scale,
+                                   float* out, float* lse, void* ws, size_t ws_bytes,
+                                   void* stream);
 
 /*
  * The whole DSA layer: dsa_indexer_score -> dsa_topk -> dsa_sparse_attn,

@@ -25,7 +25,7 @@ def test_header_declares_the_boundary():
         "dsa_workspace_size", "dsa_indexer_score", "dsa_topk", "dsa_sparse_attn",
         "dsa_layer_forward", "dsa_check_device_status", "dsa_status_string",
         "dsa_sparse_attn_noalloc", "dsa_indexer_project_workspace_size",
-        "dsa_indexer_project"])
+        "dsa_indexer_project", "dsa_masked_attn"])
 
 
 def test_library_exports_every_declared_symbol():
