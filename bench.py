@@ -286,7 +286,7 @@ def launches_per_layer(wl, sms=148):
     per = -(-max_len // chunks)
     chunk = min(max(512, -(-per // 512) * 512), 8192)
     hist = (0 < wl.Nq <= 148 and max_len >= 8192 and max_len >= 4 * wl.top_k
-            and int(nq.max()) <= 1 and -(-max_len // chunk) <= 512)
+            and -(-max_len // chunk) <= 512)
     C = 148 // max(1, wl.Nq)
     fused = (hist and wl.H <= 64 and wl.Nq <= 16 and C >= 8
              and (-(-max_len // C) + 31) // 32 <= 512)
@@ -467,7 +467,9 @@ def run_ours(args):
                           lambda: decode_workload_bench(bd, synth.decode_b8_32k(), dev, peaks,
                                                         50, 3, args.with_oracle)),
                          ("ragged_B32", lambda: ragged_bench(bd, dev, peaks, 50, 3,
-                                                             with_oracle=args.with_oracle))):
+                                                             with_oracle=args.with_oracle)),
+                         ("attention_routes_B4_L131072",
+                          lambda: mask_route_bench(bd, dev, peaks, 20, 3))):
             other[key] = _safe(run)
             torch.cuda.empty_cache()
         line["other_workloads"] = other
@@ -858,6 +860,49 @@ def ragged_bench(bd, dev, peaks, steps, warmup, layers=24, with_oracle=False):
                            "achieved_gbs": gbs, "peak": peaks["hbm_gbs"],
                            "frac": gbs / peaks["hbm_gbs"],
                            "note": "layers' algorithmic bytes only; glue time included"}}
+    return res
+
+
+def mask_route_bench(bd, dev, peaks, steps, warmup):
+    """The two ways to run step 3 on the 128K decode workload, each on the
+    layer's own index sets, L2 flushed before every timed call: the gather of
+    the selected latent rows (this library's route) and the mask over the
+    whole cache (the route the pages describe for llama.cpp)."""
+    wl = synth.decode_b4_128k()
+    dw = bd.DeviceWorkload(wl, dev)
+    ws = bd.alloc_workspace(dw.batch, wl.H, wl.top_k, dev, flags=bd.FLAG_MASKED_ROUTE)
+    out, lse, idx = dw.new_outputs()
+    dw.forward(out, lse, idx)
+    o2, l2 = torch.empty_like(out), torch.empty_like(lse)
+    res = {"workload": wl.name}
+    L = wl.ctx_lens.astype(np.int64)
+    per_q = wl.H * synth.D * 2 + wl.H * synth.DV * 4 + wl.H * 4 + wl.top_k * 4
+    routes = {
+        "gather": (lambda: bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, o2, l2,
+                                          ws),
+                   int((np.minimum(wl.top_k, L) * synth.D * 2).sum()) + per_q * wl.Nq),
+        "mask_whole_cache": (lambda: bd.masked_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k,
+                                                    wl.scale, o2, l2, ws),
+                             int((L * synth.D * 2).sum()) + per_q * wl.Nq),
+    }
+    kidx = int((L * synth.DI * 2).sum()) + wl.Nq * (synth.HI * synth.DI * 2 + synth.HI * 4)
+    for name, (fn, nbytes) in routes.items():
+        g = _graph_of(fn, dev)
+        ms = _time_flushed(g, steps, warmup, dev)
+        bd.check_device_status(ws)
+        del g
+        res[name] = {"attention_ms": ms, "attention_bytes_per_call": nbytes,
+                     "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "layer_bytes_per_token_mb": (kidx + nbytes) / wl.Nq / 1e6}
+    # both routes compute the same attention
+    bd.masked_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, o2, l2, ws)
+    bd.sparse_attn(dw.batch, dw.q, dw.kv, idx, wl.top_k, wl.scale, out, lse, ws)
+    torch.cuda.synchronize()
+    res["max_abs_diff_between_routes"] = float((o2 - out).abs().max().item())
+    res["mask_over_gather_time"] = res["mask_whole_cache"]["attention_ms"] / res["gather"][
+        "attention_ms"]
+    del dw, ws, out, lse, idx, o2, l2
     return res
 
 

@@ -120,11 +120,11 @@ struct WsLayout {
   AttnPlan plan;
 };
 
-// Few long rows with one query per sequence (decode): the indexer builds the
-// score-key histograms and the selection makes one filtering pass.
+// Few long rows (decode, one or a few new tokens per sequence): the indexer
+// builds the score-key histograms and the selection makes one filtering pass.
 bool plan_hist_topk(const dsa_batch* b, const BatchInfo& info, int top_k) {
   return b->Nq > 0 && b->Nq <= kPlanSms && info.max_len >= 8192 &&
-         info.max_len >= 4LL * top_k && indexer_single_query_items(b->h_q_offsets, b->B) &&
+         info.max_len >= 4LL * top_k &&
          topk_hist_supported(b->Nq, info.max_len);
 }
 
@@ -162,7 +162,7 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.total = w.part_off + w.part_bytes;
   // The standalone calls with DSA_FLAG_SCORE_HISTOGRAM keep the histogram
   // region right after the control block.
-  if (scores && attn && indexer_single_query_items(b->h_q_offsets, b->B)) {
+  if (scores && attn) {
     w.total = std::max(w.total, standalone_hist_need(b, info, top_k));
   }
   return w;
@@ -252,9 +252,6 @@ dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, cons
   DSA_TRY(check_batch(batch, &info));
   if ((flags & ~DSA_FLAG_SCORE_HISTOGRAM) != 0u) return DSA_ERR_INVALID_ARG;
   const bool hist = (flags & DSA_FLAG_SCORE_HISTOGRAM) != 0u;
-  if (hist && !indexer_single_query_items(batch->h_q_offsets, batch->B)) {
-    return DSA_ERR_UNSUPPORTED;
-  }
   if (batch->Nq == 0) return DSA_OK;
   DSA_TRY(check_ptr(q_idx));
   DSA_TRY(check_ptr(w));

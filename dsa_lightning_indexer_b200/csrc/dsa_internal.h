@@ -48,9 +48,6 @@ struct IndexerArgs {
   int* hist;          // per-row score-key histograms to accumulate, or null
   bool test_stall;    // test only: the TMA producer issues nothing (every wait runs out)
 };
-// True when the indexer launch for this batch processes one query per item
-// (the only case in which it can build the histograms).
-bool indexer_single_query_items(const int32_t* h_q_offsets, int B);
 cudaError_t launch_indexer_score(const IndexerArgs& a, cudaStream_t stream);
 
 struct TopkArgs {

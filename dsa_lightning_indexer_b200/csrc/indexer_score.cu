@@ -21,11 +21,13 @@
 // A work item is (sequence, group of QT queries, chunk of key tiles); items
 // are dealt to CTAs in snake order so causal prefill work balances.
 //
-// Optionally (one query per item), the epilogue also counts each stored score
-// into a 4096-bin histogram of the top 12 bits of its order-preserving key
-// (shared memory, one aggregated atomic per warp per distinct bin), flushed to
-// the row's global histogram after each item; the top-k selection then needs
-// only one filtering pass over the row.
+// Optionally, the epilogue also counts each stored score into its row's
+// 4096-bin histogram of the top 12 bits of its order-preserving key; the
+// top-k selection then needs only one filtering pass over the row.  With one
+// query per item the counts gather in shared memory (one aggregated atomic
+// per warp per distinct bin) and are flushed to the row's histogram after
+// each item; with several queries per item (multi-token decode) each warp
+// adds its aggregated counts to the rows' global histograms directly.
 #include <string.h>
 
 #include <algorithm>
@@ -288,7 +290,8 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 in the first set
     const int jset = (warp - 2) >> 2;                    // this warp's epilogue set
-    const bool do_hist = (QT == 1) && P.hist != nullptr;
+    const bool do_hist = (QT == 1) && P.hist != nullptr;     // shared-memory histogram
+    const bool do_ghist = (QT > 1) && P.hist != nullptr;     // straight to the row's
     if (do_hist) {
       for (int i = et; i < kHistBins; i += kEpiThreads) shist[i] = 0;
       named_bar_sync_idx(1, kEpiThreads);
@@ -327,10 +330,17 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           if (s == 0.f) s = 0.f;  // one zero: -0 and +0 are the same score
           const bool valid = key <= v.pos0 + jq;
           if (valid) P.scores[static_cast<size_t>(v.row0 + jq) * P.ld + key] = s;
-          if (do_hist) {
+          if (do_hist || do_ghist) {
             const uint32_t bin = valid ? (score_key(s) >> kHistShift) : 0xFFFFFFFFu;
             const unsigned grp = __match_any_sync(0xffffffffu, bin);
-            if (valid && lane == __ffs(grp) - 1) atomicAdd(&shist[bin], __popc(grp));
+            if (valid && lane == __ffs(grp) - 1) {
+              if (do_hist) {
+                atomicAdd(&shist[bin], __popc(grp));
+              } else {
+                atomicAdd(P.hist + static_cast<size_t>(v.row0 + jq) * kHistBins + bin,
+                          __popc(grp));
+              }
+            }
           }
         }
         tc_fence_before();
@@ -413,7 +423,7 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.scores = a.scores;
     P.ld = a.ld;
     P.err = a.err;
-    P.hist = QT == 1 ? a.hist : nullptr;
+    P.hist = a.hist;
     P.stall = a.test_stall ? 1 : 0;
     int items = 0, n = 0;
     for (; b < a.B && n < kMaxSeqPerLaunch; ++b) {
@@ -442,13 +452,6 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
-
-bool indexer_single_query_items(const int32_t* h_q_offsets, int B) {
-  for (int b = 0; b < B; ++b) {
-    if (h_q_offsets[b + 1] - h_q_offsets[b] > 1) return false;
-  }
-  return true;
-}
 
 cudaError_t launch_indexer_score(const IndexerArgs& a, cudaStream_t stream) {
   int max_nq = 0;

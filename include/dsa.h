@@ -145,8 +145,7 @@ DSA_API size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint
  *   flags   0, or DSA_FLAG_SCORE_HISTOGRAM: also count every score of each
  *           row into a 4096-bin histogram of its top 12 order-preserving key
  *           bits, kept in the workspace for a following dsa_topk with the
- *           same flag (as the fused layer does for decode).  Needs at most
- *           one query per sequence (else DSA_ERR_UNSUPPORTED).
+ *           same flag (as the fused layer does for decode).
  * Runs on tcgen05 tensor cores (bf16 products, fp32 accumulation).
  */
 DSA_API dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, const float* w,

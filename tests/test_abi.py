@@ -131,7 +131,6 @@ def test_valid_call_without_a_b200_is_refused():
 
 def test_flag_validation():
     b = FakeBatch([0, 1], [0, 64], [64])
-    multi = FakeBatch([0, 2], [0, 64], [64])                    # two queries in one sequence
     hist, stall = bd.FLAG_SCORE_HISTOGRAM, bd.FLAG_TEST_STALL
 
     def score(batch, flags):
@@ -143,7 +142,6 @@ def test_flag_validation():
                                         None, FAKE, FAKE, 1 << 30, flags, None)
     assert score(b, 0x2) == bd.ERR_INVALID_ARG                 # reserved bit
     assert score(b, stall) == bd.ERR_INVALID_ARG               # a layer-only flag
-    assert score(multi, hist) == bd.ERR_UNSUPPORTED            # histogram: one query per sequence
     assert _topk(b, flags=0x4) == bd.ERR_INVALID_ARG
     assert _topk(b, flags=stall) == bd.ERR_INVALID_ARG
     assert layer(hist) == bd.ERR_INVALID_ARG                   # the layer builds it itself

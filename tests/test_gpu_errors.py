@@ -139,11 +139,24 @@ def test_standalone_histogram_path_matches_the_layer():
     assert np.array_equal(sets[0], want)
 
 
-def test_histogram_flag_needs_one_query_per_sequence():
-    wl = synth.custom([300, 500], [2, 1], 16, 64, seed=164)
+def test_multi_token_decode_takes_the_histogram_path():
+    """Several new tokens per sequence (items of 2, 4 and 8 queries): the
+    indexer builds every row's histogram, the fused layer and the standalone
+    histogram path give the same index sets, and they are the oracle's."""
+    wl = synth.custom([20000, 9000, 30000], [2, 4, 8], 64, 2048, seed=164)
     dw = bd.DeviceWorkload(wl)
-    scores = torch.zeros(wl.Nq, 500, device="cuda")
-    with pytest.raises(bd.DsaError) as e:
-        bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, 500, dw.ws,
-                         flags=bd.FLAG_SCORE_HISTOGRAM)
-    assert e.value.status == bd.ERR_UNSUPPORTED
+    lay_out, lay_lse, lay_idx = (t.cpu().numpy() for t in dw.forward())
+    bd.check_device_status(dw.ws)
+    ld = _up4(wl.ctx_lens.max())
+    scores = torch.full((wl.Nq, ld), float("nan"), device="cuda")
+    bd.indexer_score(dw.batch, dw.q_idx, dw.w, dw.k_idx, scores, ld, dw.ws,
+                     flags=bd.FLAG_SCORE_HISTOGRAM)
+    idx = torch.full((wl.Nq, wl.top_k), -7, dtype=torch.int32, device="cuda")
+    bd.topk(dw.batch, scores, ld, wl.top_k, idx, dw.ws, flags=bd.FLAG_SCORE_HISTOGRAM)
+    bd.check_device_status(dw.ws)
+    assert np.array_equal(idx.cpu().numpy(), lay_idx)
+    ref_scores, ref_idx, _, _ = oracle.dsa_layer(*_args(wl), wl.q_idx, wl.w, wl.k_idx, wl.q,
+                                                 wl.kv, wl.top_k, wl.scale, ld=ld)
+    parity.check_selection(lay_idx, ref_idx, ref_scores, wl)
+    att_out, att_lse = oracle.sparse_attn(*_args(wl), wl.q, wl.kv, lay_idx, wl.scale)
+    parity.check_attention(lay_out, lay_lse, att_out, att_lse)
