@@ -89,28 +89,41 @@ def _check(status: int, where: str) -> None:
 class _CBatch(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Nq", ctypes.c_int32),
                 ("q_offsets", _P), ("kv_offsets", _P), ("ctx_lens", _P),
-                ("h_q_offsets", _P), ("h_kv_offsets", _P), ("h_ctx_lens", _P)]
+                ("h_q_offsets", _P), ("h_kv_offsets", _P), ("h_ctx_lens", _P),
+                ("page_size", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("block_table", _P), ("h_block_table", _P), ("cache_rows", ctypes.c_int64)]
 
 
 class Batch:
-    """Sequence layout of one call: device arrays plus the host mirrors."""
+    """Sequence layout of one call: device arrays plus the host mirrors.
 
-    def __init__(self, q_offsets, kv_offsets, ctx_lens, device="cuda"):
+    Contiguous caches: kv_offsets [B+1].  Paged caches: give page_size (a
+    power of two >= 64), block_table [B, max_blocks] int32 page numbers and
+    cache_rows; kv_offsets may then be None."""
+
+    def __init__(self, q_offsets, kv_offsets, ctx_lens, device="cuda", page_size=0,
+                 block_table=None, cache_rows=0):
         self.h_q_offsets = np.ascontiguousarray(q_offsets, dtype=np.int32)
-        self.h_kv_offsets = np.ascontiguousarray(kv_offsets, dtype=np.int64)
+        self.h_kv_offsets = (None if kv_offsets is None
+                             else np.ascontiguousarray(kv_offsets, dtype=np.int64))
         self.h_ctx_lens = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+        self.h_block_table = (None if block_table is None
+                              else np.ascontiguousarray(block_table, dtype=np.int32))
         self.B = int(self.h_ctx_lens.shape[0])
         self.Nq = int(self.h_q_offsets[-1]) if self.h_q_offsets.size else 0
-        if device is None:
-            self.q_offsets = self.kv_offsets = self.ctx_lens = None
-        else:
-            self.q_offsets = torch.from_numpy(self.h_q_offsets).to(device)
-            self.kv_offsets = torch.from_numpy(self.h_kv_offsets).to(device)
-            self.ctx_lens = torch.from_numpy(self.h_ctx_lens).to(device)
+        to_dev = (lambda a: None if a is None or device is None
+                  else torch.from_numpy(a).to(device))
+        self.q_offsets = to_dev(self.h_q_offsets)
+        self.kv_offsets = to_dev(self.h_kv_offsets)
+        self.ctx_lens = to_dev(self.h_ctx_lens)
+        self.block_table = to_dev(self.h_block_table)
         dp = (lambda t: t.data_ptr() if t is not None else None)
+        hp = (lambda a: a.ctypes.data if a is not None else None)
+        max_blocks = int(self.h_block_table.shape[1]) if self.h_block_table is not None else 0
         self.c = _CBatch(self.B, self.Nq, dp(self.q_offsets), dp(self.kv_offsets),
-                         dp(self.ctx_lens), self.h_q_offsets.ctypes.data,
-                         self.h_kv_offsets.ctypes.data, self.h_ctx_lens.ctypes.data)
+                         dp(self.ctx_lens), hp(self.h_q_offsets), hp(self.h_kv_offsets),
+                         hp(self.h_ctx_lens), int(page_size), max_blocks,
+                         dp(self.block_table), hp(self.h_block_table), int(cache_rows))
 
     @property
     def ref(self):
@@ -122,6 +135,10 @@ class Batch:
 
     @classmethod
     def from_workload(cls, wl, device="cuda"):
+        pg = getattr(wl, "paged", None)
+        if pg is not None:
+            return cls(wl.q_offsets, None, wl.ctx_lens, device, page_size=pg.page_size,
+                       block_table=pg.block_table, cache_rows=pg.cache_rows)
         return cls(wl.q_offsets, wl.kv_offsets, wl.ctx_lens, device)
 
 
@@ -250,11 +267,12 @@ class DeviceWorkload:
     def __init__(self, wl, device="cuda"):
         self.wl = wl
         self.batch = Batch.from_workload(wl, device)
+        pg = getattr(wl, "paged", None)
         self.q_idx = bf16_tensor(wl.q_idx, device)
         self.w = torch.from_numpy(wl.w).to(device)
-        self.k_idx = bf16_tensor(wl.k_idx, device)
+        self.k_idx = bf16_tensor(wl.k_idx if pg is None else pg.k_idx, device)
         self.q = bf16_tensor(wl.q, device)
-        self.kv = bf16_tensor(wl.kv, device)
+        self.kv = bf16_tensor(wl.kv if pg is None else pg.kv, device)
         self.top_k = wl.top_k
         self.scale = wl.scale
         self.H = wl.H

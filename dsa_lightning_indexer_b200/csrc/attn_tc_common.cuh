@@ -15,7 +15,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 struct TcParams {
   const int32_t* q_offsets;
-  const int64_t* kv_offsets;
+  CacheLayout cache;
   const int32_t* ctx_lens;
   const __nv_bfloat16* kv;
   const int32_t* idx;
@@ -133,32 +133,34 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
 }
 
 // Sequence facts of query row r, looked up by each warp with all of its
-// loads in flight at once (lane l checks sequences l, l + 32, ...): the
-// sequence's first cache row and the row's causal length p + 1.
+// loads in flight at once (lane l checks sequences l, l + 32, ...): where the
+// sequence's positions live in the caches and the row's causal length p + 1.
 struct RowSeq {
-  long long kv0;
+  SeqRows rows;
   int len;
 };
 
-__device__ __forceinline__ RowSeq row_seq_warp(const int32_t* q_offsets, const int64_t* kv_offsets,
+__device__ __forceinline__ RowSeq row_seq_warp(const int32_t* q_offsets, const CacheLayout& cache,
                                                const int32_t* ctx_lens, int B, int r) {
   long long kv0 = 0;
-  int len = 0, hit = 0;
+  int len = 0, hit = 0, seq = 0;
   for (int b = threadIdx.x & 31; b < B; b += 32) {
     const int q0 = __ldg(q_offsets + b), q1 = __ldg(q_offsets + b + 1);
-    const long long k0 = __ldg(kv_offsets + b);
+    const long long k0 = cache.block_table ? 0 : __ldg(cache.kv_offsets + b);
     const int L = __ldg(ctx_lens + b);
     if (r >= q0 && r < q1) {
       kv0 = k0;
       len = L - (q1 - q0) + (r - q0) + 1;
       hit = 1;
+      seq = b;
     }
   }
   const unsigned m = __ballot_sync(0xffffffffu, hit);
   const int src = m ? __ffs(m) - 1 : 0;
   RowSeq rs;
-  rs.kv0 = __shfl_sync(0xffffffffu, kv0, src);
   rs.len = __shfl_sync(0xffffffffu, len, src);
+  rs.rows = seq_rows(cache, __shfl_sync(0xffffffffu, seq, src),
+                     __shfl_sync(0xffffffffu, kv0, src));
   return rs;
 }
 

@@ -73,7 +73,8 @@ constexpr int kOffSel = kOffTile + kMaxWords * 4;        // selected bits
 constexpr int kOffPre = kOffSel + kMaxWords * 4;         // tile-set prefix per word
 constexpr int kOffTpos = kOffPre + kMaxWords * 4;        // [kTile] positions of the tile rows
 constexpr int kOffTsel = kOffTpos + kTile * 4;           // [kTile] selected flags
-constexpr int kOffAlpha = kOffTsel + kTile * 4;          // [64]
+constexpr int kOffTrow = kOffTsel + kTile * 4;           // [kTile] cache rows of the tile
+constexpr int kOffAlpha = kOffTrow + kTile * 4;          // [64]
 constexpr int kOffScan = kOffAlpha + kHB * 4;            // block scan buffer
 constexpr int kOffMisc = kOffScan + 128;                 // shared scalars
 constexpr int kOffBar = kOffMisc + 128;
@@ -101,7 +102,7 @@ enum {
 
 struct TailParams {
   const int32_t* q_offsets;
-  const int64_t* kv_offsets;
+  CacheLayout cache;
   const int32_t* ctx_lens;
   const __nv_bfloat16* kv;
   const float* scores;
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* const pre = reinterpret_cast<int*>(bp + kOffPre);
   int* const tpos = reinterpret_cast<int*>(bp + kOffTpos);
   int* const tsel = reinterpret_cast<int*>(bp + kOffTsel);
+  int* const trow = reinterpret_cast<int*>(bp + kOffTrow);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
   int* const buf = reinterpret_cast<int*>(bp + kOffScan);
   int* const misc = reinterpret_cast<int*>(bp + kOffMisc);
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sQ + j * kQBox, &qmap, b_qfull, 64 * j, r * P.H, pol);
     }
   }
-  const RowSeq rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
+  const RowSeq rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
   pdl_wait();
   pdl_launch_dependents();
   if (tid == 0 && error_recorded(P.err)) misc[kMAbort] = 1;
@@ -343,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pos = s0 + 32 * lo + bit;
       }
       tpos[tid] = pos;
+      trow[tid] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
     }
   };
   // Every thread copies its share of the tile's rows (16-byte cp.async,
@@ -350,11 +353,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto gather_tile = [&]() {
     for (int item = tid; item < kTile * kBoxes; item += kThreads) {
       const int bx = item / kTile, i = item - bx * kTile;
-      const int pos = tpos[i];
+      const int row = trow[i];
       const uint32_t drow = sKV + bx * kKVBox + i * 128;
       const uint32_t x = static_cast<uint32_t>(i & 7);
-      if (pos >= 0) {
-        const __nv_bfloat16* src = P.kv + static_cast<size_t>(rs.kv0 + pos) * kLatent + bx * 64;
+      if (row >= 0) {
+        const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
 #pragma unroll
         for (uint32_t cc = 0; cc < 8; ++cc) cp_async16_tc(drow + ((cc ^ x) << 4), src + cc * 8);
       } else {
@@ -872,7 +875,7 @@ cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream) {
   const int C = decode_tail_chunks(a.Nq, a.num_sms);
   TailParams P;
   P.q_offsets = a.q_offsets;
-  P.kv_offsets = a.kv_offsets;
+  P.cache = a.cache;
   P.ctx_lens = a.ctx_lens;
   P.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
   P.scores = a.scores;

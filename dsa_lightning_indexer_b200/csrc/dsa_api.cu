@@ -33,22 +33,46 @@ dsa_status check_batch(const dsa_batch* b, BatchInfo* info) {
   if (!b || b->B < 0 || b->Nq < 0) return DSA_ERR_INVALID_ARG;
   info->max_len = 0;
   info->cache_rows = 0;
+  info->page_shift = 0;
+  if (b->page_size < 0) return DSA_ERR_INVALID_ARG;
+  const bool paged = b->page_size > 0;
+  if (paged) {
+    if (b->page_size < 64 || (b->page_size & (b->page_size - 1)) != 0) return DSA_ERR_UNSUPPORTED;
+    while ((1 << info->page_shift) < b->page_size) ++info->page_shift;
+  }
   if (b->B == 0) return b->Nq == 0 ? DSA_OK : DSA_ERR_INVALID_ARG;
-  if (!b->q_offsets || !b->kv_offsets || !b->ctx_lens || !b->h_q_offsets || !b->h_kv_offsets ||
-      !b->h_ctx_lens) {
+  if (!b->q_offsets || !b->ctx_lens || !b->h_q_offsets || !b->h_ctx_lens) {
     return DSA_ERR_INVALID_ARG;
   }
-  if (b->h_q_offsets[0] != 0 || b->h_q_offsets[b->B] != b->Nq || b->h_kv_offsets[0] < 0) {
-    return DSA_ERR_INVALID_ARG;
+  if (b->h_q_offsets[0] != 0 || b->h_q_offsets[b->B] != b->Nq) return DSA_ERR_INVALID_ARG;
+  if (paged) {
+    if (!b->block_table || !b->h_block_table || b->max_blocks < 1 || b->cache_rows <= 0 ||
+        b->cache_rows % b->page_size != 0) {
+      return DSA_ERR_INVALID_ARG;
+    }
+    info->cache_rows = b->cache_rows;
+  } else {
+    if (!b->kv_offsets || !b->h_kv_offsets || b->h_kv_offsets[0] < 0) return DSA_ERR_INVALID_ARG;
+    info->cache_rows = b->h_kv_offsets[b->B];
   }
+  const int64_t pages = paged ? b->cache_rows / b->page_size : 0;
   for (int i = 0; i < b->B; ++i) {
     const int64_t nq = static_cast<int64_t>(b->h_q_offsets[i + 1]) - b->h_q_offsets[i];
-    const int64_t cap = b->h_kv_offsets[i + 1] - b->h_kv_offsets[i];
     const int64_t L = b->h_ctx_lens[i];
-    if (nq < 0 || cap < 0 || L < 0 || nq > L || L > cap) return DSA_ERR_INVALID_ARG;
+    if (nq < 0 || L < 0 || nq > L) return DSA_ERR_INVALID_ARG;
+    if (paged) {
+      const int64_t used = (L + b->page_size - 1) / b->page_size;
+      if (used > b->max_blocks) return DSA_ERR_INVALID_ARG;
+      const int32_t* bt = b->h_block_table + static_cast<int64_t>(i) * b->max_blocks;
+      for (int64_t j = 0; j < used; ++j) {
+        if (bt[j] < 0 || bt[j] >= pages) return DSA_ERR_INVALID_ARG;
+      }
+    } else {
+      const int64_t cap = b->h_kv_offsets[i + 1] - b->h_kv_offsets[i];
+      if (cap < 0 || L > cap) return DSA_ERR_INVALID_ARG;
+    }
     if (L > info->max_len) info->max_len = L;
   }
-  info->cache_rows = b->h_kv_offsets[b->B];
   // Row coordinates of the tensor maps are 32-bit.
   if (info->cache_rows >= (int64_t(1) << 31) ||
       static_cast<int64_t>(b->Nq) * kIdxHeads >= (int64_t(1) << 31)) {
@@ -174,6 +198,16 @@ dsa_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return DSA_OK;
 }
 
+CacheLayout cache_layout(const dsa_batch* b, const BatchInfo& info) {
+  CacheLayout c;
+  const bool paged = b->page_size > 0;
+  c.kv_offsets = paged ? nullptr : b->kv_offsets;
+  c.block_table = paged ? b->block_table : nullptr;
+  c.max_blocks = paged ? b->max_blocks : 0;
+  c.page_shift = info.page_shift;
+  return c;
+}
+
 inline dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
 inline unsigned* err_word(void* ws) {
@@ -196,6 +230,7 @@ IndexerArgs indexer_args(const dsa_batch* b, const BatchInfo& info, const uint16
   a.h_ctx_lens = b->h_ctx_lens;
   a.Nq = b->Nq;
   a.cache_rows = info.cache_rows;
+  a.cache = cache_layout(b, info);
   a.q_idx = q_idx;
   a.w = w;
   a.k_idx = k_idx;
@@ -323,7 +358,7 @@ dsa_status dsa_sparse_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.B = batch->B;
   a.Nq = batch->Nq;
   a.q_offsets = batch->q_offsets;
-  a.kv_offsets = batch->kv_offsets;
+  a.cache = cache_layout(batch, info);
   a.q = q;
   a.H = H;
   a.kv = kv;
@@ -356,7 +391,8 @@ dsa_status dsa_masked_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   DSA_TRY(check_ptr(out));
   if (lse) DSA_TRY(check_ptr(lse));
   if (!isfinite(scale)) return DSA_ERR_INVALID_ARG;
-  if (!masked_attn_supported(info.max_len)) return DSA_ERR_UNSUPPORTED;
+  // Contiguous caches only: the route streams each sequence's rows as tiles.
+  if (!masked_attn_supported(info.max_len) || batch->page_size > 0) return DSA_ERR_UNSUPPORTED;
   DSA_TRY(check_ws(ws, ws_bytes, masked_ws_need(batch, info, H)));
   int sms = 0;
   DSA_TRY(check_device(&sms));
@@ -364,7 +400,7 @@ dsa_status dsa_masked_attn(const dsa_batch* batch, const uint16_t* q, int H, con
   a.B = batch->B;
   a.Nq = batch->Nq;
   a.q_offsets = batch->q_offsets;
-  a.kv_offsets = batch->kv_offsets;
+  a.cache = cache_layout(batch, info);
   a.ctx_lens = batch->ctx_lens;
   a.q = q;
   a.H = H;
@@ -429,7 +465,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
     d.H = H;
     d.top_k = top_k;
     d.q_offsets = batch->q_offsets;
-    d.kv_offsets = batch->kv_offsets;
+    d.cache = cache_layout(batch, info);
     d.ctx_lens = batch->ctx_lens;
     d.q = q;
     d.kv = kv;
@@ -452,7 +488,7 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   a.B = batch->B;
   a.Nq = batch->Nq;
   a.q_offsets = batch->q_offsets;
-  a.kv_offsets = batch->kv_offsets;
+  a.cache = cache_layout(batch, info);
   a.q = q;
   a.H = H;
   a.kv = kv;
@@ -507,7 +543,7 @@ dsa_status dsa_indexer_project(const dsa_batch* batch, const uint16_t* x, int64_
   a.B = batch->B;
   a.T = batch->Nq;
   a.q_offsets = batch->q_offsets;
-  a.kv_offsets = batch->kv_offsets;
+  a.cache = cache_layout(batch, info);
   a.ctx_lens = batch->ctx_lens;
   a.x = x;
   a.c_q = c_q;

@@ -38,6 +38,38 @@ static_assert(kControlBytes == 256, "control block is 256 bytes");
 // pipeline, short enough that a broken one returns control to the host.
 constexpr long long kWaitCycles = 2000000000LL;
 
+// Where the positions of a batch's sequences live in the caches: contiguous
+// rows from kv_offsets[b], or pages of 2^page_shift rows listed in
+// block_table[b * max_blocks ...] (block_table non-null).
+struct CacheLayout {
+  const int64_t* kv_offsets;   // device (contiguous caches)
+  const int32_t* block_table;  // device (paged caches) or null
+  int max_blocks;
+  int page_shift;
+};
+
+// One sequence's part of a CacheLayout.
+struct SeqRows {
+  long long kv0;       // contiguous: the sequence's first row
+  const int32_t* bt;   // paged: its block-table row, else null
+  int page_shift;
+};
+
+__device__ __forceinline__ SeqRows seq_rows(const CacheLayout& c, int b, long long kv0) {
+  SeqRows s;
+  s.page_shift = c.page_shift;
+  s.bt = c.block_table ? c.block_table + static_cast<size_t>(b) * c.max_blocks : nullptr;
+  s.kv0 = c.block_table ? 0 : kv0;
+  return s;
+}
+
+// Cache row of position `pos` of the sequence.
+__device__ __forceinline__ long long seq_row(const SeqRows& s, int pos) {
+  if (s.bt == nullptr) return s.kv0 + pos;
+  return (static_cast<long long>(__ldg(s.bt + (pos >> s.page_shift))) << s.page_shift) |
+         static_cast<long long>(pos & ((1 << s.page_shift) - 1));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -17,8 +17,10 @@ namespace dsa {
 // Shared by every entry point; each returns DSA_OK or the status to report.
 struct BatchInfo {
   int64_t max_len;     // longest context
-  int64_t cache_rows;  // kv_offsets[B]
+  int64_t cache_rows;  // rows of the caches: kv_offsets[B], or the paged caches' rows
+  int page_shift;      // log2(page_size) for paged caches, 0 for contiguous ones
 };
+
 bool aligned16(const void* p);
 // The batch layout (host mirrors) is consistent and within the 32-bit row
 // coordinates of the tensor maps; fills `info`.
@@ -34,10 +36,11 @@ dsa_status check_device(int* num_sms);
 struct IndexerArgs {
   int B;
   const int32_t* h_q_offsets;   // host mirrors of the batch
-  const int64_t* h_kv_offsets;
+  const int64_t* h_kv_offsets;  // contiguous caches (planning only)
   const int32_t* h_ctx_lens;
   int Nq;
-  int64_t cache_rows;   // rows of k_idx (kv_offsets[B])
+  int64_t cache_rows;   // rows of k_idx
+  CacheLayout cache;    // device: where each sequence's positions live
   const uint16_t* q_idx;
   const float* w;
   const uint16_t* k_idx;
@@ -80,7 +83,7 @@ cudaError_t launch_topk_hist(const TopkArgs& a, void* ws_region, cudaStream_t st
 struct DecodeTailArgs {
   int B, Nq, H, top_k;
   const int32_t* q_offsets;   // device
-  const int64_t* kv_offsets;  // device
+  CacheLayout cache;          // device: where each sequence's positions live
   const int32_t* ctx_lens;    // device
   const uint16_t* q;
   const uint16_t* kv;
@@ -106,7 +109,7 @@ cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream);
 struct ProjectArgs {
   int B, T;                   // sequences, new tokens (query rows)
   const int32_t* q_offsets;   // device
-  const int64_t* kv_offsets;  // device
+  CacheLayout cache;          // device: where each sequence's positions live
   const int32_t* ctx_lens;    // device
   const uint16_t* x;          // [T][d_model]
   const uint16_t* c_q;        // [T][d_q]
@@ -144,7 +147,7 @@ struct AttnArgs {
   int B;
   int Nq;
   const int32_t* q_offsets;   // device
-  const int64_t* kv_offsets;  // device
+  CacheLayout cache;          // device: where each sequence's positions live
   const int32_t* ctx_lens;    // device
   const uint16_t* q;
   int H;

@@ -48,7 +48,7 @@ constexpr int kMaxN = 128;                 // tokens per item
 
 struct ProjParams {
   const int32_t* q_offsets;
-  const int64_t* kv_offsets;
+  CacheLayout cache;
   const int32_t* ctx_lens;
   int B, T;                  // sequences, tokens (query rows)
   int N;                     // tokens per item (16..128, multiple of 16)
@@ -96,7 +96,7 @@ __device__ __forceinline__ void named_bar_sync_p(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Cache row of token (query row) t: kv_offsets[b] + its position.
+// Cache row of token (query row) t: the row of its position in its sequence.
 __device__ __forceinline__ long long token_cache_row(const ProjParams& P, int t) {
   int lo = 0, hi = P.B - 1;
   while (lo < hi) {
@@ -104,7 +104,9 @@ __device__ __forceinline__ long long token_cache_row(const ProjParams& P, int t)
     if (__ldg(P.q_offsets + mid) <= t) lo = mid; else hi = mid - 1;
   }
   const int q0 = __ldg(P.q_offsets + lo), q1 = __ldg(P.q_offsets + lo + 1);
-  return __ldg(P.kv_offsets + lo) + __ldg(P.ctx_lens + lo) - (q1 - q0) + (t - q0);
+  const SeqRows sr =
+      seq_rows(P.cache, lo, P.cache.block_table ? 0 : __ldg(P.cache.kv_offsets + lo));
+  return seq_row(sr, __ldg(P.ctx_lens + lo) - (q1 - q0) + (t - q0));
 }
 
 template <int N>
@@ -442,7 +444,7 @@ cudaError_t launch_indexer_project(const ProjectArgs& a, cudaStream_t stream) {
   ProjParams P;
   memset(&P, 0, sizeof(P));
   P.q_offsets = a.q_offsets;
-  P.kv_offsets = a.kv_offsets;
+  P.cache = a.cache;
   P.ctx_lens = a.ctx_lens;
   P.B = a.B;
   P.T = a.T;

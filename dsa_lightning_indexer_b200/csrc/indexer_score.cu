@@ -44,8 +44,8 @@ constexpr int kKBoxBytes = kKTileBytes / 2;              // 128 rows x 64 dims
 constexpr int kEpiThreads = 128;  // one epilogue set: a warp per TMEM lane quadrant
 
 struct SeqItems {
-  long long kv_off;
-  int q_off, nq, L, n_chunks, item_off, pad;
+  long long kv_off;   // contiguous caches: the sequence's first row
+  int q_off, nq, L, n_chunks, item_off, b;
 };
 static_assert(sizeof(SeqItems) == 32, "packed launch record");
 
@@ -58,6 +58,8 @@ struct IdxParams {
   unsigned* err;
   int* hist;  // [Nq][kHistBins] score-key histograms, or null
   int stall;  // test only: the TMA producer issues nothing, so every wait runs out
+  CacheLayout cache;     // paged caches: the block table (contiguous: kv_off above)
+  long long cache_rows;  // rows of k_idx (a row past them reads as zeros)
 };
 
 template <int QT>
@@ -82,7 +84,7 @@ struct Cfg {
 };
 
 struct ItemView {
-  int row0, nrow, pos0, kt0, kt1;
+  int row0, nrow, pos0, kt0, kt1, b;
   long long kv0;
 };
 
@@ -102,6 +104,7 @@ __device__ __forceinline__ bool decode_item(const IdxParams& P, int item, ItemVi
   v.kt0 = c * P.chunk_tiles;
   v.kt1 = min(v.kt0 + P.chunk_tiles, n_kt);
   v.kv0 = s.kv_off;
+  v.b = s.b;
   return v.kt0 < v.kt1;
 }
 
@@ -215,9 +218,26 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
             if (st == stage) k_last[st] = sph;
           }
           const uint32_t kdst = k_smem + stage * kKTileBytes;
-          const int row = static_cast<int>(v.kv0 + static_cast<long long>(kt) * kKeysPerTile);
-          tma_load_2d(kdst, &kmap, full(stage), 0, row, pol_stream);
-          tma_load_2d(kdst + kKBoxBytes, &kmap, full(stage), 64, row, pol_stream);
+          if (P.cache.block_table == nullptr) {
+            const int row = static_cast<int>(v.kv0 + static_cast<long long>(kt) * kKeysPerTile);
+            tma_load_2d(kdst, &kmap, full(stage), 0, row, pol_stream);
+            tma_load_2d(kdst + kKBoxBytes, &kmap, full(stage), 64, row, pol_stream);
+          } else {
+            // Paged caches: two runs of 64 keys, each inside one page (pages
+            // are 64 rows or more); a run past the item's keys reads zeros.
+            const int32_t* bt = P.cache.block_table + static_cast<size_t>(v.b) * P.cache.max_blocks;
+            const int shift = P.cache.page_shift;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int s = kt * kKeysPerTile + 64 * h;
+              const int row = s < v.pos0 + v.nrow
+                                  ? (__ldg(bt + (s >> shift)) << shift) + (s & ((1 << shift) - 1))
+                                  : static_cast<int>(P.cache_rows);
+              tma_load_2d(kdst + h * 64 * 128, &kmap, full(stage), 0, row, pol_stream);
+              tma_load_2d(kdst + kKBoxBytes + h * 64 * 128, &kmap, full(stage), 64, row,
+                          pol_stream);
+            }
+          }
           if (++stage == C::kStages) {
             stage = 0;
             sph ^= 1u;
@@ -389,8 +409,9 @@ template <int QT>
 cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
   using C = Cfg<QT>;
   CUtensorMap kmap, qmap;
+  const bool paged = a.cache.block_table != nullptr;
   if (!encode_bf16_2d(&kmap, a.k_idx, kIdxDim, static_cast<uint64_t>(a.cache_rows), 64,
-                      kKeysPerTile) ||
+                      paged ? 64 : kKeysPerTile) ||
       !encode_bf16_2d(&qmap, a.q_idx, kIdxDim, static_cast<uint64_t>(a.Nq) * kIdxHeads, 64,
                       C::N)) {
     return cudaErrorInvalidValue;
@@ -425,12 +446,15 @@ cudaError_t launch_qt(const IndexerArgs& a, cudaStream_t stream) {
     P.err = a.err;
     P.hist = a.hist;
     P.stall = a.test_stall ? 1 : 0;
+    P.cache = a.cache;
+    P.cache_rows = a.cache_rows;
     int items = 0, n = 0;
     for (; b < a.B && n < kMaxSeqPerLaunch; ++b) {
       const int nq = a.h_q_offsets[b + 1] - a.h_q_offsets[b];
       if (nq <= 0) continue;
       SeqItems& r = P.seq[n++];
-      r.kv_off = a.h_kv_offsets[b];
+      r.kv_off = paged ? 0 : a.h_kv_offsets[b];
+      r.b = b;
       r.q_off = a.h_q_offsets[b];
       r.nq = nq;
       r.L = a.h_ctx_lens[b];

@@ -33,7 +33,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 
 struct AttnParams {
   const int32_t* q_offsets;
-  const int64_t* kv_offsets;
+  CacheLayout cache;
   const int32_t* ctx_lens;
   unsigned* err;        // error word for dropped index entries, or null
   const __nv_bfloat16* q;
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
   pdl_wait();
   pdl_launch_dependents();
   const int b = owner_seq(P.q_offsets, P.B, r);
-  const long long kv0 = P.kv_offsets[b];
+  const SeqRows sr = seq_rows(P.cache, b, P.cache.block_table ? 0 : P.cache.kv_offsets[b]);
   // Causal length p + 1 of the row: only positions below it are read.
   const int row_len = P.ctx_lens[b] - (P.q_offsets[b + 1] - P.q_offsets[b]) +
                       (r - P.q_offsets[b]) + 1;
@@ -157,7 +157,7 @@ __global__ void __launch_bounds__(NG * 128, 1) sparse_attn_kernel(const AttnPara
       if (ch == 0) tidx[buf * kTileRows + i] = pos;
       if (pos >= 0) {
         cp_async16(smem_u32(dstb + i * kRowPad + ch * 8),
-                   P.kv + (static_cast<size_t>(kv0 + pos)) * kLatent + ch * 8);
+                   P.kv + static_cast<size_t>(seq_row(sr, pos)) * kLatent + ch * 8);
       } else {
         *reinterpret_cast<uint4*>(dstb + i * kRowPad + ch * 8) = make_uint4(0, 0, 0, 0);
       }
@@ -499,7 +499,7 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream) {
   if (a.plan.tc) return launch_sparse_attn_tc(a, stream);
   AttnParams P;
   P.q_offsets = a.q_offsets;
-  P.kv_offsets = a.kv_offsets;
+  P.cache = a.cache;
   P.ctx_lens = a.ctx_lens;
   P.err = a.err;
   P.q = reinterpret_cast<const __nv_bfloat16*>(a.q);

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Inside the layer the batch arrays are inputs no earlier kernel writes:
   // look the row up while the previous kernel finishes.
   RowSeq rs = {};
-  if (P.batch_ready) rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
+  if (P.batch_ready) rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
   pdl_wait();
   pdl_launch_dependents();
 
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       pos_raw = __ldg(P.idx + static_cast<size_t>(r) * P.top_k + slot);
     }
   }
-  if (!P.batch_ready) rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
+  if (!P.batch_ready) rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
   const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
   const bool work = slot_lo < n_slots;  // block-uniform
 
@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           atomicOr(P.err, kErrIndex);
           pos = -1;
         }
-        tidx[g] = pos;
+        // The slot's cache row (-1: nothing to read).
+        tidx[g] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
       }
       named_bar_sync(2, kGatherThreads);
       // Each thread copies whole 128-byte box rows: eight 16-byte pieces with
@@ -141,11 +142,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the swizzled 16-byte pieces of one instruction spread over all
         // eight bank groups of shared memory.
         const int bx = item / kTD, i = item - bx * kTD;
-        const int pos = tidx[i];
+        const int row = tidx[i];
         const uint32_t drow = sKV + bx * kKVBox + i * 128;
         const uint32_t x = static_cast<uint32_t>(i & 7);
-        if (pos >= 0) {
-          const __nv_bfloat16* src = P.kv + static_cast<size_t>(rs.kv0 + pos) * kLatent + bx * 64;
+        if (row >= 0) {
+          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
 #pragma unroll
           for (uint32_t c = 0; c < 8; ++c) cp_async16_tc(drow + ((c ^ x) << 4), src + c * 8);
         } else {
@@ -366,7 +367,7 @@ cudaError_t launch_sparse_attn_decode(const AttnArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   TcParams P;
   P.q_offsets = a.q_offsets;
-  P.kv_offsets = a.kv_offsets;
+  P.cache = a.cache;
   P.ctx_lens = a.ctx_lens;
   P.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
   P.idx = a.idx;

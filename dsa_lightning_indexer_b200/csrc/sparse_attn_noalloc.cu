@@ -98,7 +98,10 @@ extern "C" DSA_API dsa_status dsa_sparse_attn_noalloc(const dsa_batch* batch, co
   a.B = batch->B;
   a.Nq = batch->Nq;
   a.q_offsets = batch->q_offsets;
-  a.kv_offsets = batch->kv_offsets;
+  a.cache.kv_offsets = batch->page_size > 0 ? nullptr : batch->kv_offsets;
+  a.cache.block_table = batch->page_size > 0 ? batch->block_table : nullptr;
+  a.cache.max_blocks = batch->page_size > 0 ? batch->max_blocks : 0;
+  a.cache.page_shift = info.page_shift;
   a.ctx_lens = batch->ctx_lens;
   a.q = q;
   a.H = H;

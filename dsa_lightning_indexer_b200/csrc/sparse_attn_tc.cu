@@ -137,8 +137,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  const RowSeq rs = row_seq_warp(P.q_offsets, P.kv_offsets, P.ctx_lens, P.B, r);
-  const long long kv0 = rs.kv0;
+  const RowSeq rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
+  const long long kv0 = rs.rows.kv0;  // the masked route's contiguous rows
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
   // With idx_prefix, slots past min(top_k, p+1) hold -1: skip their tiles.
   const int n_slots = P.idx_prefix ? min(P.top_k, rs.len) : P.top_k;
@@ -204,9 +204,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
     const int gt = threadIdx.x - (5 + 2 * grp) * 32;
     int* const gidx = tidx + grp * kT;
-    // Positions of tile t's rows (thread gt < kT holds one), loaded and the
-    // rows prefetched into L2 a tile ahead of their copy.
-    auto load_pos = [&](int t) -> int {
+    // Cache rows of tile t's slots (thread gt < kT holds one), loaded and
+    // prefetched into L2 a tile ahead of their copy.
+    auto load_row = [&](int t) -> int {
       if (gt >= kT || t >= n_tiles) return -1;
       const int slot = slot_lo + t * kT + gt;
       if (slot >= slot_hi) return -1;
@@ -217,40 +217,41 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         atomicOr(P.err, kErrIndex);
         return -1;
       }
-      return pos;
+      // The slot's cache row (-1: nothing to read).
+      return pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
     };
-    auto prefetch_row = [&](int pos) {
-      if (pos >= 0) {
+    auto prefetch_row = [&](int row) {
+      if (row >= 0) {
         asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                         P.kv + static_cast<size_t>(kv0 + pos) * kLatent),
+                         P.kv + static_cast<size_t>(row) * kLatent),
                      "r"(kLatent * 2)
                      : "memory");
       }
     };
-    int pos_cur = load_pos(grp);
-    int pos_nxt = load_pos(grp + 2);
-    prefetch_row(pos_cur);
+    int row_cur = load_row(grp);
+    int row_nxt = load_row(grp + 2);
+    prefetch_row(row_cur);
     bool ok = true;
     for (int t = grp; t < n_tiles && ok; t += 2) {
-      prefetch_row(pos_nxt);
+      prefetch_row(row_nxt);
       const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
-      if (gt < kT) gidx[gt] = pos_cur;
+      if (gt < kT) gidx[gt] = row_cur;
       named_bar_sync(2 + grp, kGroupThreads);
-      pos_cur = pos_nxt;
-      pos_nxt = load_pos(t + 4);
+      row_cur = row_nxt;
+      row_nxt = load_row(t + 4);
       const uint32_t stage = sKV + grp * kKVStage;
       for (int item = gt; item < kT * kBoxes; item += kGroupThreads) {
         // Rows fastest: a warp's lanes take consecutive rows of one box, so
         // the swizzled 16-byte pieces of one instruction spread over all
         // eight bank groups of shared memory.
         const int bx = item / kT, i = item - bx * kT;
-        const int pos = gidx[i];
+        const int row = gidx[i];
         const uint32_t drow = stage + bx * kKVBox + i * 128;
         const uint32_t x = static_cast<uint32_t>(i & 7);
-        if (pos >= 0) {
-          const __nv_bfloat16* src = P.kv + static_cast<size_t>(kv0 + pos) * kLatent + bx * 64;
+        if (row >= 0) {
+          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
 #pragma unroll
           for (uint32_t c = 0; c < 8; ++c) cp_async16_tc(drow + ((c ^ x) << 4), src + c * 8);
         } else {
@@ -581,7 +582,7 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   TcParams P;
   P.q_offsets = a.q_offsets;
-  P.kv_offsets = a.kv_offsets;
+  P.cache = a.cache;
   P.ctx_lens = a.ctx_lens;
   P.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv);
   P.idx = a.idx;

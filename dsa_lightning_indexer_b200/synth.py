@@ -189,6 +189,46 @@ def custom(lens, nq, H, top_k, seed, layer=0, caps=None, name="custom") -> Workl
     return _assemble(name, seed, layer, nq, lens, H, top_k, caps=caps)
 
 
+@dataclasses.dataclass
+class PagedCaches:
+    """The caches of a workload laid out in pages: position s of sequence b
+    is row block_table[b, s // page_size] * page_size + s % page_size."""
+    page_size: int
+    block_table: np.ndarray  # int32 [B, max_blocks]
+    cache_rows: int
+    k_idx: np.ndarray        # uint16 [cache_rows, 128]
+    kv: np.ndarray           # uint16 [cache_rows, 576]
+
+
+def paged(wl: Workload, page_size: int, seed: int, spare_pages: int = 3) -> Workload:
+    """The same workload with its caches cut into pages of `page_size` rows,
+    placed in a seeded random order among `spare_pages` unused pages (filled
+    with other values); the contiguous arrays stay on the workload for the
+    oracle.  Only the data layout changes."""
+    B = wl.B
+    caps = np.diff(wl.kv_offsets).astype(np.int64)
+    n_pages = [int((c + page_size - 1) // page_size) for c in caps]
+    total = sum(n_pages) + spare_pages
+    order = rng(seed, 0, T_PROJ + 1).permutation(total)
+    bt = np.full((B, max(1, max(n_pages))), -1, dtype=np.int32)
+    k_pg = normal_bf16(seed, 1, T_KIDX, (total * page_size, DI))
+    kv_pg = normal_bf16(seed, 1, T_KV, (total * page_size, D))
+    at = 0
+    for b in range(B):
+        k0 = int(wl.kv_offsets[b])
+        for j in range(n_pages[b]):
+            page = int(order[at])
+            at += 1
+            bt[b, j] = page
+            lo, hi = j * page_size, min(int(caps[b]), (j + 1) * page_size)
+            dst = page * page_size
+            k_pg[dst:dst + hi - lo] = wl.k_idx[k0 + lo:k0 + hi]
+            kv_pg[dst:dst + hi - lo] = wl.kv[k0 + lo:k0 + hi]
+    out = dataclasses.replace(wl, name=wl.name + f"_paged{page_size}")
+    out.paged = PagedCaches(page_size, bt, total * page_size, k_pg, kv_pg)
+    return out
+
+
 def glue_projection(seed, n_in=DV, H=64) -> np.ndarray:
     """Fixed random bf16 projection [n_in, H*576] ~ N(0, 1/n_in) chaining stacked layers."""
     return normal_bf16(seed, 0, T_PROJ, (n_in, H * D), std=1.0 / math.sqrt(n_in))

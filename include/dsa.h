@@ -104,10 +104,17 @@ typedef enum {
  *   - query rows [q_offsets[b], q_offsets[b+1]) of every per-query tensor
  *     (nq_b = q_offsets[b+1] - q_offsets[b] >= 0, q_offsets[0] = 0,
  *     q_offsets[B] = Nq);
- *   - cache rows [kv_offsets[b], kv_offsets[b+1]) of k_idx and kv (the two
- *     caches share row numbering); its context is the first ctx_lens[b] of
- *     them, so 1 <= ctx_lens[b] <= kv_offsets[b+1] - kv_offsets[b] whenever
- *     nq_b > 0, and nq_b <= ctx_lens[b].
+ *   - positions 0..ctx_lens[b]-1 of the caches k_idx and kv (the two caches
+ *     share row numbering), with nq_b <= ctx_lens[b].
+ * Where position s of sequence b lives:
+ *   - contiguous caches (page_size = 0): row kv_offsets[b] + s, inside
+ *     [kv_offsets[b], kv_offsets[b+1]), so ctx_lens[b] <= kv_offsets[b+1] -
+ *     kv_offsets[b];
+ *   - paged caches (page_size > 0, a power of two >= 64): row
+ *     block_table[b * max_blocks + s / page_size] * page_size
+ *     + s % page_size; every listed page is < cache_rows / page_size and
+ *     ctx_lens[b] <= max_blocks * page_size; kv_offsets is not used (may be
+ *     NULL).
  * The current tokens are already appended to the caches: the j-th query of
  * sequence b sits at position p = ctx_lens[b] - nq_b + j and sees positions
  * 0..p, its own included (decode: nq_b = 1, p = L-1; prefill: nq_b = L).
@@ -122,6 +129,12 @@ typedef struct {
   const int32_t* h_q_offsets;   /* host mirror, [B+1] */
   const int64_t* h_kv_offsets;  /* host mirror, [B+1] */
   const int32_t* h_ctx_lens;    /* host mirror, [B] */
+  /* paged caches (all zero / NULL for contiguous caches) */
+  int32_t page_size;            /* 0, or rows per page: a power of two >= 64 */
+  int32_t max_blocks;           /* block-table entries per sequence */
+  const int32_t* block_table;   /* device, [B][max_blocks] page numbers */
+  const int32_t* h_block_table; /* host mirror */
+  int64_t cache_rows;           /* rows of k_idx and kv (paged caches) */
 } dsa_batch;
 
 /* Bytes of workspace that dsa_layer_forward needs for this batch; it is also

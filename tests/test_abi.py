@@ -51,7 +51,7 @@ class FakeBatch:
         self.hl = np.ascontiguousarray(lens, np.int32)
         d = None if null_device else FAKE
         self.c = bd._CBatch(len(lens), int(self.hq[-1]), d, d, d, self.hq.ctypes.data,
-                            self.hk.ctypes.data, self.hl.ctypes.data)
+                            self.hk.ctypes.data, self.hl.ctypes.data, 0, 0, None, None, 0)
 
     @property
     def ref(self):
