@@ -469,7 +469,8 @@ def run_ours(args):
                          ("ragged_B32", lambda: ragged_bench(bd, dev, peaks, 50, 3,
                                                              with_oracle=args.with_oracle)),
                          ("attention_routes_B4_L131072",
-                          lambda: mask_route_bench(bd, dev, peaks, 20, 3))):
+                          lambda: mask_route_bench(bd, dev, peaks, 20, 3)),
+                         ("indexer_input_step", lambda: input_step_bench(bd, dev, peaks, 20, 3))):
             other[key] = _safe(run)
             torch.cuda.empty_cache()
         line["other_workloads"] = other
@@ -903,6 +904,57 @@ def mask_route_bench(bd, dev, peaks, steps, warmup):
     res["mask_over_gather_time"] = res["mask_whole_cache"]["attention_ms"] / res["gather"][
         "attention_ms"]
     del dw, ws, out, lse, idx, o2, l2
+    return res
+
+
+D_MODEL, D_Q = 7168, 1536  # assumed widths of the hidden state and the query latent
+
+
+def input_step_bench(bd, dev, peaks, steps, warmup):
+    """The indexer's input step (q_b, k and head-weight projections, k appended
+    to the key cache) on the decode batch's 4 new tokens (weight streaming:
+    HBM-bound) and on the 16384 tokens of the prefill (tensor-bound), at the
+    assumed widths (hidden 7168, query latent 1536), L2 flushed before every
+    timed call."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+
+    def bf(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=dev) * std).to(torch.bfloat16)
+    w_q_b = bf(4096, D_Q, std=D_Q ** -0.5)
+    w_k = bf(128, D_MODEL, std=D_MODEL ** -0.5)
+    w_proj = bf(32, D_MODEL, std=D_MODEL ** -0.5)
+    weight_bytes = 2 * (4096 * D_Q + 128 * D_MODEL + 32 * D_MODEL)
+    res = {"widths": {"d_model": D_MODEL, "d_q": D_Q, "note": "assumed; the pages give none"}}
+    for name, lens, nq in (("decode_B4_L131072", [131072] * 4, [1] * 4),
+                           ("prefill_T16384", [16384], [16384])):
+        T = sum(nq)
+        kv_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        b = bd.Batch(np.concatenate([[0], np.cumsum(nq)]).astype(np.int32), kv_off,
+                     np.array(lens, np.int32), dev)
+        x, c_q = bf(T, D_MODEL), bf(T, D_Q)
+        k_cache = torch.zeros(int(kv_off[-1]), 128, dtype=torch.bfloat16, device=dev)
+        q_idx = torch.empty(T, 32, 128, dtype=torch.bfloat16, device=dev)
+        w = torch.empty(T, 32, device=dev)
+        ws = bd.indexer_project_workspace(b, D_MODEL, D_Q, dev)
+        fn = (lambda: bd.indexer_project(b, x, c_q, w_q_b, w_k, w_proj, q_idx, k_cache, w, ws))
+        gr = _graph_of(fn, dev)
+        ms = _time_flushed(gr, steps, warmup, dev)
+        bd.check_device_status(ws)
+        del gr
+        flops = 2.0 * T * (4096 * D_Q + 160 * D_MODEL)
+        nbytes = weight_bytes + 2 * T * (D_MODEL + D_Q) + T * (4096 * 2 + 128 * 2 + 32 * 4)
+        r = {"tokens": T, "ms": ms, "tokens_per_s": T / (ms * 1e-3), "bytes": nbytes,
+             "flops": flops, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+             "achieved_tflops": flops / (ms * 1e-3) / 1e12}
+        if T <= 64:
+            r["roofline"] = {"bound": "hbm", "frac": r["achieved_gbs"] / peaks["hbm_gbs"],
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        else:
+            r["roofline"] = {"bound": "tensor", "frac": r["achieved_tflops"] / peaks["bf16_tflops"],
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+        res[name] = r
+        del x, c_q, k_cache, q_idx, w, ws, b
     return res
 
 

@@ -52,7 +52,9 @@ constexpr int kQBox = kHB * 128;
 constexpr int kKVBox = kTile * 128;
 constexpr int kPBlk = kHB * 128;          // P^T block: 64 heads x 64 keys bf16
 constexpr int kMaxWords = 512;            // chunk <= 16384 positions
+constexpr int kWordsPerWarp = kMaxWords / 16;  // 32-position words per warp (16 warps)
 constexpr int kCandMax = 8192;            // candidates kept per row
+constexpr int kCandPer = kCandMax / 512;  // candidates per thread in phase B
 constexpr int kMemberMax = 512;           // sub-bin members ranked in shared memory
 constexpr int kFineBits = 11;
 constexpr int kFineShift = kHistShift - kFineBits;
@@ -245,6 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   int c_above = 0, c_in = 0;
   uint32_t bstar = 0;
   if (ok && !full) {
+    // All of this warp's scores (one 32-position word per step) in flight at
+    // once, together with the histogram loads below.
+    float sv[kWordsPerWarp];
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+      const int w = warp + i * kWarps;
+      const int s = s0 + 32 * w + lane;
+      sv[i] = (w < nw && s < s1) ? __ldcg(sc + s) : 0.f;
+    }
     // Bin of the k-th largest key: thread t holds bins 8u .. 8u+7 (u = 511 - t),
     // so the exclusive prefix in thread order counts the keys in higher bins.
     const int u = kThreads - 1 - tid;
@@ -273,35 +284,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     bstar = static_cast<uint32_t>(misc[kMBin]);
     c_above = misc[kMAbove];
     c_in = misc[kMInBin];
-    // Classify the chunk, one 32-position word per warp step.
+    // Classify: sure and candidate bits per word; candidates counted into the
+    // row's sub-histogram (reductions, nothing waits on them).
     int* const fine = P.fine + static_cast<size_t>(r) * kFineBins;
-    uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
-    int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
-    for (int w = warp; w < nw; w += kWarps) {
-      const int s = s0 + 32 * w + lane;
-      const bool in = s < s1;
-      const uint32_t key = in ? score_key(__ldcg(sc + s)) : 0u;
+    int n_cand = 0;
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+      const int w = warp + i * kWarps;
+      if (w >= nw) break;
+      const bool in = s0 + 32 * w + lane < s1;
+      const uint32_t key = score_key(sv[i]);
       const uint32_t bin = key >> kHistShift;
-      const bool gt = in && bin > bstar;
       const bool eq = in && bin == bstar;
-      const unsigned mg = __ballot_sync(0xffffffffu, gt);
+      const unsigned mg = __ballot_sync(0xffffffffu, in && bin > bstar);
       const unsigned me = __ballot_sync(0xffffffffu, eq);
       if (lane == 0) {
         tbits[w] = mg | me;
         sbits[w] = mg;
       }
-      if (me) {
-        int at = 0;
-        if (lane == 0) at = atomicAdd(ctr + kCtrCand, __popc(me));
-        at = __shfl_sync(0xffffffffu, at, 0) + __popc(me & lt);
-        if (eq) {
-          atomicAdd(fine + ((key >> kFineShift) & (kFineBins - 1)), 1);
-          if (at < kCandMax) {
-            ck[at] = key;
-            cp[at] = s;
-          }
+      if (eq) atomicAdd(fine + ((key >> kFineShift) & (kFineBins - 1)), 1);
+      n_cand += __popc(me);
+    }
+    // One reservation in the row's candidate list for the whole CTA.
+    int* const wcnt = reinterpret_cast<int*>(alpha_s);  // [kWarps] counts, then bases
+    if (lane == 0) wcnt[warp] = n_cand;
+    __syncthreads();
+    if (tid == 0) {
+      int sum = 0;
+      for (int w = 0; w < kWarps; ++w) sum += wcnt[w];
+      int at = sum > 0 ? atomicAdd(ctr + kCtrCand, sum) : 0;
+      for (int w = 0; w < kWarps; ++w) {
+        const int cnt = wcnt[w];
+        wcnt[w] = at;
+        at += cnt;
+      }
+    }
+    __syncthreads();
+    uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
+    int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
+    int at = wcnt[warp];
+#pragma unroll
+    for (int i = 0; i < kWordsPerWarp; ++i) {
+      const int w = warp + i * kWarps;
+      if (w >= nw) break;
+      const int s = s0 + 32 * w + lane;
+      const uint32_t key = score_key(sv[i]);
+      const bool eq = s < s1 && (key >> kHistShift) == bstar;
+      const unsigned me = __ballot_sync(0xffffffffu, eq);
+      if (eq) {
+        const int slot = at + __popc(me & lt);
+        if (slot < kCandMax) {
+          ck[slot] = key;
+          cp[slot] = s;
         }
       }
+      at += __popc(me);
     }
   } else if (ok) {
     for (int w = tid; w < nw; w += kThreads) {
@@ -330,20 +367,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   int n_tile = misc[kMNTile];
 
-  // Positions of the rows of tile t of the tile set (ascending), -1 past the end.
+  // Position of the g-th row of the tile set (ascending positions).
+  auto pos_of = [&](int g) {
+    int lo = 0, hi = nw - 1;  // last word with pre[w] <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    return s0 + 32 * lo + __fns(tbits[lo], 0, g - pre[lo] + 1);
+  };
+  // Positions and cache rows of tile t of the tile set, -1 past the end.
   auto map_tile = [&](int t) {
     if (tid < kTile) {
       const int g = t * kTile + tid;
-      int pos = -1;
-      if (g < n_tile) {
-        int lo = 0, hi = nw - 1;  // last word with pre[w] <= g
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (pre[mid] <= g) lo = mid; else hi = mid - 1;
-        }
-        const int bit = __fns(tbits[lo], 0, g - pre[lo] + 1);
-        pos = s0 + 32 * lo + bit;
-      }
+      const int pos = g < n_tile ? pos_of(g) : -1;
       tpos[tid] = pos;
       trow[tid] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
     }
@@ -393,18 +430,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
-  // Speculative tile 0: sure positions and own candidates.
-  if (ok) map_tile(0);
-  __syncthreads();
-  if (ok) gather_tile();
-  __syncthreads();  // phase A's global writes (candidates, counts) are all issued
+  // Arrive on the row counter as soon as this CTA's phase-A writes (the
+  // candidates, the sub-histogram counts, the chunk's count) are issued; the
+  // wait comes after this CTA's own gather and S product.
   bool row_ok = true;
   if (ok && !full && tid == 0) {
-    // Arrive now; the wait comes after this CTA's own gather and S product.
     __threadfence();
     atomicAdd(ctr + kCtrBarA, 1);
   }
-  if (ok) gather_done();
+  // Speculative tile 0: sure positions and own candidates.
+  if (ok) map_tile(0);
+  __syncthreads();
+  if (ok) {
+    gather_tile();
+    // Rows of further tiles (a chunk with more than one tile's worth) go to L2 now.
+    for (int g = kTile + tid; g < n_tile; g += kThreads) {
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                       P.kv + static_cast<size_t>(seq_row(rs.rows, pos_of(g))) * kLatent),
+                   "r"(kLatent * 2)
+                   : "memory");
+    }
+    gather_done();
+  }
   int s_round = 0;  // S products issued so far
   if (ok && warp == 4) {
     if (!issue_s(0)) row_ok = false;
@@ -434,6 +481,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool respec = false;  // the speculative tile is discarded (fallback selection)
   if (ok && !full) {
     const int need = k - c_above;  // keys to keep from the threshold bin, 1 .. c_in
+    const bool listed = c_in <= kCandMax;  // every candidate of the row is in the list
+    // Everything phase B reads, in flight at once: the sub-histogram, the
+    // row's candidates (kCandPer per thread) and the earlier chunks' counts.
+    const uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
+    const int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
+    uint32_t ckr[kCandPer];
+    int cpr[kCandPer];
+#pragma unroll
+    for (int i = 0; i < kCandPer; ++i) {
+      const int j = tid + i * kThreads;
+      const bool in = listed && j < c_in;
+      ckr[i] = in ? __ldcg(ck + j) : 0u;
+      cpr[i] = in ? __ldcg(cp + j) : -1;
+    }
+    const int nsure_before =
+        tid < c ? __ldcg(P.chunk_nsure + static_cast<size_t>(r) * P.C + tid) : 0;
     // Sub-bin of the need-th key of the bin: thread t holds sub-bins 4u .. 4u+3.
     {
       const int u = kThreads - 1 - tid;
@@ -461,19 +524,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const uint32_t b2 = static_cast<uint32_t>(misc[kMB2]);
     const int need2 = need - misc[kMAbove2];  // members of the sub-bin to keep
-    const bool fallback = c_in > kCandMax || misc[kMC2] > kMemberMax;  // the same row-wide
-    const uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
-    const int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
+    const bool fallback = !listed || misc[kMC2] > kMemberMax;  // the same row-wide
     if (!fallback) {
       uint32_t* const mk = reinterpret_cast<uint32_t*>(bp + kOffP);
       int* const mp = reinterpret_cast<int*>(mk + kMemberMax);
-      for (int j = tid; j < c_in; j += kThreads) {
-        const uint32_t key = __ldcg(ck + j);
-        if (((key >> kFineShift) & (kFineBins - 1)) == b2) {
+#pragma unroll
+      for (int i = 0; i < kCandPer; ++i) {
+        if (cpr[i] >= 0 && ((ckr[i] >> kFineShift) & (kFineBins - 1)) == b2) {
           const int at = atomicAdd(&misc[kMNm], 1);
           if (at < kMemberMax) {
-            mk[at] = key;
-            mp[at] = __ldcg(cp + j);
+            mk[at] = ckr[i];
+            mp[at] = cpr[i];
           }
         }
       }
@@ -495,12 +556,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int th_pos = misc[kMThPos];
       // Selected candidates: this chunk's into the selected bits, earlier
       // chunks' counted for the output offset.
-      int before = 0;
-      for (int j = tid; j < c_in; j += kThreads) {
-        const uint32_t key = __ldcg(ck + j);
-        const int pos = __ldcg(cp + j);
+      int before = nsure_before;
+#pragma unroll
+      for (int i = 0; i < kCandPer; ++i) {
+        const uint32_t key = ckr[i];
+        const int pos = cpr[i];
         const uint32_t sub = (key >> kFineShift) & (kFineBins - 1);
-        const bool selc = sub > b2 || (sub == b2 && (key > th_key || (key == th_key && pos <= th_pos)));
+        const bool selc = pos >= 0 && (sub > b2 || (sub == b2 && (key > th_key ||
+                                                                  (key == th_key && pos <= th_pos))));
         if (selc) {
           if (pos < s0) {
             ++before;
@@ -508,10 +571,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicOr(&sbits[(pos - s0) >> 5], 1u << ((pos - s0) & 31));
           }
         }
-      }
-      // Sure positions of earlier chunks.
-      for (int j = tid; j < c; j += kThreads) {
-        before += __ldcg(P.chunk_nsure + static_cast<size_t>(r) * P.C + j);
       }
       int offset;
       block_excl_sum_nw<kWarps>(before, buf, offset);
@@ -719,30 +778,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------------------------------- partial results of the chunk ----
+  // Every warp stores a quarter of its TMEM lane quadrant's share: warps w,
+  // w+4, w+8, w+12 read quadrant w % 4, two (block, half) pieces each.
   const size_t rec = (static_cast<size_t>(r) * P.C + c) * kHB;
-  if (ok && warp < 4) {
+  if (ok) {
     bool good = true;
     if (n_tiles > 0) good = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     if (good) {
       tc_fence_after();
       if (n_tiles > 0) {
+        const uint32_t qbase = static_cast<uint32_t>((warp & 3) * 32) << 16;
 #pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            uint32_t o[32];
-            tmem_ld_32x32b_x32(tmem + lane_base + kColO + 64u * blk + 32u * half, o);
-            tmem_ld_wait();
-            const int dv = 128 * blk + 32 * q4 + lane;
+        for (int piece = 2 * (warp >> 2); piece < 2 * (warp >> 2) + 2; ++piece) {
+          const int blk = piece >> 1, half = piece & 1;
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(tmem + qbase + kColO + 64u * blk + 32u * half, o);
+          tmem_ld_wait();
+          const int dv = 128 * blk + 32 * (warp & 3) + lane;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int h = 32 * half + j;
-              if (h < P.H) __stcg(P.part_o + (rec + h) * kValue + dv, __uint_as_float(o[j]));
-            }
+          for (int j = 0; j < 32; ++j) {
+            const int h = 32 * half + j;
+            if (h < P.H) __stcg(P.part_o + (rec + h) * kValue + dv, __uint_as_float(o[j]));
           }
         }
       }
-      if (owner && hl < P.H) P.part_ml[rec + hl] = make_float2(m_run, l_run);
+      if (warp < 4 && owner && hl < P.H) P.part_ml[rec + hl] = make_float2(m_run, l_run);
     } else {
       row_ok = false;
     }
@@ -784,30 +844,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
-      for (int u = u0 + tid; u < u1; u += kThreads) {
-        const int h = u / (kValue / 4), d4 = u - h * (kValue / 4);
-        const float* const wr = wgt + (h - hlo) * P.C;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float* const po = P.part_o + (static_cast<size_t>(r) * P.C * kHB + h) * kValue + 4 * d4;
-        constexpr int kU = 8;
-        for (int j0 = 0; j0 < P.C; j0 += kU) {
-          float4 x[kU];
+      // G threads per output unit (a float4 of one head), each summing every
+      // G-th chunk's partial with all of its loads in flight, then combined
+      // with shuffles; chunks in a fixed order, so the result is deterministic.
+      const int nu = u1 - u0;
+      int G = 1;
+      while (G < 32 && 2 * G * nu <= kThreads) G *= 2;
+      const int ui = tid / G, sub = tid - ui * G;
+      const int u = u0 + ui;
+      const bool act = ui < nu;
+      const int h = act ? u / (kValue / 4) : hlo;
+      const int d4 = act ? u - h * (kValue / 4) : 0;
+      const float* const wr = wgt + (h - hlo) * P.C;
+      const float* const po = P.part_o + (static_cast<size_t>(r) * P.C * kHB + h) * kValue + 4 * d4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      constexpr int kU = 10;
+      for (int j0 = sub; j0 < P.C; j0 += kU * G) {
+        float4 x[kU];
 #pragma unroll
-          for (int j = 0; j < kU; ++j) {
-            x[j] = (j0 + j < P.C && wr[j0 + j] != 0.f)
-                       ? __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(j0 + j) *
-                                                                         kHB * kValue))
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-#pragma unroll
-          for (int j = 0; j < kU; ++j) {
-            const float wj = j0 + j < P.C ? wr[j0 + j] : 0.f;
-            acc.x = fmaf(wj, x[j].x, acc.x);
-            acc.y = fmaf(wj, x[j].y, acc.y);
-            acc.z = fmaf(wj, x[j].z, acc.z);
-            acc.w = fmaf(wj, x[j].w, acc.w);
-          }
+        for (int jj = 0; jj < kU; ++jj) {
+          const int j = j0 + jj * G;
+          x[jj] = (act && j < P.C && wr[j] != 0.f)
+                      ? __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(j) * kHB *
+                                                                        kValue))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+#pragma unroll
+        for (int jj = 0; jj < kU; ++jj) {
+          const int j = j0 + jj * G;
+          const float wj = (act && j < P.C) ? wr[j] : 0.f;
+          acc.x = fmaf(wj, x[jj].x, acc.x);
+          acc.y = fmaf(wj, x[jj].y, acc.y);
+          acc.z = fmaf(wj, x[jj].z, acc.z);
+          acc.w = fmaf(wj, x[jj].w, acc.w);
+        }
+      }
+      for (int o2 = 1; o2 < G; o2 <<= 1) {  // the G threads of a unit are adjacent lanes
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o2);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o2);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o2);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o2);
+      }
+      if (act && sub == 0) {
         *reinterpret_cast<float4*>(P.out + (static_cast<size_t>(r) * P.H + h) * kValue + 4 * d4) =
             acc;
       }

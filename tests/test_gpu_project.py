@@ -1,10 +1,13 @@
 """The indexer's input step (dsa_indexer_project) against the oracle (needs a B200).
 
-q_idx and the new tokens' indexer keys are bf16 roundings of fp32 sums: they
-must equal the oracle's (which rounds its double sums the same way) except
-where the two sums straddle a rounding boundary, i.e. within one bf16 unit in
-the last place; w (fp32) within 2e-5 of (|ref| + rms of the row).  Rows of
-the key cache other than the new tokens' must be left untouched.
+q_idx and the new tokens' indexer keys are bf16 roundings of fp32 sums.  The
+oracle rounds its double sums the same way, so the two agree except where
+the fp32 sum's own error (a small multiple of 2^-24 times the sum of the
+products' magnitudes, i.e. absolute, not relative to the result) moves a
+result across a rounding boundary: one bf16 unit of the result, plus 1e-5
+of the row's rms for results that cancel to near zero; more than 99% must
+agree bit for bit.  w (fp32) within 2e-5 of (|ref| + rms of the row).  Rows
+of the key cache other than the new tokens' must be left untouched.
 """
 import numpy as np
 import pytest
@@ -73,8 +76,13 @@ def test_indexer_project_matches_oracle(name):
     got_w = w.cpu().numpy()
     dq = _ulp_diff(got_q, want_q)
     dk = _ulp_diff(got_k, want_k)
-    assert dq.max() <= 1 and dk.max() <= 1, (int(dq.max()), int(dk.max()))
     assert (dq == 0).mean() > 0.99 and (dk == 0).mean() > 0.99
+    for got, want in ((got_q.reshape(T, -1), want_q.reshape(T, -1)), (got_k, want_k)):
+        g32, w32 = synth.bf16_to_f32(got).astype(np.float64), synth.bf16_to_f32(want).astype(
+            np.float64)
+        rms = np.sqrt((w32 ** 2).mean(axis=1, keepdims=True))
+        bound = 2.0 ** -7 * np.abs(w32) + 1e-5 * rms
+        assert (np.abs(g32 - w32) <= bound).all(), float((np.abs(g32 - w32) / bound).max())
     new_rows = set()
     for bi in range(len(c["cl"])):
         nq = int(c["qo"][bi + 1] - c["qo"][bi])
