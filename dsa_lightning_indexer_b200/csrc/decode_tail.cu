@@ -10,24 +10,24 @@
 // key-only latent cache whose leading 512 entries serve as V.)
 //
 // One cooperative launch of Nq x C CTAs (one per SM); CTA (r, c) owns chunk
-// c of row r's causal positions [s0, s1).  Phases:
+// c of row r's causal positions [s0, s1) for the selection and an equal
+// share of the row's selected slots for the attention.  Phases:
 //   A  From the row's 4096-bin histogram of the top 12 key bits (built by the
 //      indexer) find the bin holding the k-th largest key.  Read the chunk's
 //      scores once: positions above that bin are selected for sure, positions
 //      in it are candidates (appended to the row's candidate list and counted
-//      into the row's 2048-bin sub-histogram of the next 11 key bits).  Start
-//      gathering the rows of sure positions and own candidates (one tile of
-//      up to 96 rows) and compute S = Q K^T on them, then arrive on the row's
+//      into the row's 2048-bin sub-histogram of the next 11 key bits).  The
+//      latent rows of both start coming into L2; then arrive on the row's
 //      counter.
 //   B  When every CTA of the row has arrived, find the sub-bin of the k-th
 //      key and rank its few members exactly; write this chunk's selected
 //      positions, in order, into the row's index set.  Heavily tied rows
 //      (candidate list or sub-bin too full) fall back to an exact whole-row
-//      select by the row's first CTA, which the others wait for.
-//   C  Softmax over the tile with unselected candidates masked, P as bf16
-//      hi + lo, O^T = V^T P^T into TMEM (further tiles, if any, with a
-//      running maximum); the unnormalised O and (max, sum) of every head go
-//      to the row's partial results.
+//      select by the row's first CTA.  Arrive on the row's second counter.
+//   C  When the index set is complete, take slots [c*ceil(k/C), ...) of it:
+//      gather those rows in tiles of 96, S = Q K^T, softmax, P as bf16 hi +
+//      lo, O^T = V^T P^T into TMEM with a running maximum; the unnormalised
+//      O and (max, sum) of every head go to the row's partial results.
 //   D  When every CTA of the row has stored its partials, each merges a
 //      1/C share of the row's output with the log-sum-exp rule.
 // Every wait is bounded; a wait that runs out sets the workspace error word
@@ -52,9 +52,9 @@ constexpr int kQBox = kHB * 128;
 constexpr int kKVBox = kTile * 128;
 constexpr int kPBlk = kHB * 128;          // P^T block: 64 heads x 64 keys bf16
 constexpr int kMaxWords = 512;            // chunk <= 16384 positions
-constexpr int kWordsPerWarp = kMaxWords / 16;  // 32-position words per warp (16 warps)
+constexpr int kWordsPerWarp = 8;          // 32-position words per warp per pass (16 warps)
 constexpr int kCandMax = 8192;            // candidates kept per row
-constexpr int kCandPer = kCandMax / 512;  // candidates per thread in phase B
+constexpr int kCandPer = 4;               // candidates per thread per batch in phase B
 constexpr int kMemberMax = 512;           // sub-bin members ranked in shared memory
 constexpr int kFineBits = 11;
 constexpr int kFineShift = kHistShift - kFineBits;
@@ -64,18 +64,15 @@ constexpr int kSoftThreads = 128;
 constexpr float kRescaleLog2 = 0.0f;      // raise the running max whenever it grows
 
 // Per-row counters (int): candidates appended, arrivals after phase A,
-// arrivals after the partials, fallback selection ready.
-constexpr int kCtrCand = 0, kCtrBarA = 1, kCtrBarD = 2, kCtrFallback = 3, kCtrInts = 8;
+// arrivals after the partials, arrivals after the index set is written.
+constexpr int kCtrCand = 0, kCtrBarA = 1, kCtrBarD = 2, kCtrBarC = 3, kCtrInts = 8;
 
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kBoxes * kQBox;           // 73728
 constexpr int kOffP = kOffKV + kBoxes * kKVBox;          // 184320: [hi b0, hi b1, lo b0, lo b1]
-constexpr int kOffTile = kOffP + 4 * kPBlk;              // 217088: tile-set bits
-constexpr int kOffSel = kOffTile + kMaxWords * 4;        // selected bits
-constexpr int kOffPre = kOffSel + kMaxWords * 4;         // tile-set prefix per word
-constexpr int kOffTpos = kOffPre + kMaxWords * 4;        // [kTile] positions of the tile rows
-constexpr int kOffTsel = kOffTpos + kTile * 4;           // [kTile] selected flags
-constexpr int kOffTrow = kOffTsel + kTile * 4;           // [kTile] cache rows of the tile
+constexpr int kOffSel = kOffP + 4 * kPBlk;               // 217088: selected bits
+constexpr int kOffTpos = kOffSel + kMaxWords * 4;        // [kTile] positions of the tile rows
+constexpr int kOffTrow = kOffTpos + kTile * 4;           // [kTile] cache rows of the tile
 constexpr int kOffAlpha = kOffTrow + kTile * 4;          // [64]
 constexpr int kOffScan = kOffAlpha + kHB * 4;            // block scan buffer
 constexpr int kOffMisc = kOffScan + 128;                 // shared scalars
@@ -98,8 +95,7 @@ constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-ma
 
 // Shared scalars.
 enum {
-  kMAbort, kMBin, kMAbove, kMInBin, kMB2, kMAbove2, kMC2, kMNm, kMFallback, kMNTile,
-  kMNSure, kMOffset, kMThKey, kMThPos, kMBefore, kMScratch
+  kMAbort, kMBin, kMAbove, kMInBin, kMB2, kMAbove2, kMC2, kMNm, kMThKey, kMThPos
 };
 
 struct TailParams {
@@ -152,23 +148,6 @@ __device__ bool row_arrive_wait(int* ctr, int target, unsigned* err) {
   return true;
 }
 
-// Thread 0 only: wait (bounded) until *flag is nonzero.
-__device__ bool wait_flag(const int* flag, unsigned* err) {
-  const long long t0 = clock64();
-  for (unsigned it = 1;; ++it) {
-    if (ld_acquire(flag) != 0) break;
-    if ((it & 15u) == 0u) {
-      if (*reinterpret_cast<volatile unsigned*>(err) != 0u) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        atomicOr(err, kErrTimeout);
-        return false;
-      }
-    }
-  }
-  __threadfence();
-  return true;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     decode_tail_kernel(const __grid_constant__ CUtensorMap qmap, const TailParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -176,11 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* const bp = smem_raw + (base - raw);
   const uint32_t sQ = base + kOffQ, sKV = base + kOffKV, sP = base + kOffP;
-  uint32_t* const tbits = reinterpret_cast<uint32_t*>(bp + kOffTile);
   uint32_t* const sbits = reinterpret_cast<uint32_t*>(bp + kOffSel);
-  int* const pre = reinterpret_cast<int*>(bp + kOffPre);
   int* const tpos = reinterpret_cast<int*>(bp + kOffTpos);
-  int* const tsel = reinterpret_cast<int*>(bp + kOffTsel);
   int* const trow = reinterpret_cast<int*>(bp + kOffTrow);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
   int* const buf = reinterpret_cast<int*>(bp + kOffScan);
@@ -247,15 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   int c_above = 0, c_in = 0;
   uint32_t bstar = 0;
   if (ok && !full) {
-    // All of this warp's scores (one 32-position word per step) in flight at
-    // once, together with the histogram loads below.
+    // The first pass's scores (one 32-position word per warp step, kWordsPerWarp
+    // per warp) in flight at once, together with the histogram loads below.
     float sv[kWordsPerWarp];
+    auto load_pass = [&](int wbase) {
 #pragma unroll
-    for (int i = 0; i < kWordsPerWarp; ++i) {
-      const int w = warp + i * kWarps;
-      const int s = s0 + 32 * w + lane;
-      sv[i] = (w < nw && s < s1) ? __ldcg(sc + s) : 0.f;
-    }
+      for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int w = wbase + warp + i * kWarps;
+        const int s = s0 + 32 * w + lane;
+        sv[i] = (w < nw && s < s1) ? __ldcg(sc + s) : 0.f;
+      }
+    };
+    load_pass(0);
     // Bin of the k-th largest key: thread t holds bins 8u .. 8u+7 (u = 511 - t),
     // so the exclusive prefix in thread order counts the keys in higher bins.
     const int u = kThreads - 1 - tid;
@@ -284,217 +263,123 @@ __global__ void __launch_bounds__(kThreads, 1)
     bstar = static_cast<uint32_t>(misc[kMBin]);
     c_above = misc[kMAbove];
     c_in = misc[kMInBin];
-    // Classify: sure and candidate bits per word; candidates counted into the
-    // row's sub-histogram (reductions, nothing waits on them).
     int* const fine = P.fine + static_cast<size_t>(r) * kFineBins;
-    int n_cand = 0;
-#pragma unroll
-    for (int i = 0; i < kWordsPerWarp; ++i) {
-      const int w = warp + i * kWarps;
-      if (w >= nw) break;
-      const bool in = s0 + 32 * w + lane < s1;
-      const uint32_t key = score_key(sv[i]);
-      const uint32_t bin = key >> kHistShift;
-      const bool eq = in && bin == bstar;
-      const unsigned mg = __ballot_sync(0xffffffffu, in && bin > bstar);
-      const unsigned me = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) {
-        tbits[w] = mg | me;
-        sbits[w] = mg;
-      }
-      if (eq) atomicAdd(fine + ((key >> kFineShift) & (kFineBins - 1)), 1);
-      n_cand += __popc(me);
-    }
-    // One reservation in the row's candidate list for the whole CTA.
-    int* const wcnt = reinterpret_cast<int*>(alpha_s);  // [kWarps] counts, then bases
-    if (lane == 0) wcnt[warp] = n_cand;
-    __syncthreads();
-    if (tid == 0) {
-      int sum = 0;
-      for (int w = 0; w < kWarps; ++w) sum += wcnt[w];
-      int at = sum > 0 ? atomicAdd(ctr + kCtrCand, sum) : 0;
-      for (int w = 0; w < kWarps; ++w) {
-        const int cnt = wcnt[w];
-        wcnt[w] = at;
-        at += cnt;
-      }
-    }
-    __syncthreads();
     uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
     int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
-    int at = wcnt[warp];
+    int* const wcnt = reinterpret_cast<int*>(alpha_s);  // [kWarps] counts, then bases
+#pragma unroll 1
+    for (int wbase = 0; wbase < nw; wbase += kWordsPerWarp * kWarps) {
+      if (wbase > 0) load_pass(wbase);
+      // Classify: sure and candidate bits per word; the rows of both start
+      // coming into L2 now; candidates are counted into the row's
+      // sub-histogram (reductions, nothing waits on them).
+      int n_cand = 0;
 #pragma unroll
-    for (int i = 0; i < kWordsPerWarp; ++i) {
-      const int w = warp + i * kWarps;
-      if (w >= nw) break;
-      const int s = s0 + 32 * w + lane;
-      const uint32_t key = score_key(sv[i]);
-      const bool eq = s < s1 && (key >> kHistShift) == bstar;
-      const unsigned me = __ballot_sync(0xffffffffu, eq);
-      if (eq) {
-        const int slot = at + __popc(me & lt);
-        if (slot < kCandMax) {
-          ck[slot] = key;
-          cp[slot] = s;
+      for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int w = wbase + warp + i * kWarps;
+        if (w >= nw) break;
+        const int s = s0 + 32 * w + lane;
+        const bool in = s < s1;
+        const uint32_t key = score_key(sv[i]);
+        const uint32_t bin = key >> kHistShift;
+        const bool gt = in && bin > bstar;
+        const bool eq = in && bin == bstar;
+        const unsigned mg = __ballot_sync(0xffffffffu, gt);
+        const unsigned me = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) sbits[w] = mg;
+        if (gt || eq) {
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                           P.kv + static_cast<size_t>(seq_row(rs.rows, s)) * kLatent),
+                       "r"(kLatent * 2)
+                       : "memory");
+        }
+        if (eq) atomicAdd(fine + ((key >> kFineShift) & (kFineBins - 1)), 1);
+        n_cand += __popc(me);
+      }
+      // One reservation in the row's candidate list per pass for the whole CTA.
+      if (lane == 0) wcnt[warp] = n_cand;
+      __syncthreads();
+      if (tid == 0) {
+        int sum = 0;
+        for (int w = 0; w < kWarps; ++w) sum += wcnt[w];
+        int at = sum > 0 ? atomicAdd(ctr + kCtrCand, sum) : 0;
+        for (int w = 0; w < kWarps; ++w) {
+          const int cnt = wcnt[w];
+          wcnt[w] = at;
+          at += cnt;
         }
       }
-      at += __popc(me);
+      __syncthreads();
+      int at = wcnt[warp];
+#pragma unroll
+      for (int i = 0; i < kWordsPerWarp; ++i) {
+        const int w = wbase + warp + i * kWarps;
+        if (w >= nw) break;
+        const int s = s0 + 32 * w + lane;
+        const uint32_t key = score_key(sv[i]);
+        const bool eq = s < s1 && (key >> kHistShift) == bstar;
+        const unsigned me = __ballot_sync(0xffffffffu, eq);
+        if (eq) {
+          const int slot = at + __popc(me & lt);
+          if (slot < kCandMax) {
+            ck[slot] = key;
+            cp[slot] = s;
+          }
+        }
+        at += __popc(me);
+      }
+      __syncthreads();  // the counts area is reused by the next pass
     }
   } else if (ok) {
     for (int w = tid; w < nw; w += kThreads) {
       const int rem = s1 - (s0 + 32 * w);
       const uint32_t m = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-      tbits[w] = m;
       sbits[w] = m;
     }
   }
   __syncthreads();
-  // Tile-set prefix per word and the number of sure positions.
+  // The number of sure positions of the chunk, for the output offsets.
   {
-    const uint32_t tw = (ok && tid < nw) ? tbits[tid] : 0u;
-    const uint32_t sw = (ok && tid < nw) ? sbits[tid] : 0u;
-    int n_tile;
-    const int ex = block_excl_sum_nw<kWarps>(__popc(tw), buf, n_tile);
-    if (tid < kMaxWords) pre[tid] = ex;
+    const uint32_t sw = (ok && !full && tid < nw) ? sbits[tid] : 0u;
     int n_sure;
     block_excl_sum_nw<kWarps>(__popc(sw), buf, n_sure);
-    if (tid == 0) {
-      misc[kMNTile] = n_tile;
-      misc[kMNSure] = n_sure;
-      if (ok && !full) P.chunk_nsure[static_cast<size_t>(r) * P.C + c] = n_sure;
-    }
+    if (tid == 0 && ok && !full) P.chunk_nsure[static_cast<size_t>(r) * P.C + c] = n_sure;
   }
   __syncthreads();
-  int n_tile = misc[kMNTile];
-
-  // Position of the g-th row of the tile set (ascending positions).
-  auto pos_of = [&](int g) {
-    int lo = 0, hi = nw - 1;  // last word with pre[w] <= g
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (pre[mid] <= g) lo = mid; else hi = mid - 1;
-    }
-    return s0 + 32 * lo + __fns(tbits[lo], 0, g - pre[lo] + 1);
-  };
-  // Positions and cache rows of tile t of the tile set, -1 past the end.
-  auto map_tile = [&](int t) {
-    if (tid < kTile) {
-      const int g = t * kTile + tid;
-      const int pos = g < n_tile ? pos_of(g) : -1;
-      tpos[tid] = pos;
-      trow[tid] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
-    }
-  };
-  // Every thread copies its share of the tile's rows (16-byte cp.async,
-  // 128-byte swizzle), then arrives on kv_full once its copies have landed.
-  auto gather_tile = [&]() {
-    for (int item = tid; item < kTile * kBoxes; item += kThreads) {
-      const int bx = item / kTile, i = item - bx * kTile;
-      const int row = trow[i];
-      const uint32_t drow = sKV + bx * kKVBox + i * 128;
-      const uint32_t x = static_cast<uint32_t>(i & 7);
-      if (row >= 0) {
-        const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
-#pragma unroll
-        for (uint32_t cc = 0; cc < 8; ++cc) cp_async16_tc(drow + ((cc ^ x) << 4), src + cc * 8);
-      } else {
-#pragma unroll
-        for (uint32_t cc = 0; cc < 8; ++cc) {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(drow + (cc << 4)), "r"(0u)
-                       : "memory");
-        }
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  auto gather_done = [&]() {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    fence_proxy_async_smem();
-    mbar_arrive(b_kvfull);
-  };
-  // Warp 4: S = Q K_tile^T for the gathered tile (round `it`).
-  auto issue_s = [&](int it) -> bool {
-    bool good = __all_sync(0xffffffffu, mbar_wait(b_qfull, 0, P.err));
-    good = good && __all_sync(0xffffffffu, mbar_wait(b_kvfull, static_cast<uint32_t>(it & 1), P.err));
-    if (!good) return false;
-    tc_fence_after();
-    const uint64_t dq = sdesc_sw128(sQ), dk = sdesc_sw128(sKV);
-#pragma unroll
-    for (int ks = 0; ks < kLatent / 16; ++ks) {
-      const uint32_t off = (ks & 3) * 32;
-      tc_mma_bf16_warp(tmem + kColS, dq + static_cast<uint64_t>(((ks >> 2) * kQBox + off) >> 4),
-                       dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4), kIdescS,
-                       ks > 0 ? 1u : 0u);
-    }
-    tc_commit_warp(b_sfull);
-    return true;
-  };
 
   // Arrive on the row counter as soon as this CTA's phase-A writes (the
-  // candidates, the sub-histogram counts, the chunk's count) are issued; the
-  // wait comes after this CTA's own gather and S product.
+  // candidates, the sub-histogram counts, the chunk's count) are issued, and
+  // wait for the row's other CTAs.
   bool row_ok = true;
   if (ok && !full && tid == 0) {
-    __threadfence();
-    atomicAdd(ctr + kCtrBarA, 1);
+    if (!row_arrive_wait(ctr + kCtrBarA, P.C, P.err)) row_ok = false;
   }
-  // Speculative tile 0: sure positions and own candidates.
-  if (ok) map_tile(0);
-  __syncthreads();
-  if (ok) {
-    gather_tile();
-    // Rows of further tiles (a chunk with more than one tile's worth) go to L2 now.
-    for (int g = kTile + tid; g < n_tile; g += kThreads) {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                       P.kv + static_cast<size_t>(seq_row(rs.rows, pos_of(g))) * kLatent),
-                   "r"(kLatent * 2)
-                   : "memory");
-    }
-    gather_done();
-  }
-  int s_round = 0;  // S products issued so far
-  if (ok && warp == 4) {
-    if (!issue_s(0)) row_ok = false;
-  }
-  s_round = 1;
-  if (ok && !full && tid == 0) {
-    const long long t0 = clock64();
-    for (unsigned it = 1;; ++it) {
-      if (ld_acquire(ctr + kCtrBarA) >= P.C) break;
-      if ((it & 15u) == 0u) {
-        if (*reinterpret_cast<volatile unsigned*>(P.err) != 0u) {
-          row_ok = false;
-          break;
-        }
-        if (clock64() - t0 > kWaitCycles) {
-          atomicOr(P.err, kErrTimeout);
-          row_ok = false;
-          break;
-        }
-      }
-    }
-    __threadfence();
-  }
+  __syncwarp();  // warp 0 meets the CTA barrier reconverged
   ok = ok && !__syncthreads_or(!row_ok);
 
   // ---------------------------------------------------------- phase B ----
-  bool respec = false;  // the speculative tile is discarded (fallback selection)
   if (ok && !full) {
     const int need = k - c_above;  // keys to keep from the threshold bin, 1 .. c_in
     const bool listed = c_in <= kCandMax;  // every candidate of the row is in the list
     // Everything phase B reads, in flight at once: the sub-histogram, the
-    // row's candidates (kCandPer per thread) and the earlier chunks' counts.
+    // row's candidates (batches of kCandPer per thread; usually one batch,
+    // which then stays in registers for both passes) and the earlier chunks'
+    // counts.
     const uint32_t* const ck = P.cand_key + static_cast<size_t>(r) * kCandMax;
     const int* const cp = P.cand_pos + static_cast<size_t>(r) * kCandMax;
+    const int n_batches = listed ? (c_in + kCandPer * kThreads - 1) / (kCandPer * kThreads) : 0;
     uint32_t ckr[kCandPer];
     int cpr[kCandPer];
+    auto load_batch = [&](int bt) {
 #pragma unroll
-    for (int i = 0; i < kCandPer; ++i) {
-      const int j = tid + i * kThreads;
-      const bool in = listed && j < c_in;
-      ckr[i] = in ? __ldcg(ck + j) : 0u;
-      cpr[i] = in ? __ldcg(cp + j) : -1;
-    }
+      for (int i = 0; i < kCandPer; ++i) {
+        const int j = (bt * kCandPer + i) * kThreads + tid;
+        const bool in = listed && j < c_in;
+        ckr[i] = in ? __ldcg(ck + j) : 0u;
+        cpr[i] = in ? __ldcg(cp + j) : -1;
+      }
+    };
+    load_batch(0);
     const int nsure_before =
         tid < c ? __ldcg(P.chunk_nsure + static_cast<size_t>(r) * P.C + tid) : 0;
     // Sub-bin of the need-th key of the bin: thread t holds sub-bins 4u .. 4u+3.
@@ -516,10 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           misc[kMB2] = 4 * u; misc[kMAbove2] = above + f.w + f.z + f.y; misc[kMC2] = f.x;
         }
       }
-      if (tid == 0) {
-        misc[kMNm] = 0;
-        misc[kMBefore] = 0;
-      }
+      if (tid == 0) misc[kMNm] = 0;
       __syncthreads();
     }
     const uint32_t b2 = static_cast<uint32_t>(misc[kMB2]);
@@ -528,13 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!fallback) {
       uint32_t* const mk = reinterpret_cast<uint32_t*>(bp + kOffP);
       int* const mp = reinterpret_cast<int*>(mk + kMemberMax);
+#pragma unroll 1
+      for (int bt = 0; bt < n_batches; ++bt) {
+        if (bt > 0) load_batch(bt);
 #pragma unroll
-      for (int i = 0; i < kCandPer; ++i) {
-        if (cpr[i] >= 0 && ((ckr[i] >> kFineShift) & (kFineBins - 1)) == b2) {
-          const int at = atomicAdd(&misc[kMNm], 1);
-          if (at < kMemberMax) {
-            mk[at] = ckr[i];
-            mp[at] = cpr[i];
+        for (int i = 0; i < kCandPer; ++i) {
+          if (cpr[i] >= 0 && ((ckr[i] >> kFineShift) & (kFineBins - 1)) == b2) {
+            const int at = atomicAdd(&misc[kMNm], 1);
+            if (at < kMemberMax) {
+              mk[at] = ckr[i];
+              mp[at] = cpr[i];
+            }
           }
         }
       }
@@ -557,18 +443,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Selected candidates: this chunk's into the selected bits, earlier
       // chunks' counted for the output offset.
       int before = nsure_before;
+#pragma unroll 1
+      for (int bt = 0; bt < n_batches; ++bt) {
+        if (n_batches > 1) load_batch(bt);
 #pragma unroll
-      for (int i = 0; i < kCandPer; ++i) {
-        const uint32_t key = ckr[i];
-        const int pos = cpr[i];
-        const uint32_t sub = (key >> kFineShift) & (kFineBins - 1);
-        const bool selc = pos >= 0 && (sub > b2 || (sub == b2 && (key > th_key ||
-                                                                  (key == th_key && pos <= th_pos))));
-        if (selc) {
-          if (pos < s0) {
-            ++before;
-          } else if (pos < s1) {
-            atomicOr(&sbits[(pos - s0) >> 5], 1u << ((pos - s0) & 31));
+        for (int i = 0; i < kCandPer; ++i) {
+          const uint32_t key = ckr[i];
+          const int pos = cpr[i];
+          const uint32_t sub = (key >> kFineShift) & (kFineBins - 1);
+          const bool selc =
+              pos >= 0 && (sub > b2 || (sub == b2 && (key > th_key ||
+                                                       (key == th_key && pos <= th_pos))));
+          if (selc) {
+            if (pos < s0) {
+              ++before;
+            } else if (pos < s1) {
+              atomicOr(&sbits[(pos - s0) >> 5], 1u << ((pos - s0) & 31));
+            }
           }
         }
       }
@@ -577,103 +468,127 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       // This chunk's selected positions, in order, at `offset`.
       const uint32_t sw = tid < nw ? sbits[tid] : 0u;
-      int n_sel;
-      const int ex = offset + block_excl_sum_nw<kWarps>(__popc(sw), buf, n_sel);
+      int n_sel_chunk;
+      const int ex = offset + block_excl_sum_nw<kWarps>(__popc(sw), buf, n_sel_chunk);
       uint32_t m = sw;
       for (int j = 0; m != 0u; ++j) {
         const int bit = __ffs(m) - 1;
         m &= m - 1u;
         if (ex + j < k) idx_row[ex + j] = s0 + 32 * tid + bit;
       }
-    } else {
-      // Heavily tied row: the row's first CTA selects over the whole row;
-      // the others take their chunk's positions from its result.
-      if (c == 0) {
-        int* const fh = reinterpret_cast<int*>(bp + kOffP);
-        row_select_global<kWarps>(sc, n, k, idx_row, fh, buf);
-        __syncthreads();
-        if (tid == 0) {
-          __threadfence();
-          atomicExch(ctr + kCtrFallback, 1);
-        }
-      } else if (tid == 0) {
-        if (!wait_flag(ctr + kCtrFallback, P.err)) misc[kMAbort] = 1;
-      }
-      __syncthreads();
-      if (misc[kMAbort] != 0) ok = false;
-      if (ok) {
-        for (int w = tid; w < nw; w += kThreads) sbits[w] = 0u;
-        __syncthreads();
-        for (int i = tid; i < k; i += kThreads) {
-          const int pos = __ldcg(idx_row + i);
-          if (pos >= s0 && pos < s1) atomicOr(&sbits[(pos - s0) >> 5], 1u << ((pos - s0) & 31));
-        }
-        __syncthreads();
-        // Tiles from the selected positions alone.
-        const uint32_t sw = tid < nw ? sbits[tid] : 0u;
-        if (tid < nw) tbits[tid] = sw;
-        int nt;
-        const int ex = block_excl_sum_nw<kWarps>(__popc(sw), buf, nt);
-        if (tid < kMaxWords) pre[tid] = ex;
-        if (tid == 0) misc[kMNTile] = nt;
-        respec = true;
-      }
+    } else if (c == 0) {
+      // Heavily tied row: the row's first CTA selects over the whole row.
+      int* const fh = reinterpret_cast<int*>(bp + kOffP);
+      row_select_global<kWarps>(sc, n, k, idx_row, fh, buf);
     }
   } else if (ok && full) {
-    // Every position is kept: this chunk's positions at their own index, and
-    // the padding past n from the first CTA.
+    // Every position is kept, in its own slot; the padding past n from the
+    // first CTA.
     for (int i = s0 + tid; i < s1; i += kThreads) idx_row[i] = i;
     if (c == 0) {
       for (int i = n + tid; i < k; i += kThreads) idx_row[i] = -1;
     }
   }
   __syncthreads();
-  n_tile = misc[kMNTile];
-  const int n_tiles = ok ? (n_tile + kTile - 1) / kTile : 0;
+  // The row's index set is complete once every CTA of the row has written its
+  // part (rows that keep every position need no wait: slot i holds i).
+  if (ok && !full && tid == 0) {
+    if (!row_arrive_wait(ctr + kCtrBarC, P.C, P.err)) row_ok = false;
+  }
+  __syncwarp();
+  ok = ok && !__syncthreads_or(!row_ok);
 
   // ---------------------------------------------------------- phase C ----
+  // This CTA's equal share of the row's selected slots, in tiles of kTile.
+  const int n_sel = min(k, n);
+  const int share = (n_sel + P.C - 1) / P.C;
+  const int slot_lo = min(n_sel, c * share);
+  const int slot_hi = min(n_sel, slot_lo + share);
+  const int n_tiles = ok ? (slot_hi - slot_lo + kTile - 1) / kTile : 0;
+  // Positions and cache rows of tile t of the share, -1 past its end.
+  auto map_tile = [&](int t) {
+    if (tid < kTile) {
+      const int g = slot_lo + t * kTile + tid;
+      const int pos = g < slot_hi ? (full ? g : __ldcg(idx_row + g)) : -1;
+      tpos[tid] = pos;
+      trow[tid] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
+    }
+  };
+  // The tile's rows in 16-byte pieces (cp.async, 128-byte swizzle): thread
+  // (sub, piece) copies piece `piece` of every box of rows sub, sub + 64: a
+  // warp instruction reads four whole 128-byte lines, its four swizzled rows
+  // cover every shared-memory bank four times, and the swizzle (row & 7 ==
+  // sub & 7) is fixed per thread.  Every thread arrives on kv_full once its
+  // copies have landed.
+  auto gather_tile = [&]() {
+    const uint32_t piece = static_cast<uint32_t>(tid & 7);
+    const int sub = tid >> 3;
+    const uint32_t sw = (piece ^ static_cast<uint32_t>(sub & 7)) << 4;
+    for (int i = sub; i < kTile; i += kThreads >> 3) {
+      const int row = trow[i];
+      const uint32_t dst = sKV + i * 128 + sw;
+      if (row >= 0) {
+        const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + piece * 8;
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) cp_async16_tc(dst + bx * kKVBox, src + bx * 64);
+      } else {
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + bx * kKVBox), "r"(0u)
+                       : "memory");
+        }
+      }
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+    fence_proxy_async_smem();
+    mbar_arrive(b_kvfull);
+  };
+  // Warp 4: S = Q K_tile^T for the gathered tile t.
+  auto issue_s = [&](int t) -> bool {
+    bool good = __all_sync(0xffffffffu, mbar_wait(b_qfull, 0, P.err));
+    good = good && __all_sync(0xffffffffu, mbar_wait(b_kvfull, static_cast<uint32_t>(t & 1), P.err));
+    if (!good) return false;
+    tc_fence_after();
+    const uint64_t dq = sdesc_sw128(sQ), dk = sdesc_sw128(sKV);
+#pragma unroll 4
+    for (int ks = 0; ks < kLatent / 16; ++ks) {
+      const uint32_t off = (ks & 3) * 32;
+      tc_mma_bf16_warp(tmem + kColS, dq + static_cast<uint64_t>(((ks >> 2) * kQBox + off) >> 4),
+                       dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4), kIdescS,
+                       ks > 0 ? 1u : 0u);
+    }
+    tc_commit_warp(b_sfull);
+    return true;
+  };
+
   float m_run = -INFINITY, l_run = 0.f;
   const int q4 = warp;  // softmax warps 0-3: TMEM lane quadrant
   const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
   const bool owner = lane < 16;
   const int hl = 16 * q4 + (lane & 15);
-  int o_round = 0;  // P.V products issued (== tiles done)
   for (int t = 0; t < n_tiles && ok; ++t) {
-    const bool spec = t == 0 && !respec;
-    if (!spec) {
-      // The previous round's products must be done with KV, S and P.
-      bool good = true;
-      if (t > 0) good = mbar_wait(b_odone, static_cast<uint32_t>((t - 1) & 1), P.err);
-      else good = mbar_wait(b_sfull, 0, P.err);  // the discarded speculative S
+    if (t > 0) {  // the previous tile's products must be done with KV, S and P
+      const bool good = mbar_wait(b_odone, static_cast<uint32_t>((t - 1) & 1), P.err);
       ok = !__syncthreads_or(!good);
       if (!ok) break;
       tc_fence_after();
-      map_tile(t);
-      __syncthreads();
-      gather_tile();
-      gather_done();
-      if (warp == 4 && !issue_s(s_round)) row_ok = false;
-      ++s_round;
     }
-    const int it = s_round - 1;  // this tile's gather/S round
-    if (tid < kTile) {
-      const int pos = tpos[tid];
-      tsel[tid] = pos >= 0 && ((sbits[(pos - s0) >> 5] >> ((pos - s0) & 31)) & 1u);
-    }
+    map_tile(t);
     __syncthreads();
+    gather_tile();
+    if (warp == 4 && !issue_s(t)) row_ok = false;
     if (warp < 4) {
       // ------------------------------------------------------- softmax --
-      bool good = mbar_wait(b_sfull, static_cast<uint32_t>(it & 1), P.err);
-      if (good && t > 0) good = mbar_wait(b_odone, static_cast<uint32_t>((t - 1) & 1), P.err);
+      const bool good = mbar_wait(b_sfull, static_cast<uint32_t>(t & 1), P.err);
       if (good) {
         tc_fence_after();
         uint32_t va[32], vb[16];
         tmem_ld_16x32bx2_x32<kHalf>(tmem + lane_base + kColS, va);
         tmem_ld_16x32bx2_x16<kHalf>(tmem + lane_base + kColS + 32u, vb);
         tmem_ld_wait();
-        const unsigned v0 = __ballot_sync(0xffffffffu, tsel[lane] != 0);
-        const unsigned v1 = __ballot_sync(0xffffffffu, tsel[32 + lane] != 0);
-        const unsigned v2 = __ballot_sync(0xffffffffu, tsel[64 + lane] != 0);
+        const unsigned v0 = __ballot_sync(0xffffffffu, tpos[lane] >= 0);
+        const unsigned v1 = __ballot_sync(0xffffffffu, tpos[32 + lane] >= 0);
+        const unsigned v2 = __ballot_sync(0xffffffffu, tpos[64 + lane] >= 0);
         const int k0 = (lane >> 4) * kHalf;
         const unsigned long long valid =
             k0 == 0 ? (static_cast<unsigned long long>(v1 & 0xFFFFu) << 32) | v0
@@ -730,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (good && any) {
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll
+#pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             uint32_t o[32];
             const uint32_t ta = tmem + lane_base + kColO + 64u * blk + 32u * half;
@@ -755,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint64_t dv = sdesc_sw128_mn(sKV, kKVBox);
         const uint64_t dp = sdesc_sw128(sP);
-#pragma unroll
+#pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
@@ -769,7 +684,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         tc_commit_warp(b_odone);
-        ++o_round;
       } else {
         row_ok = false;
       }
@@ -811,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok && tid == 0) {
     if (!row_arrive_wait(ctr + kCtrBarD, P.C, P.err)) misc[kMAbort] = 1;
   }
+  __syncwarp();
   __syncthreads();
   ok = ok && misc[kMAbort] == 0;
 
@@ -845,49 +760,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncthreads();
       // G threads per output unit (a float4 of one head), each summing every
-      // G-th chunk's partial with all of its loads in flight, then combined
-      // with shuffles; chunks in a fixed order, so the result is deterministic.
+      // G-th chunk's partial with its loads in flight together, combined with
+      // shuffles; chunks in a fixed order, so the result is deterministic.
+      // Units beyond kThreads / G per pass take further passes.
       const int nu = u1 - u0;
       int G = 1;
       while (G < 32 && 2 * G * nu <= kThreads) G *= 2;
-      const int ui = tid / G, sub = tid - ui * G;
-      const int u = u0 + ui;
-      const bool act = ui < nu;
-      const int h = act ? u / (kValue / 4) : hlo;
-      const int d4 = act ? u - h * (kValue / 4) : 0;
-      const float* const wr = wgt + (h - hlo) * P.C;
-      const float* const po = P.part_o + (static_cast<size_t>(r) * P.C * kHB + h) * kValue + 4 * d4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      constexpr int kU = 10;
-      for (int j0 = sub; j0 < P.C; j0 += kU * G) {
-        float4 x[kU];
+      const int per_pass = kThreads / G;
+      const int sub = tid % G;
+#pragma unroll 1
+      for (int ub = 0; ub < nu; ub += per_pass) {
+        const int ui = ub + tid / G;
+        const bool act = ui < nu;
+        const int u = u0 + (act ? ui : 0);
+        const int h = u / (kValue / 4);
+        const int d4 = u - h * (kValue / 4);
+        const float* const wr = wgt + (h - hlo) * P.C;
+        const float* const po =
+            P.part_o + (static_cast<size_t>(r) * P.C * kHB + h) * kValue + 4 * d4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        constexpr int kU = 10;
+#pragma unroll 1
+        for (int j0 = sub; j0 < P.C; j0 += kU * G) {
+          float4 x[kU];
 #pragma unroll
-        for (int jj = 0; jj < kU; ++jj) {
-          const int j = j0 + jj * G;
-          x[jj] = (act && j < P.C && wr[j] != 0.f)
-                      ? __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(j) * kHB *
-                                                                        kValue))
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+          for (int jj = 0; jj < kU; ++jj) {
+            const int j = j0 + jj * G;
+            x[jj] = (act && j < P.C && wr[j] != 0.f)
+                        ? __ldcg(reinterpret_cast<const float4*>(po + static_cast<size_t>(j) *
+                                                                          kHB * kValue))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
 #pragma unroll
-        for (int jj = 0; jj < kU; ++jj) {
-          const int j = j0 + jj * G;
-          const float wj = (act && j < P.C) ? wr[j] : 0.f;
-          acc.x = fmaf(wj, x[jj].x, acc.x);
-          acc.y = fmaf(wj, x[jj].y, acc.y);
-          acc.z = fmaf(wj, x[jj].z, acc.z);
-          acc.w = fmaf(wj, x[jj].w, acc.w);
+          for (int jj = 0; jj < kU; ++jj) {
+            const int j = j0 + jj * G;
+            const float wj = (act && j < P.C) ? wr[j] : 0.f;
+            acc.x = fmaf(wj, x[jj].x, acc.x);
+            acc.y = fmaf(wj, x[jj].y, acc.y);
+            acc.z = fmaf(wj, x[jj].z, acc.z);
+            acc.w = fmaf(wj, x[jj].w, acc.w);
+          }
         }
-      }
-      for (int o2 = 1; o2 < G; o2 <<= 1) {  // the G threads of a unit are adjacent lanes
-        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o2);
-        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o2);
-        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o2);
-        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o2);
-      }
-      if (act && sub == 0) {
-        *reinterpret_cast<float4*>(P.out + (static_cast<size_t>(r) * P.H + h) * kValue + 4 * d4) =
-            acc;
+        for (int o2 = 1; o2 < G; o2 <<= 1) {  // the G threads of a unit are adjacent lanes
+          acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o2);
+          acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o2);
+          acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o2);
+          acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o2);
+        }
+        if (act && sub == 0) {
+          *reinterpret_cast<float4*>(P.out + (static_cast<size_t>(r) * P.H + h) * kValue +
+                                     4 * d4) = acc;
+        }
       }
     }
   }
@@ -949,6 +872,7 @@ cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   }
   cudaError_t e = ensure_smem_limit<decode_tail_kernel>(kSmemBytes);
+  if (e == cudaSuccess) e = prefer_max_shared(reinterpret_cast<const void*>(decode_tail_kernel));
   if (e != cudaSuccess) return e;
   const int C = decode_tail_chunks(a.Nq, a.num_sms);
   TailParams P;

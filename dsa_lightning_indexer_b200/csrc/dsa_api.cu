@@ -6,6 +6,8 @@
 
 #include <algorithm>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "../../include/dsa.h"
 #include "dsa_common.cuh"
@@ -25,6 +27,20 @@ EncodeTiledFn get_encode_tiled() {
     return reinterpret_cast<EncodeTiledFn>(p);
   }();
   return fn;
+}
+
+cudaError_t prefer_max_shared(const void* kernel) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev}) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done.insert({kernel, dev});
+  return e;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -191,11 +191,20 @@ cudaError_t ensure_smem_limit(int bytes) {
   return e;
 }
 
+// Asks for the largest shared-memory carveout for `kernel`, once per device.
+// Every kernel of the library then runs with the same L1 / shared-memory
+// split, so an SM moving from one kernel's CTAs to the next one's (dependent
+// launches start CTAs as soon as SMs free up) does not first have to change
+// its split.
+cudaError_t prefer_max_shared(const void* kernel);
+
 // Launches `kernel` on `stream` as a programmatic dependent of the work before
 // it (see pdl_wait), optionally as clusters of `cluster_x` CTAs.
 template <typename Kernel, typename... Args>
 cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        int cluster_x, Args... args) {
+  const cudaError_t ce = prefer_max_shared(reinterpret_cast<const void*>(kernel));
+  if (ce != cudaSuccess) return ce;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

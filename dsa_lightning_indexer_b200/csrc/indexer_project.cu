@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[s] != 2u) mbar_drain(full(s), last[s], P.err);
       }
     }
+    __syncwarp();  // the warp meets the CTA barrier below reconverged
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0 && !abort) {
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain);
       mbar_drain(drain, 0, P.err);
     }
+    __syncwarp();
   } else {
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;

@@ -24,10 +24,10 @@
 // Optionally, the epilogue also counts each stored score into its row's
 // 4096-bin histogram of the top 12 bits of its order-preserving key; the
 // top-k selection then needs only one filtering pass over the row.  With one
-// query per item the counts gather in shared memory (one aggregated atomic
-// per warp per distinct bin) and are flushed to the row's histogram after
-// each item; with several queries per item (multi-token decode) each warp
-// adds its aggregated counts to the rows' global histograms directly.
+// query per item the counts gather in shared memory (one atomic per key) and
+// are flushed to the row's histogram after each item; with several queries
+// per item (multi-token decode) each warp adds its counts, aggregated per
+// distinct bin, to the rows' global histograms directly.
 #include <string.h>
 
 #include <algorithm>
@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         if (q_last[i] != 2u) mbar_drain(qfull(i), q_last[i], P.err);
       }
     }
+    __syncwarp();  // the warp meets the CTA barrier below reconverged
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0 && !abort) {
@@ -304,6 +305,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       tc_commit(drain);
       mbar_drain(drain, 0, P.err);
     }
+    __syncwarp();
   } else {
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
@@ -350,16 +352,16 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           if (s == 0.f) s = 0.f;  // one zero: -0 and +0 are the same score
           const bool valid = key <= v.pos0 + jq;
           if (valid) P.scores[static_cast<size_t>(v.row0 + jq) * P.ld + key] = s;
-          if (do_hist || do_ghist) {
+          if (do_hist) {
+            // One shared-memory atomic per key: the keys of a warp are spread
+            // over many bins, so they rarely collide.
+            if (valid) atomicAdd(&shist[score_key(s) >> kHistShift], 1);
+          } else if (do_ghist) {
+            // Global atomics are costly: one per distinct bin of the warp.
             const uint32_t bin = valid ? (score_key(s) >> kHistShift) : 0xFFFFFFFFu;
             const unsigned grp = __match_any_sync(0xffffffffu, bin);
             if (valid && lane == __ffs(grp) - 1) {
-              if (do_hist) {
-                atomicAdd(&shist[bin], __popc(grp));
-              } else {
-                atomicAdd(P.hist + static_cast<size_t>(v.row0 + jq) * kHistBins + bin,
-                          __popc(grp));
-              }
+              atomicAdd(P.hist + static_cast<size_t>(v.row0 + jq) * kHistBins + bin, __popc(grp));
             }
           }
         }

@@ -135,24 +135,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tidx[g] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
       }
       named_bar_sync(2, kGatherThreads);
-      // Each thread copies whole 128-byte box rows: eight 16-byte pieces with
-      // the swizzle applied.
-      for (int item = g; item < kTD * kBoxes; item += kGatherThreads) {
-        // Rows fastest: a warp's lanes take consecutive rows of one box, so
-        // the swizzled 16-byte pieces of one instruction spread over all
-        // eight bank groups of shared memory.
-        const int bx = item / kTD, i = item - bx * kTD;
+      // Thread (sub, piece) copies 16-byte piece `piece` of every box of
+      // rows sub, sub + 16, ...: a warp instruction reads four whole 128-byte
+      // lines, its four swizzled rows cover every shared-memory bank four
+      // times, and the swizzle (row & 7 == sub & 7) is fixed per thread.
+      const uint32_t piece = static_cast<uint32_t>(g & 7);
+      const int sub = g >> 3;
+      const uint32_t sw = (piece ^ static_cast<uint32_t>(sub & 7)) << 4;
+      for (int i = sub; i < kTD; i += kGatherThreads >> 3) {
         const int row = tidx[i];
-        const uint32_t drow = sKV + bx * kKVBox + i * 128;
-        const uint32_t x = static_cast<uint32_t>(i & 7);
+        const uint32_t dst = sKV + i * 128 + sw;
         if (row >= 0) {
-          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
+          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + piece * 8;
 #pragma unroll
-          for (uint32_t c = 0; c < 8; ++c) cp_async16_tc(drow + ((c ^ x) << 4), src + c * 8);
+          for (int bx = 0; bx < kBoxes; ++bx) cp_async16_tc(dst + bx * kKVBox, src + bx * 64);
         } else {
 #pragma unroll
-          for (uint32_t c = 0; c < 8; ++c) {
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(drow + (c << 4)),
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + bx * kKVBox),
                          "r"(0u)
                          : "memory");
           }

@@ -199,8 +199,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
   } else if (warp >= 5) {
     // ------------------------------------------------------------ gather --
-    // Each thread copies whole 128-byte box rows (eight 16-byte pieces with
-    // the swizzle applied), after the group has staged the tile's positions.
+    // The group copies the tile's rows in 16-byte pieces with the swizzle
+    // applied, after it has staged the tile's positions.
     const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
     const int gt = threadIdx.x - (5 + 2 * grp) * 32;
     int* const gidx = tidx + grp * kT;
@@ -242,22 +242,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       row_cur = row_nxt;
       row_nxt = load_row(t + 4);
       const uint32_t stage = sKV + grp * kKVStage;
-      for (int item = gt; item < kT * kBoxes; item += kGroupThreads) {
-        // Rows fastest: a warp's lanes take consecutive rows of one box, so
-        // the swizzled 16-byte pieces of one instruction spread over all
-        // eight bank groups of shared memory.
-        const int bx = item / kT, i = item - bx * kT;
+      // Thread (sub, piece) copies 16-byte piece `piece` of every box of
+      // rows sub, sub + 8, ...: a warp instruction reads four whole 128-byte
+      // lines, its four swizzled rows cover every shared-memory bank four
+      // times, and the swizzle (row & 7 == sub) is fixed per thread.
+      const uint32_t piece = static_cast<uint32_t>(gt & 7);
+      const int sub = gt >> 3;
+      const uint32_t sw = (piece ^ static_cast<uint32_t>(sub)) << 4;
+      for (int i = sub; i < kT; i += kGroupThreads >> 3) {
         const int row = gidx[i];
-        const uint32_t drow = stage + bx * kKVBox + i * 128;
-        const uint32_t x = static_cast<uint32_t>(i & 7);
+        const uint32_t dst = stage + i * 128 + sw;
         if (row >= 0) {
-          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + bx * 64;
+          const __nv_bfloat16* src = P.kv + static_cast<size_t>(row) * kLatent + piece * 8;
 #pragma unroll
-          for (uint32_t c = 0; c < 8; ++c) cp_async16_tc(drow + ((c ^ x) << 4), src + c * 8);
+          for (int bx = 0; bx < kBoxes; ++bx) cp_async16_tc(dst + bx * kKVBox, src + bx * 64);
         } else {
 #pragma unroll
-          for (uint32_t c = 0; c < 8; ++c) {
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(drow + (c << 4)),
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + bx * kKVBox),
                          "r"(0u)
                          : "memory");
           }

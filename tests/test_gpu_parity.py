@@ -414,3 +414,10 @@ def test_layer_decode_concentrated_selection():
     # row 0 really concentrates: most of its selection lies in the planted range
     sel = got_idx[0]
     assert ((sel >= 5000) & (sel < 8000)).sum() >= 1500
+
+
+def test_layer_decode_14_rows():
+    """14 decode rows: 10 chunks per row in the fused tail, so each CTA merges
+    more output units than it has threads (several passes)."""
+    _layer_check(synth.custom([20000, 20000, 9000, 9000, 9000, 9000] + [30000] * 8, [1] * 14, 64,
+                              2048, seed=165))
