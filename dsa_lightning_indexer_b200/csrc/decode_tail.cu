@@ -10,8 +10,7 @@
 // key-only latent cache whose leading 512 entries serve as V.)
 //
 // One cooperative launch of Nq x C CTAs (one per SM); CTA (r, c) owns chunk
-// c of row r's causal positions [s0, s1) for the selection and an equal
-// share of the row's selected slots for the attention.  Phases:
+// c of row r's causal positions [s0, s1).  Phases:
 //   A  From the row's 4096-bin histogram of the top 12 key bits (built by the
 //      indexer) find the bin holding the k-th largest key.  Read the chunk's
 //      scores once: positions above that bin are selected for sure, positions
@@ -23,11 +22,14 @@
 //      key and rank its few members exactly; write this chunk's selected
 //      positions, in order, into the row's index set.  Heavily tied rows
 //      (candidate list or sub-bin too full) fall back to an exact whole-row
-//      select by the row's first CTA.  Arrive on the row's second counter.
-//   C  When the index set is complete, take slots [c*ceil(k/C), ...) of it:
-//      gather those rows in tiles of 96, S = Q K^T, softmax, P as bf16 hi +
-//      lo, O^T = V^T P^T into TMEM with a running maximum; the unnormalised
-//      O and (max, sum) of every head go to the row's partial results.
+//      select by the row's first CTA.
+//   C  Attend over the chunk's own selected positions when every chunk of
+//      the row holds at most one tile of them (known to every CTA from the
+//      per-chunk counts, so no further barrier); otherwise, once the index
+//      set is complete, over slots [c*ceil(k/C), ...) of it.  Rows are
+//      gathered in tiles of 96: S = Q K^T, softmax, P as bf16 hi + lo,
+//      O^T = V^T P^T into TMEM with a running maximum; the unnormalised O
+//      and (max, sum) of every head go to the row's partial results.
 //   D  When every CTA of the row has stored its partials, each merges a
 //      1/C share of the row's output with the log-sum-exp rule.
 // Every wait is bounded; a wait that runs out sets the workspace error word
@@ -84,13 +86,12 @@ constexpr int kSmemBytes = kSmemUsed + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 // Phase-B scratch (member list, fallback histogram) and the merge weights
 // live in the P region, which phase C writes only after them.
-static_assert(kMemberMax * 12 <= 4 * kPBlk, "member list fits the P region");
+static_assert(kMemberMax * 8 + 160 * 4 <= 4 * kPBlk, "member list and chunk counts fit the P region");
 static_assert(2048 * 4 <= 4 * kPBlk, "fallback histogram fits the P region");
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S: 96 columns (M = 64 layout)
 constexpr uint32_t kColO = 128;    // O^T blocks at 128, 192, 256, 320
-constexpr uint32_t kIdescS = idesc_bf16_f32(64, kTile);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
 
 // Shared scalars.
@@ -358,6 +359,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   ok = ok && !__syncthreads_or(!row_ok);
 
   // ---------------------------------------------------------- phase B ----
+  // own: every chunk of the row holds at most kTile selected positions, and
+  // this CTA attends over its own chunk's (n_own of them, in tpos) with no
+  // further row barrier.  The decision is the same in every CTA of the row.
+  bool own = false;
+  int n_own = 0;
   if (ok && !full) {
     const int need = k - c_above;  // keys to keep from the threshold bin, 1 .. c_in
     const bool listed = c_in <= kCandMax;  // every candidate of the row is in the list
@@ -380,8 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     load_batch(0);
-    const int nsure_before =
-        tid < c ? __ldcg(P.chunk_nsure + static_cast<size_t>(r) * P.C + tid) : 0;
+    const int nsure_t = tid < P.C ? __ldcg(P.chunk_nsure + static_cast<size_t>(r) * P.C + tid) : 0;
+    const int nsure_before = tid < c ? nsure_t : 0;
+    int* const ccount = reinterpret_cast<int*>(bp + kOffP + kMemberMax * 8);  // [C]
     // Sub-bin of the need-th key of the bin: thread t holds sub-bins 4u .. 4u+3.
     {
       const int u = kThreads - 1 - tid;
@@ -402,6 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (tid == 0) misc[kMNm] = 0;
+      for (int i = tid; i < P.C; i += kThreads) ccount[i] = 0;
       __syncthreads();
     }
     const uint32_t b2 = static_cast<uint32_t>(misc[kMB2]);
@@ -455,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               pos >= 0 && (sub > b2 || (sub == b2 && (key > th_key ||
                                                        (key == th_key && pos <= th_pos))));
           if (selc) {
+            atomicAdd(&ccount[pos / S], 1);
             if (pos < s0) {
               ++before;
             } else if (pos < s1) {
@@ -463,19 +472,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      __syncthreads();
+      own = !__syncthreads_or(tid < P.C && nsure_t + ccount[tid] > kTile);
+      if (tid < kTile) tpos[tid] = -1;
       int offset;
       block_excl_sum_nw<kWarps>(before, buf, offset);
       __syncthreads();
-      // This chunk's selected positions, in order, at `offset`.
+      // This chunk's selected positions, in order, at `offset` (and, when
+      // attending over the own chunk, at 0.. in tpos).
       const uint32_t sw = tid < nw ? sbits[tid] : 0u;
       int n_sel_chunk;
-      const int ex = offset + block_excl_sum_nw<kWarps>(__popc(sw), buf, n_sel_chunk);
+      const int lx = block_excl_sum_nw<kWarps>(__popc(sw), buf, n_sel_chunk);
+      const int ex = offset + lx;
       uint32_t m = sw;
       for (int j = 0; m != 0u; ++j) {
         const int bit = __ffs(m) - 1;
         m &= m - 1u;
-        if (ex + j < k) idx_row[ex + j] = s0 + 32 * tid + bit;
+        const int pos = s0 + 32 * tid + bit;
+        if (ex + j < k) idx_row[ex + j] = pos;
+        if (own) tpos[lx + j] = pos;  // lx + j < n_sel_chunk <= kTile
       }
+      n_own = n_sel_chunk;
     } else if (c == 0) {
       // Heavily tied row: the row's first CTA selects over the whole row.
       int* const fh = reinterpret_cast<int*>(bp + kOffP);
@@ -492,25 +509,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   // The row's index set is complete once every CTA of the row has written its
   // part (rows that keep every position need no wait: slot i holds i).
-  if (ok && !full && tid == 0) {
+  if (ok && !full && !own && tid == 0) {
     if (!row_arrive_wait(ctr + kCtrBarC, P.C, P.err)) row_ok = false;
   }
   __syncwarp();
   ok = ok && !__syncthreads_or(!row_ok);
 
   // ---------------------------------------------------------- phase C ----
-  // This CTA's equal share of the row's selected slots, in tiles of kTile.
+  // The own chunk's selected positions (one tile), or else this CTA's equal
+  // share of the row's selected slots, in tiles of kTile.
   const int n_sel = min(k, n);
   const int share = (n_sel + P.C - 1) / P.C;
   const int slot_lo = min(n_sel, c * share);
   const int slot_hi = min(n_sel, slot_lo + share);
-  const int n_tiles = ok ? (slot_hi - slot_lo + kTile - 1) / kTile : 0;
-  // Positions and cache rows of tile t of the share, -1 past its end.
+  const int n_tiles = !ok ? 0 : own ? (n_own > 0 ? 1 : 0) : (slot_hi - slot_lo + kTile - 1) / kTile;
+  // Positions and cache rows of tile t, -1 past its end.
   auto map_tile = [&](int t) {
     if (tid < kTile) {
-      const int g = slot_lo + t * kTile + tid;
-      const int pos = g < slot_hi ? (full ? g : __ldcg(idx_row + g)) : -1;
-      tpos[tid] = pos;
+      int pos;
+      if (own) {
+        pos = tpos[tid];
+      } else {
+        const int g = slot_lo + t * kTile + tid;
+        pos = g < slot_hi ? (full ? g : __ldcg(idx_row + g)) : -1;
+        tpos[tid] = pos;
+      }
       trow[tid] = pos >= 0 ? static_cast<int>(seq_row(rs.rows, pos)) : -1;
     }
   };
@@ -520,11 +543,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // cover every shared-memory bank four times, and the swizzle (row & 7 ==
   // sub & 7) is fixed per thread.  Every thread arrives on kv_full once its
   // copies have landed.
-  auto gather_tile = [&]() {
+  // Only the ncol rows the products read are copied (zeros past the tile's
+  // own rows).
+  auto gather_tile = [&](int ncol) {
     const uint32_t piece = static_cast<uint32_t>(tid & 7);
     const int sub = tid >> 3;
     const uint32_t sw = (piece ^ static_cast<uint32_t>(sub & 7)) << 4;
-    for (int i = sub; i < kTile; i += kThreads >> 3) {
+    for (int i = sub; i < ncol; i += kThreads >> 3) {
       const int row = trow[i];
       const uint32_t dst = sKV + i * 128 + sw;
       if (row >= 0) {
@@ -543,8 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
     mbar_arrive(b_kvfull);
   };
-  // Warp 4: S = Q K_tile^T for the gathered tile t.
-  auto issue_s = [&](int t) -> bool {
+  // Warp 4: S = Q K_tile^T for the gathered tile t (its first ncol rows).
+  auto issue_s = [&](int t, int ncol) -> bool {
     bool good = __all_sync(0xffffffffu, mbar_wait(b_qfull, 0, P.err));
     good = good && __all_sync(0xffffffffu, mbar_wait(b_kvfull, static_cast<uint32_t>(t & 1), P.err));
     if (!good) return false;
@@ -554,7 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int ks = 0; ks < kLatent / 16; ++ks) {
       const uint32_t off = (ks & 3) * 32;
       tc_mma_bf16_warp(tmem + kColS, dq + static_cast<uint64_t>(((ks >> 2) * kQBox + off) >> 4),
-                       dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4), kIdescS,
+                       dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4),
+                       idesc_bf16_f32(64, static_cast<uint32_t>(ncol)),
                        ks > 0 ? 1u : 0u);
     }
     tc_commit_warp(b_sfull);
@@ -573,10 +599,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
     }
+    // Rows of this tile, and the product width: a multiple of 16 covering them.
+    const int rows_t = own ? n_own : min(kTile, slot_hi - slot_lo - t * kTile);
+    const int ncol = min(kTile, max(16, (rows_t + 15) & ~15));
     map_tile(t);
     __syncthreads();
-    gather_tile();
-    if (warp == 4 && !issue_s(t)) row_ok = false;
+    gather_tile(ncol);
+    if (warp == 4 && !issue_s(t, ncol)) row_ok = false;
     if (warp < 4) {
       // ------------------------------------------------------- softmax --
       const bool good = mbar_wait(b_sfull, static_cast<uint32_t>(t & 1), P.err);
@@ -672,8 +701,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dp = sdesc_sw128(sP);
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
+#pragma unroll 2
+          for (int kk = 0; kk < ncol / 16; ++kk) {
             const uint64_t a = dv + static_cast<uint64_t>(((2 * blk) * kKVBox + kk * 2048) >> 4);
             const uint32_t d = tmem + kColO + 64u * blk;
             const uint64_t bo =

@@ -289,7 +289,10 @@ size_t dsa_workspace_size(const dsa_batch* batch, int H, int top_k, uint32_t fla
       check_topk(top_k) != DSA_OK || (flags & ~DSA_FLAG_MASKED_ROUTE) != 0u) {
     return 0;
   }
-  size_t total = plan_ws(batch, info, H, top_k, true, true).total;
+  // The layer call and the standalone attention call (whose slice partials
+  // the fused layer does not need) on the same workspace.
+  size_t total = std::max(plan_ws(batch, info, H, top_k, true, true).total,
+                          plan_ws(batch, info, H, top_k, false, true).total);
   if ((flags & DSA_FLAG_MASKED_ROUTE) != 0u) {
     total = std::max(total, masked_ws_need(batch, info, H));
   }

@@ -117,8 +117,11 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_workspace_grows_with_the_problem():
-    small = FakeBatch([0, 1], [0, 1024], [1024])
-    big = FakeBatch([0, 1], [0, 131072], [131072])
+    # One row of 4M positions needs its 16 MB of scores on top of the control
+    # block; one row of 128K fits in far less.
+    small = FakeBatch([0, 1], [0, 131072], [131072])
+    big = FakeBatch([0, 1], [0, 1 << 22], [1 << 22])
+    assert bd.lib.dsa_workspace_size(big.ref, 64, 2048, 0) > (1 << 22) * 4
     assert bd.lib.dsa_workspace_size(big.ref, 64, 2048, 0) > bd.lib.dsa_workspace_size(
         small.ref, 64, 2048, 0)
 
