@@ -274,8 +274,8 @@ def indexer_causal_flops(wl):
 def launches_per_layer(wl, sms=148):
     """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
     sequences with queries), then either the fused decode tail (selection,
-    attention and merge in one kernel: few long single-query rows, at most 64
-    heads), or the top-k selection -- two kernels (filter and emit) when the
+    attention and merge in one kernel: 6 to 12 long rows, at most 64 heads),
+    or the top-k selection -- two kernels (filter and emit) when the
     indexer's histograms drive it, else one -- followed by the sparse
     attention and, when few rows split the selected set over CTAs, the merge
     of the slices."""
@@ -288,7 +288,7 @@ def launches_per_layer(wl, sms=148):
     hist = (0 < wl.Nq <= 148 and max_len >= 8192 and max_len >= 4 * wl.top_k
             and -(-max_len // chunk) <= 512)
     C = 148 // max(1, wl.Nq)
-    fused = (hist and wl.H <= 64 and wl.Nq <= 16 and C >= 8
+    fused = (hist and wl.H <= 64 and 6 <= wl.Nq <= 12 and C >= 8
              and (-(-max_len // C) + 31) // 32 <= 512)
     if fused:
         return (seqs + 63) // 64 + 1

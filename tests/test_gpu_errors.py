@@ -115,7 +115,8 @@ def test_out_of_range_indices_are_skipped_and_reported(name):
 
 
 def _hist_decode():
-    return synth.custom([9000, 1500, 20000, 40000], [1] * 4, 16, 2048, seed=163)
+    # six single-token rows: the layer takes the fused tail
+    return synth.custom([9000, 1500, 20000, 40000, 7000, 12000], [1] * 6, 16, 2048, seed=163)
 
 
 def test_standalone_histogram_path_matches_the_layer():

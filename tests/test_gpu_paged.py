@@ -28,9 +28,12 @@ def _up4(x):
 
 
 CASES = {
-    # decode, fused tail: ragged lengths, pages of 64 rows
-    "decode_fused_p64": (lambda: synth.custom([20000, 9000, 3000, 50000], [1] * 4, 64, 2048,
-                                              seed=200), 64),
+    # decode, fused tail (six rows): ragged lengths, pages of 64 rows
+    "decode_fused_p64": (lambda: synth.custom([20000, 9000, 3000, 50000, 15000, 8000], [1] * 6,
+                                              64, 2048, seed=200), 64),
+    # decode, separate selection and attention kernels (four rows), pages of 64
+    "decode_chain_p64": (lambda: synth.custom([20000, 9000, 3000, 50000], [1] * 4, 64, 2048,
+                                              seed=204), 64),
     # multi-token decode (items of 2 and 4 queries), pages of 256 rows
     "multi_token_p256": (lambda: synth.custom([12000, 30000], [2, 4], 64, 2048, seed=201), 256),
     # prefill-like rows: many-row attention, one-CTA-per-row selection, pages of 128

@@ -391,8 +391,9 @@ def _concentrated_batch():
     """Decode rows whose selected positions are not spread evenly: in row 0 the
     top scores sit in one contiguous range of 3000 positions (so a few chunks
     of the row hold hundreds of selected positions each, several 96-row tiles),
-    row 1 mixes that range with the rest, rows 2-3 are plain."""
-    wl = synth.custom([20000, 30000, 9000, 50000], [1] * 4, 64, 2048, seed=170)
+    row 1 mixes that range with the rest, rows 2-5 are plain.  Six rows: the
+    fused tail, which attends over balanced shares of such rows."""
+    wl = synth.custom([20000, 30000, 9000, 50000, 12000, 25000], [1] * 6, 64, 2048, seed=170)
     g = np.random.Generator(np.random.PCG64(171))
     v = g.standard_normal(128).astype(np.float32)
     v /= np.linalg.norm(v)
@@ -416,8 +417,14 @@ def test_layer_decode_concentrated_selection():
     assert ((sel >= 5000) & (sel < 8000)).sum() >= 1500
 
 
+def test_layer_decode_12_rows():
+    """12 decode rows: 12 chunks per row in the fused tail, so each CTA merges
+    683 output units, more than it has threads (two passes)."""
+    _layer_check(synth.custom([20000, 20000, 9000, 9000, 9000, 9000] + [30000] * 6, [1] * 12, 64,
+                              2048, seed=165))
+
+
 def test_layer_decode_14_rows():
-    """14 decode rows: 10 chunks per row in the fused tail, so each CTA merges
-    more output units than it has threads (several passes)."""
+    """14 decode rows: the separate selection, attention and merge kernels."""
     _layer_check(synth.custom([20000, 20000, 9000, 9000, 9000, 9000] + [30000] * 8, [1] * 14, 64,
                               2048, seed=165))
