@@ -14,7 +14,8 @@
 // S lands in TMEM with one head per lane, so each softmax thread owns one
 // head row: max, exp2 and row sum stay in registers.  P is written to shared
 // memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
-// 2^-16.  The gathered tile is stored once, in the 128-byte swizzled layout,
+// 2^-16, on rows with fewer than kHiOnlyRows selected; longer rows take the
+// hi part alone.  The gathered tile is stored once, in the 128-byte swizzled layout,
 // and read by both MMAs: K-major as the B operand of S, MN-major as the A
 // operand of O^T.  The running maximum is raised lazily (only when a tile's
 // maximum exceeds it by more than 2^8), and O^T in TMEM is then rescaled.
@@ -52,6 +53,12 @@ constexpr int kThreadsTc = 288;
 constexpr int kSoftThreads = 128;
 constexpr int kGroupThreads = 64;         // one gather group
 constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
+// Rows with at least this many selected slots take P as bf16 alone (no lo
+// part): the weights of so many keys are spread thin enough that their
+// rounding stays far inside the output tolerance (about 4e-4 at 1024 keys of
+// N(0,1) latents against 2e-3), and the row sum is taken over the rounded
+// values, so the weights still sum to one.
+constexpr int kHiOnlyRows = 1024;
 
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kBoxes * kQBox;
@@ -146,6 +153,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int slot_lo = sp * P.split_len;
   const int slot_hi = min(kMasked ? rs.len : n_slots, slot_lo + P.split_len);
   const int n_tiles = slot_hi > slot_lo ? (slot_hi - slot_lo + kT - 1) / kT : 0;
+  // The lo part of P only for rows with fewer than kHiOnlyRows selected.
+  const bool use_lo = min(P.top_k, rs.len) < kHiOnlyRows;
   if (kMasked) {
     // Bitmap of the chunk's positions that the index set lists.
     const int nwords = (P.split_len + 31) >> 5;
@@ -305,7 +314,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           const uint32_t d = tmem + kColO + 64u * blk;
           const uint64_t ko = static_cast<uint64_t>((kk * 32) >> 4);
           tc_mma_bf16_warp(d, a, dhi + ko, kIdescPV, (u > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_bf16_warp(d, a, dlo + ko, kIdescPV, 1u);
+          if (use_lo) tc_mma_bf16_warp(d, a, dlo + ko, kIdescPV, 1u);
         }
       }
       tc_commit_warp(b_kvempty(st));
@@ -379,7 +388,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const bool owner = lane < 16;                // owns head row 16q + lane
     const int hl = 16 * q + (lane & 15);
-    float m_run = -INFINITY, l_run = 0.f;
+    // l_run: the row sum (log-sum-exp, merge); lh_run: the sum of the weights
+    // the product used (the same with the lo part; the rounded hi parts
+    // without it), which normalises the output.
+    float m_run = -INFINITY, l_run = 0.f, lh_run = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int st = t & 1;
@@ -418,7 +430,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const float m_new = raise ? tmax : m_run;
       const float alpha = raise ? exp2_fast(m_run - m_new) : 1.f;
       const float m_ref = m_new == -INFINITY ? 0.f : m_new;  // masked logits give 2^-inf = 0
-      float sum = 0.f;
+      float sum = 0.f, sumh = 0.f;
       uint32_t hi[kSplitCols / 2], lo[kSplitCols / 2];
 #pragma unroll
       for (int k = 0; k < kSplitCols; k += 2) {
@@ -427,10 +439,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         sum += p0 + p1;
         const uint32_t h2 = pack2_bf16(p0, p1);
         hi[k / 2] = h2;
-        lo[k / 2] = pack2_bf16(p0 - __uint_as_float(h2 << 16), p1 - __uint_as_float(h2 & 0xFFFF0000u));
+        const float r0 = __uint_as_float(h2 << 16), r1 = __uint_as_float(h2 & 0xFFFF0000u);
+        if (use_lo) {
+          lo[k / 2] = pack2_bf16(p0 - r0, p1 - r1);
+        } else {
+          sumh += r0 + r1;  // the weights the product uses
+        }
       }
       sum += __shfl_xor_sync(0xffffffffu, sum, 16);
+      sumh += __shfl_xor_sync(0xffffffffu, sumh, 16);
       l_run = l_run * alpha + sum;
+      lh_run = lh_run * alpha + (use_lo ? sum : sumh);
       m_run = m_new;
       if (owner) alpha_s[hl] = alpha;
       // P buffer `st` is free once the P.V of tile t-2 has completed.
@@ -446,9 +465,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_hi + off),
                        "r"(hi[4 * j]), "r"(hi[4 * j + 1]), "r"(hi[4 * j + 2]), "r"(hi[4 * j + 3])
                        : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_lo + off),
-                       "r"(lo[4 * j]), "r"(lo[4 * j + 1]), "r"(lo[4 * j + 2]), "r"(lo[4 * j + 3])
-                       : "memory");
+          if (use_lo) {
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(prow_lo + off),
+                         "r"(lo[4 * j]), "r"(lo[4 * j + 1]), "r"(lo[4 * j + 2]), "r"(lo[4 * j + 3])
+                         : "memory");
+          }
         }
       }
       fence_proxy_async_smem();
@@ -479,7 +500,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_arrive(b_pfull(st));
     }
     // ------------------------------------------------------------ output --
-    if (owner) rl_s[hl] = l_run > 0.f ? 1.f / l_run : 0.f;
+    // Per head: 1 / lh for a finished row; for a slice, lh -> l, so that the
+    // merge's exact sums normalise it.
+    if (owner) {
+      rl_s[hl] = !(lh_run > 0.f) ? 0.f : (P.n_split > 1 ? l_run / lh_run : 1.f / lh_run);
+    }
     named_bar_sync(1, kSoftThreads);
     if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
     tc_fence_after();
@@ -515,7 +540,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           for (int j = 0; j < 32; ++j) {
             const int hh = 32 * half + j;
             float v = __uint_as_float(o[j]);
-            if (!split) v *= rl_s[hh];
+            if (!split || !use_lo) v *= rl_s[hh];
             stg[hh * kValue + dv] = v;
           }
         }

@@ -158,6 +158,9 @@ ATTN = {
     # runs with slices of the selected set and the merge
     "decode_12rows_split": lambda: synth.custom([2200 + 150 * i for i in range(12)], [1] * 12, 64,
                                                 2048, seed=116),
+    # 48 query rows of 2048 selected each: P without its lo part, split over
+    # CTAs and merged
+    "long_rows_hi_only": lambda: synth.custom([3000], [48], 64, 2048, seed=117),
 }
 
 
