@@ -1030,6 +1030,30 @@ def cpu_baseline(wl):
                       f"{dt:.1f} s)"}
 
 
+def profile_layer(spec, calls):
+    """Runs dsa_layer_forward on one synthetic workload `calls` times, each
+    after an L2 flush, checks the device status and exits (no timing: a
+    driver for ncu, whose own launch list and counters are the output)."""
+    from dsa_lightning_indexer_b200 import binding as bd
+    kind, *dims = spec.split(",")
+    if kind == "decode":
+        wl = synth.decode(int(dims[0]), int(dims[1]), 64, 2048, seed=3)
+    elif kind == "prefill":
+        wl = synth.prefill(int(dims[0]), 64, 2048, seed=2, planted=True)
+    else:
+        raise SystemExit(f"--profile-layer: unknown workload {spec!r}")
+    dw = bd.DeviceWorkload(wl)
+    out, lse, idx = dw.new_outputs()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 2x the L2
+    for i in range(calls):
+        flush.fill_(i & 0xFF)
+        dw.forward(out, lse, idx)
+    torch.cuda.synchronize()
+    bd.check_device_status(dw.ws)
+    print(f"profile-layer {wl.name}: {calls} calls ok", flush=True)
+    return 0
+
+
 def main():
     faulthandler.enable()
     ap = argparse.ArgumentParser(description=__doc__)
@@ -1053,7 +1077,13 @@ def main():
                     help="rotating copies of the decode inputs (L2 defeat)")
     ap.add_argument("--dry-run", action="store_true",
                     help="check the multi-rank launch path without a GPU (gloo)")
+    ap.add_argument("--profile-layer", default=None, metavar="SPEC",
+                    help="profiling aid: 'decode,B,L' or 'prefill,T' -- run the layer "
+                         "--profile-calls times (L2 flushed before each) and exit")
+    ap.add_argument("--profile-calls", type=int, default=3)
     args = ap.parse_args()
+    if args.profile_layer:
+        return profile_layer(args.profile_layer, args.profile_calls)
     _, _, world = env_rank()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         # One process per GPU: run this script again as --gpus ranks.
