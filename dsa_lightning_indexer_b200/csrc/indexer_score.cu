@@ -67,7 +67,11 @@ struct Cfg {
   static constexpr int N = 32 * QT;
   // Epilogue sets: with 4 or 8 queries per item the read-out of a tile takes
   // longer than its MMAs, so two or four sets of four warps split the queries.
-  static constexpr int kEpiSets = QT >= 8 ? 4 : (QT >= 4 ? 2 : 1);
+  // With one query per item two sets take alternate tiles (set s reads
+  // accumulator s), so the read-out, score store and histogram count of a
+  // tile overlap the next one's.
+  static constexpr bool kSplitTiles = QT == 1;
+  static constexpr int kEpiSets = QT >= 8 ? 4 : (QT >= 4 ? 2 : (kSplitTiles ? 2 : 1));
   static constexpr int kThreads = 64 + kEpiSets * kEpiThreads;
   static constexpr int kQBufs = QT <= 4 ? 2 : 1;
   // K ring depth: deep for decode (HBM streaming), shallower when Q is large.
@@ -110,6 +114,20 @@ __device__ __forceinline__ bool decode_item(const IdxParams& P, int item, ItemVi
 
 __device__ __forceinline__ void named_bar_sync_idx(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Named barrier over `threads` threads; true if `pred` held in any of them.
+__device__ __forceinline__ bool named_bar_any(int id, int threads, bool pred) {
+  uint32_t res;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(res)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
+      : "memory");
+  return res != 0u;
 }
 
 __device__ __forceinline__ int snake_item(int j) {
@@ -156,7 +174,7 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       mbar_init(qfull(i), 1);
       mbar_init(qempty(i), 1);
       mbar_init(tfull(i), 1);
-      mbar_init(tempty(i), C::kEpiSets * kEpiThreads);
+      mbar_init(tempty(i), C::kSplitTiles ? kEpiThreads : C::kEpiSets * kEpiThreads);
     }
     mbar_init(drain, 1);
     fence_mbar_init();
@@ -310,13 +328,14 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
     // --------------------------------------------------------- epilogue --
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const int et = static_cast<int>(threadIdx.x) - 64;  // 0..127 in the first set
+    const int et = static_cast<int>(threadIdx.x) - 64;  // 0.. over all epilogue sets
     const int jset = (warp - 2) >> 2;                    // this warp's epilogue set
+    constexpr int kAllEpi = C::kEpiSets * kEpiThreads;
     const bool do_hist = (QT == 1) && P.hist != nullptr;     // shared-memory histogram
     const bool do_ghist = (QT > 1) && P.hist != nullptr;     // straight to the row's
     if (do_hist) {
-      for (int i = et; i < kHistBins; i += kEpiThreads) shist[i] = 0;
-      named_bar_sync_idx(1, kEpiThreads);
+      for (int i = et; i < kHistBins; i += kAllEpi) shist[i] = 0;
+      named_bar_sync_idx(1, kAllEpi);
     }
     int acc = 0;
     uint32_t aph = 0;
@@ -327,12 +346,17 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
       ItemView v;
       if (!decode_item<QT>(P, item, v)) continue;
       for (int kt = v.kt0; kt < v.kt1; ++kt) {
+        if (C::kSplitTiles && acc != jset) {  // the other set's tile
+          acc ^= 1;
+          if (acc == 0) aph ^= 1u;
+          continue;
+        }
         ok = mbar_wait(tfull(acc), aph, P.err);
         if (!ok) break;
         tc_fence_after();
         const int key = kt * kKeysPerTile + quad * 32 + lane;
 #pragma unroll 1
-        for (int jq = jset; jq < QT; jq += C::kEpiSets) {
+        for (int jq = C::kSplitTiles ? 0 : jset; jq < QT; jq += C::kSplitTiles ? 1 : C::kEpiSets) {
           if (jq >= v.nrow) break;
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem + lane_base + static_cast<uint32_t>(acc * C::N + jq * 32), r);
@@ -371,16 +395,20 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
         if (acc == 0) aph ^= 1u;
       }
       if (do_hist) {  // flush this item's counts into the row's histogram
-        named_bar_sync_idx(1, kEpiThreads);
-        int* const gh = P.hist + static_cast<size_t>(v.row0) * kHistBins;
-        for (int i = et; i < kHistBins; i += kEpiThreads) {
-          const int c = shist[i];
-          if (c != 0) {
-            atomicAdd(gh + i, c);
-            shist[i] = 0;
+        // Every set has counted its tiles of the item; a wait that ran out
+        // in either set ends both (they meet at every barrier below).
+        ok = !named_bar_any(1, kAllEpi, !ok);
+        if (ok) {
+          int* const gh = P.hist + static_cast<size_t>(v.row0) * kHistBins;
+          for (int i = et; i < kHistBins; i += kAllEpi) {
+            const int c = shist[i];
+            if (c != 0) {
+              atomicAdd(gh + i, c);
+              shist[i] = 0;
+            }
           }
         }
-        named_bar_sync_idx(1, kEpiThreads);
+        named_bar_sync_idx(1, kAllEpi);
       }
     }
   }
