@@ -43,6 +43,38 @@ cudaError_t prefer_max_shared(const void* kernel) {
   return e;
 }
 
+namespace {
+
+// Zeroes `words` 32-bit words at `p` as a programmatic dependent launch: it
+// waits for the kernels before it (they may still read the region) and lets
+// the next kernel's CTAs start their set-up at once.  A memset node in the
+// stream instead makes the next kernel wait for it to finish before its
+// launch begins.
+__global__ void __launch_bounds__(256) zero_words_kernel(uint32_t* p, size_t words) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const size_t n4 = words / 4;
+  uint4* const p4 = reinterpret_cast<uint4*>(p);
+  for (size_t i = blockIdx.x * 256 + threadIdx.x; i < n4; i += static_cast<size_t>(gridDim.x) * 256) {
+    p4[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (size_t i = n4 * 4 + blockIdx.x * 256 + threadIdx.x; i < words;
+       i += static_cast<size_t>(gridDim.x) * 256) {
+    p[i] = 0u;
+  }
+}
+
+// `bytes` (a multiple of 4) at the 16-byte aligned `p`.
+cudaError_t zero_async(void* p, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return cudaSuccess;
+  const size_t words = bytes / 4;
+  const unsigned grid = static_cast<unsigned>(std::min<size_t>((words / 4 + 255) / 256 + 1, 148));
+  return launch_pdl(zero_words_kernel, dim3(grid), dim3(256), 0, st, 0,
+                    static_cast<uint32_t*>(p), words);
+}
+
+}  // namespace
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 dsa_status check_batch(const dsa_batch* b, BatchInfo* info) {
@@ -320,7 +352,7 @@ dsa_status dsa_indexer_score(const dsa_batch* batch, const uint16_t* q_idx, cons
   IndexerArgs ia = indexer_args(batch, info, q_idx, w, k_idx, scores, ld_scores, ws, sms);
   if (hist) {
     void* const region = static_cast<uint8_t*>(ws) + kControlBytes;
-    DSA_TRY(cuda_status(cudaMemsetAsync(region, 0, topk_hist_zero_bytes(batch->Nq), st)));
+    DSA_TRY(cuda_status(zero_async(region, topk_hist_zero_bytes(batch->Nq), st)));
     ia.hist = static_cast<int*>(region);
   }
   return cuda_status(launch_indexer_score(ia, st));
@@ -350,8 +382,8 @@ dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld_scor
   // the histograms: clear those, so the same histograms serve every call.
   uint8_t* const region = static_cast<uint8_t*>(ws) + kControlBytes;
   const size_t hist_bytes = static_cast<size_t>(batch->Nq) * kHistBins * sizeof(int);
-  DSA_TRY(cuda_status(cudaMemsetAsync(region + hist_bytes, 0,
-                                      topk_hist_zero_bytes(batch->Nq) - hist_bytes, st)));
+  DSA_TRY(cuda_status(zero_async(region + hist_bytes,
+                                 topk_hist_zero_bytes(batch->Nq) - hist_bytes, st)));
   return cuda_status(launch_topk_hist(a, region, st));
 }
 
@@ -471,8 +503,8 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   if (L.hist_topk) {
     // The histograms and counters start from zero on every call: no state is
     // carried in the workspace from one call to the next.
-    DSA_TRY(cuda_status(cudaMemsetAsync(
-        hist_region, 0,
+    DSA_TRY(cuda_status(zero_async(
+        hist_region,
         L.fused_tail ? decode_tail_zero_bytes(batch->Nq) : topk_hist_zero_bytes(batch->Nq), st)));
     ia.hist = static_cast<int*>(hist_region);
   }
@@ -578,8 +610,8 @@ dsa_status dsa_indexer_project(const dsa_batch* batch, const uint16_t* x, int64_
   a.err = err_word(ws);
   a.num_sms = kPlanSms;
   // The split-K tickets start from zero on every call.
-  DSA_TRY(cuda_status(cudaMemsetAsync(a.ws_region, 0,
-                                      project_zero_bytes(a.T, a.d_q, a.d_model, kPlanSms), st)));
+  DSA_TRY(cuda_status(zero_async(a.ws_region,
+                                 project_zero_bytes(a.T, a.d_q, a.d_model, kPlanSms), st)));
   return cuda_status(launch_indexer_project(a, st));
 }
 
