@@ -272,13 +272,14 @@ def indexer_causal_flops(wl):
 
 
 def launches_per_layer(wl, sms=148):
-    """Kernels one dsa_layer_forward launches: the indexer (one launch per 64
-    sequences with queries), then either the fused decode tail (selection,
-    attention and merge in one kernel: 6 to 12 long rows, at most 64 heads),
-    or the top-k selection -- two kernels (filter and emit) when the
-    indexer's histograms drive it, else one -- followed by the sparse
-    attention and, when few rows split the selected set over CTAs, the merge
-    of the slices."""
+    """Kernels one dsa_layer_forward launches: when the indexer builds score
+    histograms, first the kernel that zeroes their region; the indexer (one
+    launch per 64 sequences with queries); then either the fused decode tail
+    (selection, attention and merge in one kernel: 6 to 12 long rows, at most
+    64 heads), or the selection -- the tail kernel's selection alone for 13 to
+    16 long rows, two kernels (filter and emit) for other histogram-driven
+    rows, else one -- followed by the sparse attention and, when few rows
+    split the selected set over CTAs, the merge of the slices."""
     nq = np.diff(wl.q_offsets)
     seqs = int((nq > 0).sum())
     max_len = int(wl.ctx_lens.max()) if wl.B else 0
@@ -288,12 +289,15 @@ def launches_per_layer(wl, sms=148):
     hist = (0 < wl.Nq <= 148 and max_len >= 8192 and max_len >= 4 * wl.top_k
             and -(-max_len // chunk) <= 512)
     C = 148 // max(1, wl.Nq)
-    fused = (hist and wl.H <= 64 and 6 <= wl.Nq <= 12 and C >= 8
-             and (-(-max_len // C) + 31) // 32 <= 512)
+    tail_fits = (0 < wl.Nq <= 16 and C >= 8 and (-(-max_len // C) + 31) // 32 <= 512)
+    fused = hist and wl.H <= 64 and 6 <= wl.Nq <= 12 and tail_fits
+    indexer = (seqs + 63) // 64 + (1 if hist else 0)
     if fused:
-        return (seqs + 63) // 64 + 1
+        return indexer + 1
+    select_tail = hist and wl.Nq > 12 and tail_fits
     few_rows = wl.Nq * ((wl.H + 63) // 64) < sms
-    return (seqs + 63) // 64 + (2 if hist else 1) + 1 + (1 if few_rows and wl.top_k > 16 else 0)
+    selection = 1 if select_tail else (2 if hist else 1)
+    return indexer + selection + 1 + (1 if few_rows and wl.top_k > 16 else 0)
 
 
 def profiled_traffic(profile="profiles/decode_b4_128k_layer.md"):

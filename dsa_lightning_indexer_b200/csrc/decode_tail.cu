@@ -120,6 +120,7 @@ struct TailParams {
   unsigned* err;
   int B, Nq, H, top_k, C;
   float scale_log2;
+  int select_only;  // stop after writing the index sets (the attention runs separately)
 };
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   // The queries and the batch arrays are inputs of the layer, final before
   // the indexer ran: load and look them up while the indexer finishes.
-  if (warp == 4 && lane == 0) {
+  if (warp == 4 && lane == 0 && !P.select_only) {
     tma_prefetch_map(&qmap);
     mbar_arrive_expect_tx(b_qfull, kBoxes * kQBox);
     const uint64_t pol = l2_policy_evict_first();
@@ -507,6 +508,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
+  // Selection only: the index sets are written; phases C and D are skipped
+  // (the rows that phase A started bringing into L2 serve the attention).
+  if (P.select_only) ok = false;
   // The row's index set is complete once every CTA of the row has written its
   // part (rows that keep every position need no wait: slot i holds i).
   if (ok && !full && !own && tid == 0) {
@@ -852,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_commit_warp(b_drain);
     if (lane == 0) {
       mbar_drain(b_drain, 0, P.err);
-      mbar_drain(b_qfull, 0, P.err);
+      if (!P.select_only) mbar_drain(b_qfull, 0, P.err);
     }
     __syncwarp();
   }
@@ -867,6 +871,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 int decode_tail_chunks(int Nq, int num_sms) { return std::max(1, num_sms / std::max(1, Nq)); }
+
+bool decode_tail_fits(int Nq, int64_t max_len, int num_sms) {
+  const int C = decode_tail_chunks(Nq, num_sms);
+  return Nq > 0 && Nq <= 16 && C >= 8 &&
+         ((max_len + C - 1) / C + 31) / 32 <= kMaxWords;
+}
 
 bool decode_tail_supported(int Nq, int H, int64_t max_len, int num_sms) {
   const int C = decode_tail_chunks(Nq, num_sms);
@@ -942,6 +952,7 @@ cudaError_t launch_decode_tail(const DecodeTailArgs& a, cudaStream_t stream) {
   P.top_k = a.top_k;
   P.C = C;
   P.scale_log2 = a.scale * kLog2e;
+  P.select_only = a.select_only ? 1 : 0;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.Nq * C));

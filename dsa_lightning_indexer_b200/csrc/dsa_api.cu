@@ -189,6 +189,7 @@ struct WsLayout {
   int64_t ld;
   bool hist_topk;   // selection driven by histograms the indexer builds
   bool fused_tail;  // ... and everything after the indexer in one kernel
+  bool select_tail; // ... or the selection in that kernel, the attention after it
   AttnPlan plan;
 };
 
@@ -223,9 +224,14 @@ WsLayout plan_ws(const dsa_batch* b, const BatchInfo& info, int H, int top_k, bo
   w.scores_bytes = scores ? round_up(static_cast<size_t>(b->Nq) * w.ld * sizeof(float), 256) : 0;
   w.hist_topk = scores && plan_hist_topk(b, info, top_k);
   w.fused_tail = w.hist_topk && attn && decode_tail_supported(b->Nq, H, info.max_len, kPlanSms);
+  // The tail's selection alone (then the separate attention) measured faster
+  // than the filter and emit kernels for 13 to 16 rows, and no faster for 5
+  // or fewer.
+  w.select_tail = w.hist_topk && attn && !w.fused_tail && b->Nq > 12 &&
+                  decode_tail_fits(b->Nq, info.max_len, kPlanSms);
   w.hist_off = w.scores_off + w.scores_bytes;
   w.hist_bytes =
-      w.fused_tail
+      (w.fused_tail || w.select_tail)
           ? round_up(decode_tail_ws_bytes(b->Nq, decode_tail_chunks(b->Nq, kPlanSms)), 256)
           : (w.hist_topk ? round_up(topk_hist_ws_bytes(b->Nq, top_k, info.max_len), 256) : 0);
   w.part_off = w.hist_off + w.hist_bytes;
@@ -503,13 +509,15 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
   if (L.hist_topk) {
     // The histograms and counters start from zero on every call: no state is
     // carried in the workspace from one call to the next.
-    DSA_TRY(cuda_status(zero_async(
-        hist_region,
-        L.fused_tail ? decode_tail_zero_bytes(batch->Nq) : topk_hist_zero_bytes(batch->Nq), st)));
+    DSA_TRY(cuda_status(zero_async(hist_region,
+                                   (L.fused_tail || L.select_tail)
+                                       ? decode_tail_zero_bytes(batch->Nq)
+                                       : topk_hist_zero_bytes(batch->Nq),
+                                   st)));
     ia.hist = static_cast<int*>(hist_region);
   }
   DSA_TRY(cuda_status(launch_indexer_score(ia, st)));
-  if (L.fused_tail) {
+  if (L.fused_tail || L.select_tail) {
     DecodeTailArgs d;
     d.B = batch->B;
     d.Nq = batch->Nq;
@@ -529,11 +537,14 @@ dsa_status dsa_layer_forward(const dsa_batch* batch, const uint16_t* q, int H,
     d.err = err_word(ws);
     d.scale = scale;
     d.num_sms = std::min(sms, kPlanSms);  // the workspace holds kPlanSms / Nq chunks
-    return cuda_status(launch_decode_tail(d, st));
+    d.select_only = L.select_tail;
+    DSA_TRY(cuda_status(launch_decode_tail(d, st)));
+    if (L.fused_tail) return DSA_OK;
+  } else {
+    const TopkArgs t = topk_args(batch, info, scores, L.ld, top_k, idx, ws, sms);
+    DSA_TRY(
+        cuda_status(L.hist_topk ? launch_topk_hist(t, hist_region, st) : launch_topk(t, st)));
   }
-
-  const TopkArgs t = topk_args(batch, info, scores, L.ld, top_k, idx, ws, sms);
-  DSA_TRY(cuda_status(L.hist_topk ? launch_topk_hist(t, hist_region, st) : launch_topk(t, st)));
 
   AttnArgs a;
   a.B = batch->B;

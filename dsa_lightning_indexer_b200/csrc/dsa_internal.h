@@ -97,8 +97,12 @@ struct DecodeTailArgs {
   unsigned* err;
   float scale;
   int num_sms;       // SMs the launch may fill (one CTA per SM)
+  bool select_only;  // write the index sets only (q, kv, out, lse unused)
 };
 int decode_tail_chunks(int Nq, int num_sms);
+// The kernel's limits (rows, chunks, chunk length), for either mode.
+bool decode_tail_fits(int Nq, int64_t max_len, int num_sms);
+// Where the whole fused tail is the faster route.
 bool decode_tail_supported(int Nq, int H, int64_t max_len, int num_sms);
 size_t decode_tail_zero_bytes(int Nq);
 size_t decode_tail_ws_bytes(int Nq, int C);

@@ -53,14 +53,17 @@ def test_prefill_16k_indexer_flops():
 
 
 def test_kernels_per_layer_call():
-    # decode 8 x 32K: indexer, then the fused tail (selection, attention, merge)
-    assert bench.launches_per_layer(_layout([32768] * 8, [1] * 8, 64, 2048)) == 2
-    # decode 4 x 128K: indexer, top-k filter + emit, attention, merge of the slices
-    assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 64, 2048)) == 5
-    # 32 ragged decode rows: indexer, top-k filter + emit, attention, merge of the slices
-    assert bench.launches_per_layer(_layout([40000] * 32, [1] * 32, 64, 2048)) == 5
+    # decode 8 x 32K: histogram zeroing, indexer, the fused tail (selection,
+    # attention, merge)
+    assert bench.launches_per_layer(_layout([32768] * 8, [1] * 8, 64, 2048)) == 3
+    # decode 4 x 128K: zeroing, indexer, top-k filter + emit, attention, merge of the slices
+    assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 64, 2048)) == 6
+    # decode 14 x 32K: zeroing, indexer, the tail's selection, attention, merge
+    assert bench.launches_per_layer(_layout([32768] * 14, [1] * 14, 64, 2048)) == 5
+    # 32 ragged decode rows: zeroing, indexer, filter + emit, attention, merge of the slices
+    assert bench.launches_per_layer(_layout([40000] * 32, [1] * 32, 64, 2048)) == 6
     # more than 64 heads: no fused tail
-    assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 128, 2048)) == 5
+    assert bench.launches_per_layer(_layout([131072] * 4, [1] * 4, 128, 2048)) == 6
     # prefill 16K: indexer, one top-k kernel, attention
     assert bench.launches_per_layer(_layout([16384], [16384], 64, 2048)) == 3
 
