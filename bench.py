@@ -1040,6 +1040,31 @@ def profile_layer(spec, calls):
     driver for ncu, whose own launch list and counters are the output)."""
     from dsa_lightning_indexer_b200 import binding as bd
     kind, *dims = spec.split(",")
+    if kind == "project":  # the indexer's input step on T new tokens (one per sequence)
+        T = int(dims[0])
+        dev = torch.device("cuda")
+        g = torch.Generator(device=dev)
+        g.manual_seed(7)
+
+        def bf(*shape, std=1.0):
+            return (torch.randn(*shape, generator=g, device=dev) * std).to(torch.bfloat16)
+        lens = [131072] * T
+        kv_off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        b = bd.Batch(np.arange(T + 1, dtype=np.int32), kv_off, np.array(lens, np.int32), dev)
+        args = (b, bf(T, D_MODEL), bf(T, D_Q), bf(4096, D_Q, std=D_Q ** -0.5),
+                bf(128, D_MODEL, std=D_MODEL ** -0.5), bf(32, D_MODEL, std=D_MODEL ** -0.5),
+                torch.empty(T, 32, 128, dtype=torch.bfloat16, device=dev),
+                torch.zeros(int(kv_off[-1]), 128, dtype=torch.bfloat16, device=dev),
+                torch.empty(T, 32, device=dev))
+        ws = bd.indexer_project_workspace(b, D_MODEL, D_Q, dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 2x the L2
+        for i in range(calls):
+            flush.fill_(i & 0xFF)
+            bd.indexer_project(*args, ws)
+        torch.cuda.synchronize()
+        bd.check_device_status(ws)
+        print(f"profile-layer input step, {T} tokens: {calls} calls ok", flush=True)
+        return 0
     if kind == "decode":
         wl = synth.decode(int(dims[0]), int(dims[1]), 64, 2048, seed=3)
     elif kind == "prefill":
@@ -1082,8 +1107,9 @@ def main():
     ap.add_argument("--dry-run", action="store_true",
                     help="check the multi-rank launch path without a GPU (gloo)")
     ap.add_argument("--profile-layer", default=None, metavar="SPEC",
-                    help="profiling aid: 'decode,B,L' or 'prefill,T' -- run the layer "
-                         "--profile-calls times (L2 flushed before each) and exit")
+                    help="profiling aid: 'decode,B,L', 'prefill,T' or 'project,T' -- run "
+                         "the layer (or the indexer's input step) --profile-calls times "
+                         "(L2 flushed before each) and exit")
     ap.add_argument("--profile-calls", type=int, default=3)
     args = ap.parse_args()
     if args.profile_layer:

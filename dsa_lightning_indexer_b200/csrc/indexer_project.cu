@@ -336,15 +336,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            for (int sl = 0; sl < it.nslice; ++sl) {
-              const float* src = part_at(sl, c0);
+            // Eight slices' loads in flight at a time, added in slice order.
+            constexpr int kBatch = 8;
+#pragma unroll 1
+            for (int sl0 = 0; sl0 < it.nslice; sl0 += kBatch) {
+              float4 x[kBatch][4];
 #pragma unroll
-              for (int j = 0; j < 16; j += 4) {
-                const float4 x4 = __ldcg(reinterpret_cast<const float4*>(src + j));
-                v[j] += x4.x;
-                v[j + 1] += x4.y;
-                v[j + 2] += x4.z;
-                v[j + 3] += x4.w;
+              for (int a = 0; a < kBatch; ++a) {
+                const bool in = sl0 + a < it.nslice;
+                const float* src = part_at(in ? sl0 + a : 0, c0);
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  x[a][b] = in ? __ldcg(reinterpret_cast<const float4*>(src + 4 * b))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+              }
+#pragma unroll
+              for (int a = 0; a < kBatch; ++a) {
+                if (sl0 + a < it.nslice) {
+#pragma unroll
+                  for (int b = 0; b < 4; ++b) {
+                    v[4 * b] += x[a][b].x;
+                    v[4 * b + 1] += x[a][b].y;
+                    v[4 * b + 2] += x[a][b].z;
+                    v[4 * b + 3] += x[a][b].w;
+                  }
+                }
               }
             }
             emit16(c0, v);
@@ -406,15 +423,32 @@ void plan_project(int T, int d_q, int d_model, int num_sms, int* N, int* ksq, in
   *N = n;
   const int ttiles = (T + n - 1) / n;
   const int kq = d_q / kKStep, kx = d_model / kKStep;
-  // Split the K range until about two items per SM, slices of at least 4 steps.
   *ksq = 1;
   *ksx = 1;
-  while ((kTileQ * *ksq + 2 * *ksx) * ttiles < 2 * num_sms) {
-    const bool more_q = kq / (*ksq * 2) >= 4;
-    const bool more_x = kx / (*ksx * 2) >= 4;
-    if (!more_q && !more_x) break;
-    if (more_q) *ksq *= 2;
-    if (more_x && (kx / *ksx) > (kq / *ksq)) *ksx *= 2;
+  if ((kTileQ + 2) * ttiles >= num_sms) return;  // whole K ranges already fill the GPU
+  // Few tokens: split the K ranges so that the items fit one wave of the SMs
+  // and the longest slice (the weight bytes one SM streams) is as short as
+  // possible; among equal longest slices, fewer slices (a shorter sum).
+  int best = 1 << 30, best_items = 1 << 30;
+  for (int q = 1; q <= kq; ++q) {
+    const int left = num_sms / ttiles - kTileQ * q;
+    if (left < 2) break;
+    const int x = std::min(kx, left / 2);
+    const int qs = (kq + q - 1) / q;
+    int xs = (kx + x - 1) / x;
+    int xx = x;
+    while (xx > 1 && (kx + xx - 2) / (xx - 1) <= std::max(qs, xs)) {  // no longer a longer slice
+      --xx;
+    }
+    xs = (kx + xx - 1) / xx;
+    const int cost = std::max(qs, xs);
+    const int items = kTileQ * q + 2 * xx;
+    if (cost < best || (cost == best && items < best_items)) {
+      best = cost;
+      best_items = items;
+      *ksq = q;
+      *ksx = xx;
+    }
   }
 }
 
