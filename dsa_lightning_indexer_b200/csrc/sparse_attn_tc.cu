@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (gt < kT) gidx[gt] = row_cur;
       named_bar_sync(2 + grp, kGroupThreads);
       row_cur = row_nxt;
-      row_nxt = load_row(t + 4);
       const uint32_t stage = sKV + grp * kKVStage;
       // Thread (sub, piece) copies 16-byte piece `piece` of every box of
       // rows sub, sub + 8, ...: a warp instruction reads four whole 128-byte
@@ -274,7 +273,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           }
         }
       }
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      // The slot two tiles ahead is looked up while this tile's copies are in
+      // flight (its bounds check branches on the loaded entry).
+      row_nxt = load_row(t + 4);
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
       fence_proxy_async_smem();
       mbar_arrive(b_kvfull(grp));
     }
