@@ -182,6 +182,19 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&kmap);
     tma_prefetch_map(&qmap);
+    // The key tiles of this CTA's first item start coming into L2 while the
+    // kernel before this one finishes (a prefetch reads the current data and
+    // writes nothing, so it is safe before the dependent-launch wait).
+    ItemView v0;
+    const int item0 = snake_item(0);
+    if (!P.stall && P.cache.block_table == nullptr && item0 < P.n_items &&
+        decode_item<QT>(P, item0, v0)) {
+      for (int kt = v0.kt0; kt < min(v0.kt1, v0.kt0 + C::kStages + 2); ++kt) {
+        const int row = static_cast<int>(v0.kv0 + static_cast<long long>(kt) * kKeysPerTile);
+        tma_prefetch_2d(&kmap, 0, row);
+        tma_prefetch_2d(&kmap, 64, row);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
