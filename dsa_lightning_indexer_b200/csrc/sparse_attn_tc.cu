@@ -8,9 +8,9 @@
 // leading 512 entries serve as V.)
 //
 // One CTA owns one query row and a block of 64 heads, and walks the row's
-// selected set in tiles of 48 gathered cache rows:
-//   S    = Q[64 heads, 576] . K_tile[48, 576]^T      M = 64,  N = 48, K = 576
-//   O^T += V_tile^T[512, 48] . P^T[48, 64 heads]     M = 128 (x4), N = 64, K = 48
+// selected set in tiles of 32 gathered cache rows:
+//   S    = Q[64 heads, 576] . K_tile[32, 576]^T      M = 64,  N = 32, K = 576
+//   O^T += V_tile^T[512, 32] . P^T[32, 64 heads]     M = 128 (x4), N = 64, K = 32
 // S lands in TMEM with one head per lane, so each softmax thread owns one
 // head row: max, exp2 and row sum stay in registers.  P is written to shared
 // memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
@@ -20,9 +20,13 @@
 // operand of O^T.  The running maximum is raised lazily (only when a tile's
 // maximum exceeds it by more than 2^8), and O^T in TMEM is then rescaled.
 //
-// Warp roles (288 threads): warps 0-3 softmax and output (TMEM quadrants
+// Warp roles (352 threads): warps 0-3 softmax and output (TMEM quadrants
 // 0-3), warp 4 TMEM allocation, the Q load (TMA) and single-thread MMA issue,
-// warps 5-6 and 7-8 gather even and odd tiles with 16-byte cp.async.
+// warps 5-6, 7-8 and 9-10 gather tiles t = 0, 1, 2 (mod 3) with 16-byte
+// cp.async into three stages.  A stage is busy from its gather until its
+// tile's P.V completes (gather, S, softmax, P.V in a chain), so three stages
+// of 32 rows keep more of that chain in flight than two of 48 in the same
+// shared memory.
 //
 // The same kernel, instantiated with kMasked, is the mask-over-the-whole-
 // cache route the pages describe for llama.cpp (aiaulis.com paragraph 4;
@@ -42,16 +46,18 @@ namespace {
 
 using namespace attn_tc;
 
-constexpr int kT = 48;                    // gathered rows per tile
+constexpr int kT = 32;                    // gathered rows per tile
+constexpr int kStages = 3;                // gather stages (and S buffers)
+constexpr int kPStages = 2;               // P buffers
 constexpr int kHB = 64;                   // heads per CTA
 constexpr int kBoxes = kLatent / 64;      // 64-dim column boxes of a latent row
 constexpr int kQBox = kHB * 128;          // bytes of one Q box
 constexpr int kKVBox = kT * 128;          // bytes of one gathered-tile box
 constexpr int kKVStage = kBoxes * kKVBox;
-constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 48 used)
-constexpr int kThreadsTc = 288;
+constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 32 used)
 constexpr int kSoftThreads = 128;
 constexpr int kGroupThreads = 64;         // one gather group
+constexpr int kThreadsTc = kSoftThreads + 32 + kStages * kGroupThreads;
 constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
 // Rows with at least this many selected slots take P as bf16 alone (no lo
 // part): the weights of so many keys are spread thin enough that their
@@ -63,12 +69,12 @@ constexpr int kHiOnlyRows = 1024;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kBoxes * kQBox;
 constexpr int kOffStage = kOffQ;  // output staging [64][512] fp32 over Q and the gather stages
-constexpr int kOffP = kOffKV + 2 * kKVStage;           // [stage][hi, lo]
-constexpr int kOffBar = kOffP + 4 * kPBuf;
-constexpr int kNumBars = 15;
+constexpr int kOffP = kOffKV + kStages * kKVStage;     // [P stage][hi, lo]
+constexpr int kOffBar = kOffP + 2 * kPStages * kPBuf;
+constexpr int kNumBars = 3 + 4 * kStages + 2 * kPStages;
 constexpr int kOffTmem = kOffBar + 8 * kNumBars;
-constexpr int kOffIdx = kOffTmem + 16;                  // [2][kT] int
-constexpr int kOffAlpha = kOffIdx + 2 * kT * 4;         // [64] float
+constexpr int kOffIdx = kOffTmem + 16;                  // [kStages][kT] int
+constexpr int kOffAlpha = kOffIdx + kStages * kT * 4;   // [64] float
 constexpr int kOffM = kOffAlpha + kHB * 4;              // [64] float
 constexpr int kOffL = kOffM + kHB * 4;                  // [64] float
 constexpr int kOffMask = kOffL + kHB * 4;               // masked route: chunk bitmap
@@ -79,14 +85,14 @@ static_assert(kOffStage + kHB * kValue * 4 <= kOffP, "output staging overlaps th
 static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S buffers at columns 0 and 64 (M = 64 layout)
+constexpr uint32_t kColS = 0;     // S buffers at columns 0, 32, 64 (M = 64 layout)
 constexpr uint32_t kColO = 128;   // O^T blocks at 128, 192, 256, 320
 
 // kind::f16 instruction descriptors (bf16 in, fp32 accumulate).
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, kT);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
-constexpr int kSplitCols = kT / 2;  // logits per half warp (16 + 8 columns)
-static_assert(kSplitCols == 24, "the logit loads cover 16 + 8 columns per half warp");
+constexpr int kSplitCols = kT / 2;  // logits per half warp
+static_assert(kSplitCols == 16, "one 16-column load per half warp covers its logits");
 
 template <bool kMasked>
 __global__ void __launch_bounds__(kThreadsTc, 1)
@@ -100,13 +106,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t bars = base + kOffBar;
   const uint32_t b_qfull = bars;
   auto b_kvfull = [&](int s) { return bars + 8u * (1 + s); };
-  auto b_kvempty = [&](int s) { return bars + 8u * (3 + s); };
-  auto b_sfull = [&](int s) { return bars + 8u * (5 + s); };
-  auto b_sempty = [&](int s) { return bars + 8u * (7 + s); };
-  auto b_pfull = [&](int s) { return bars + 8u * (9 + s); };
-  auto b_pempty = [&](int s) { return bars + 8u * (11 + s); };
-  const uint32_t b_odone = bars + 8u * 13;
-  const uint32_t b_drain = bars + 8u * 14;
+  auto b_kvempty = [&](int s) { return bars + 8u * (1 + kStages + s); };
+  auto b_sfull = [&](int s) { return bars + 8u * (1 + 2 * kStages + s); };
+  auto b_sempty = [&](int s) { return bars + 8u * (1 + 3 * kStages + s); };
+  auto b_pfull = [&](int s) { return bars + 8u * (1 + 4 * kStages + s); };
+  auto b_pempty = [&](int s) { return bars + 8u * (1 + 4 * kStages + kPStages + s); };
+  const uint32_t b_odone = bars + 8u * (1 + 4 * kStages + 2 * kPStages);
+  const uint32_t b_drain = b_odone + 8u;
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
@@ -121,11 +127,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(b_kvfull(s), kMasked ? 1 : kGroupThreads);
       mbar_init(b_kvempty(s), 1);
       mbar_init(b_sfull(s), 1);
       mbar_init(b_sempty(s), kSoftThreads);
+    }
+    for (int s = 0; s < kPStages; ++s) {
       mbar_init(b_pfull(s), kSoftThreads);
       mbar_init(b_pempty(s), 1);
     }
@@ -181,8 +189,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint64_t pol = l2_policy_evict_first();
     bool ok = true;
     int last_t = -1;  // the last tile this group loaded
-    for (int t = grp; t < n_tiles && ok; t += 2) {
-      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+    for (int t = grp; t < n_tiles && ok; t += kStages) {
+      const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
       if (gt < kT) {
@@ -204,13 +212,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     // The loads this group issued land before the CTA may exit.
     if (gt == 0 && last_t >= 0) {
-      mbar_drain(b_kvfull(grp), static_cast<uint32_t>((last_t >> 1) & 1), P.err);
+      mbar_drain(b_kvfull(grp), static_cast<uint32_t>((last_t / kStages) & 1), P.err);
     }
   } else if (warp >= 5) {
     // ------------------------------------------------------------ gather --
     // The group copies the tile's rows in 16-byte pieces with the swizzle
     // applied, after it has staged the tile's positions.
-    const int grp = (warp - 5) >> 1;            // 0: even tiles, 1: odd tiles
+    const int grp = (warp - 5) >> 1;            // tiles t = grp (mod kStages)
     const int gt = threadIdx.x - (5 + 2 * grp) * 32;
     int* const gidx = tidx + grp * kT;
     // Cache rows of tile t's slots (thread gt < kT holds one), loaded and
@@ -238,12 +246,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
     };
     int row_cur = load_row(grp);
-    int row_nxt = load_row(grp + 2);
+    int row_nxt = load_row(grp + kStages);
     prefetch_row(row_cur);
     bool ok = true;
-    for (int t = grp; t < n_tiles && ok; t += 2) {
+    for (int t = grp; t < n_tiles && ok; t += kStages) {
       prefetch_row(row_nxt);
-      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
       if (gt < kT) gidx[gt] = row_cur;
@@ -274,9 +282,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
-      // The slot two tiles ahead is looked up while this tile's copies are in
-      // flight (its bounds check branches on the loaded entry).
-      row_nxt = load_row(t + 4);
+      // The group's slot two tiles ahead is looked up while this tile's
+      // copies are in flight (its bounds check branches on the loaded entry).
+      row_nxt = load_row(t + 2 * kStages);
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       fence_proxy_async_smem();
       mbar_arrive(b_kvfull(grp));
@@ -305,9 +313,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     };
     bool ok = wait_all(b_qfull, 0);
     auto issue_pv = [&](int u) {
-      const int st = u & 1;
+      const int st = u % kStages;
+      const int pb = u % kPStages;
       const uint64_t dv = dv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
-      const uint64_t dhi = dp0 + static_cast<uint64_t>((2 * st * kPBuf) >> 4);
+      const uint64_t dhi = dp0 + static_cast<uint64_t>((2 * pb * kPBuf) >> 4);
       const uint64_t dlo = dhi + static_cast<uint64_t>(kPBuf >> 4);
 #pragma unroll
       for (int blk = 0; blk < 4; ++blk) {
@@ -321,28 +330,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         }
       }
       tc_commit_warp(b_kvempty(st));
-      tc_commit_warp(b_pempty(st));
+      tc_commit_warp(b_pempty(pb));
       tc_commit_warp(b_odone);
     };
     auto p_ready = [&](int u) {
-      return mbar_try_wait(b_pfull(u & 1), static_cast<uint32_t>((u >> 1) & 1));
+      return mbar_test_wait(b_pfull(u % kPStages), static_cast<uint32_t>((u / kPStages) & 1));
     };
     for (int t = 0; t < n_tiles && ok; ++t) {
-      const int st = t & 1;
-      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
-      // While tile t's rows are still arriving, issue the previous tile's
-      // P.V as soon as its P is ready: that frees its gather stage early.
+      const int st = t % kStages;
+      const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
+      // S(t) goes first: the softmax waits on it.  While tile t's rows are
+      // still arriving, the previous tile's P.V is issued as soon as its P is
+      // ready, which frees its gather stage early.  The polls do not block
+      // (a suspending wait on one barrier would hold up the other).
       bool pv_pending = t > 0;
       const long long w0 = clock64();
       for (unsigned it = 1;; ++it) {
+        if (__all_sync(0xffffffffu, mbar_test_wait(b_kvfull(st), ph) &&
+                                        mbar_test_wait(b_sempty(st), ph ^ 1u))) {
+          break;
+        }
         if (pv_pending && __all_sync(0xffffffffu, p_ready(t - 1))) {
           tc_fence_after();
           issue_pv(t - 1);
           pv_pending = false;
-        }
-        if (__all_sync(0xffffffffu, mbar_try_wait(b_kvfull(st), ph) &&
-                                        mbar_try_wait(b_sempty(st), ph ^ 1u))) {
-          break;
         }
         if ((it & 63u) == 0u) {
           const bool late = clock64() - w0 > kWaitCycles;
@@ -356,7 +367,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!ok) break;
       tc_fence_after();
       const uint64_t dk = dkv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
-      const uint32_t d = tmem + kColS + 64u * st;
+      const uint32_t d = tmem + kColS + 32u * st;
 #pragma unroll
       for (int ks = 0; ks < kLatent / 16; ++ks) {
         const uint32_t off = (ks & 3) * 32;
@@ -366,14 +377,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       tc_commit_warp(b_sfull(st));
       if (pv_pending) {
-        ok = wait_all(b_pfull((t - 1) & 1), static_cast<uint32_t>(((t - 1) >> 1) & 1));
+        ok = wait_all(b_pfull((t - 1) % kPStages), static_cast<uint32_t>(((t - 1) / kPStages) & 1));
         if (!ok) break;
         tc_fence_after();
         issue_pv(t - 1);
       }
     }
     if (ok && n_tiles > 0 &&
-        wait_all(b_pfull((n_tiles - 1) & 1), static_cast<uint32_t>(((n_tiles - 1) >> 1) & 1))) {
+        wait_all(b_pfull((n_tiles - 1) % kPStages),
+                 static_cast<uint32_t>(((n_tiles - 1) / kPStages) & 1))) {
       tc_fence_after();
       issue_pv(n_tiles - 1);
     }
@@ -397,16 +409,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     float m_run = -INFINITY, l_run = 0.f, lh_run = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
-      const int st = t & 1;
-      const uint32_t ph = static_cast<uint32_t>((t >> 1) & 1);
+      const int st = t % kStages;
+      const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
       ok = mbar_wait(b_sfull(st), ph, P.err);
       if (!ok) break;
       tc_fence_after();
-      // This thread's half of its head row: keys k0 .. k0 + 23 of the tile.
-      uint32_t va[16], vb[8];
-      const uint32_t sa = tmem + lane_base + kColS + 64u * st;
-      tmem_ld_16x32bx2_x16<kSplitCols>(sa, va);
-      tmem_ld_16x32bx2_x8<kSplitCols>(sa + 16u, vb);
+      // This thread's half of its head row: keys k0 .. k0 + 15 of the tile.
+      uint32_t va[kSplitCols];
+      tmem_ld_16x32bx2_x16<kSplitCols>(tmem + lane_base + kColS + 32u * st, va);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(b_sempty(st));
@@ -415,17 +425,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!ok) break;
       // Logits in base 2; unused slots masked.
       const int* const ti = tidx + st * kT;
-      const unsigned v_lo = __ballot_sync(0xffffffffu, ti[lane] >= 0);
-      const unsigned v_hi = __ballot_sync(0xffffffffu, lane < kT - 32 && ti[32 + lane] >= 0);
       const int k0 = (lane >> 4) * kSplitCols;
-      const unsigned long long valid =
-          ((static_cast<unsigned long long>(v_hi) << 32) | v_lo) >> k0;
+      const unsigned valid = __ballot_sync(0xffffffffu, ti[lane] >= 0) >> k0;
       float s[kSplitCols];
       float tmax = -INFINITY;
 #pragma unroll
       for (int k = 0; k < kSplitCols; ++k) {
-        const float raw_s = __uint_as_float(k < 16 ? va[k] : vb[k - 16]);
-        s[k] = ((valid >> k) & 1ull) ? raw_s * P.scale_log2 : -INFINITY;
+        const float raw_s = __uint_as_float(va[k]);
+        s[k] = ((valid >> k) & 1u) ? raw_s * P.scale_log2 : -INFINITY;
         tmax = fmaxf(tmax, s[k]);
       }
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
@@ -455,11 +462,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       lh_run = lh_run * alpha + (use_lo ? sum : sumh);
       m_run = m_new;
       if (owner) alpha_s[hl] = alpha;
-      // P buffer `st` is free once the P.V of tile t-2 has completed.
-      ok = mbar_wait(b_pempty(st), ph ^ 1u, P.err);
+      // P buffer `pb` is free once the P.V of tile t-2 has completed.
+      const int pb = t % kPStages;
+      ok = mbar_wait(b_pempty(pb), static_cast<uint32_t>(((t / kPStages) & 1) ^ 1), P.err);
       if (!ok) break;
       {
-        const uint32_t prow_hi = sP + (2 * st) * kPBuf + hl * 128;
+        const uint32_t prow_hi = sP + (2 * pb) * kPBuf + hl * 128;
         const uint32_t prow_lo = prow_hi + kPBuf;
 #pragma unroll
         for (int j = 0; j < kSplitCols / 8; ++j) {
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         tmem_st_wait();
         tc_fence_before();
       }
-      mbar_arrive(b_pfull(st));
+      mbar_arrive(b_pfull(pb));
     }
     // ------------------------------------------------------------ output --
     // Per head: 1 / lh for a finished row; for a slice, lh -> l, so that the
@@ -509,7 +517,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       rl_s[hl] = !(lh_run > 0.f) ? 0.f : (P.n_split > 1 ? l_run / lh_run : 1.f / lh_run);
     }
     named_bar_sync(1, kSoftThreads);
-    if (ok && n_tiles > 0) ok = mbar_wait(b_odone, static_cast<uint32_t>((n_tiles - 1) & 1), P.err);
+    // The MMA warp's closing commit lands once every product it issued has
+    // completed (the P.V count is not enough: the product before the last
+    // may still be running when the last tile's softmax ends).
+    if (ok && n_tiles > 0) ok = mbar_wait(b_drain, 0, P.err);
     tc_fence_after();
     // The Q block and the gather stages are free once the last product has
     // completed (or, with no tile, once Q has landed): the 64 heads' rows of
