@@ -21,7 +21,6 @@ import faulthandler
 import json
 import math
 import os
-import re
 import subprocess
 import sys
 import threading
@@ -300,21 +299,20 @@ def launches_per_layer(wl, sms=148):
     return indexer + selection + 1 + (1 if few_rows and wl.top_k > 16 else 0)
 
 
-def profiled_traffic(profile="profiles/decode_b4_128k_layer.md"):
-    """DRAM bytes per indexer launch from the committed ncu summary, or None
-    once the kernel's sources differ from the ones the counters were taken on."""
+def profiled_traffic(profile="profiles/indexer_score_b4_128k_traffic.json"):
+    """DRAM bytes per in-layer indexer launch from the committed ncu record,
+    or None once the kernel's sources differ from the ones the counters were
+    taken on."""
     import hashlib
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), profile)
+    root = os.path.dirname(os.path.abspath(__file__))
     try:
-        text = open(path).read()
-        traffic = int(re.search(r"traffic_bytes:\s*(\d+)", text).group(1))
-        pins = re.search(r"source_sha256_prefix:\s*(.+)", text).group(1).split()
-    except (OSError, AttributeError, ValueError):
+        rec = json.load(open(os.path.join(root, profile)))
+        traffic = int(rec["traffic_bytes"])
+        pins = dict(rec["source_sha256_prefix"])
+    except (OSError, KeyError, TypeError, ValueError):
         return None
-    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "dsa_lightning_indexer_b200",
-                        "csrc")
-    for pin in pins:
-        name, _, prefix = pin.partition("=")
+    csrc = os.path.join(root, "dsa_lightning_indexer_b200", "csrc")
+    for name, prefix in pins.items():
         try:
             digest = hashlib.sha256(open(os.path.join(csrc, name), "rb").read()).hexdigest()
         except OSError:

@@ -8,11 +8,15 @@
 // leading 512 entries serve as V.)
 //
 // One CTA owns one query row and a block of 64 heads, and walks the row's
-// selected set in tiles of 32 gathered cache rows:
-//   S    = Q[64 heads, 576] . K_tile[32, 576]^T      M = 64,  N = 32, K = 576
-//   O^T += V_tile^T[512, 32] . P^T[32, 64 heads]     M = 128 (x4), N = 64, K = 32
-// S lands in TMEM with one head per lane, so each softmax thread owns one
-// head row: max, exp2 and row sum stay in registers.  P is written to shared
+// selected set in tiles of 48 gathered cache rows:
+//   S    = Q[64 heads, 576] . K_tile[48, 576]^T      M = 64,  N = 48, K = 576
+//   O^T += V_tile^T[512, 48] . P^T[48, 64 heads]     M = 128 (x4), N = 64, K = 48
+// Q's first 384 dims sit in TMEM for the whole row, so the S products read
+// that part of their A operand from tensor memory and only the last 192 dims
+// from shared memory: the tensor core's operand reads from shared memory set
+// the tile rate, and Q is the largest of them.  S lands in TMEM with one head
+// per lane, so each softmax thread owns one head row: max, exp2 and row sum
+// stay in registers.  P is written to shared
 // memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
 // 2^-16, on rows with fewer than kHiOnlyRows selected; longer rows take the
 // hi part alone.  The gathered tile is stored once, in the 128-byte swizzled layout,
@@ -25,8 +29,9 @@
 // warps 5-6, 7-8 and 9-10 gather tiles t = 0, 1, 2 (mod 3) with 16-byte
 // cp.async into three stages.  A stage is busy from its gather until its
 // tile's P.V completes (gather, S, softmax, P.V in a chain), so three stages
-// of 32 rows keep more of that chain in flight than two of 48 in the same
-// shared memory.
+// keep more of that chain in flight than two; the tensor core's cost per
+// product (about the same for N = 32 as for N = 48) makes the larger tile
+// the cheaper one per key.
 //
 // The same kernel, instantiated with kMasked, is the mask-over-the-whole-
 // cache route the pages describe for llama.cpp (aiaulis.com paragraph 4;
@@ -46,15 +51,18 @@ namespace {
 
 using namespace attn_tc;
 
-constexpr int kT = 32;                    // gathered rows per tile
-constexpr int kStages = 3;                // gather stages (and S buffers)
+constexpr int kT = 48;                    // gathered rows per tile
+constexpr int kStages = 3;                // gather stages
+constexpr int kSBufs = 1;                 // S buffers in TMEM
 constexpr int kPStages = 2;               // P buffers
 constexpr int kHB = 64;                   // heads per CTA
 constexpr int kBoxes = kLatent / 64;      // 64-dim column boxes of a latent row
 constexpr int kQBox = kHB * 128;          // bytes of one Q box
+constexpr int kQTmemBoxes = 6;            // Q dims 0..383: TMEM (A operand of S)
+constexpr int kQSmemBoxes = kBoxes - kQTmemBoxes;  // Q dims 384..575: shared memory
 constexpr int kKVBox = kT * 128;          // bytes of one gathered-tile box
 constexpr int kKVStage = kBoxes * kKVBox;
-constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 32 used)
+constexpr int kPBuf = kHB * 128;          // one P operand (64 heads x 64 keys, 48 used)
 constexpr int kSoftThreads = 128;
 constexpr int kGroupThreads = 64;         // one gather group
 constexpr int kThreadsTc = kSoftThreads + 32 + kStages * kGroupThreads;
@@ -67,11 +75,11 @@ constexpr float kRescaleLog2 = 8.0f;      // raise the running max only past 2^8
 constexpr int kHiOnlyRows = 1024;
 
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kBoxes * kQBox;
+constexpr int kOffKV = kOffQ + kQSmemBoxes * kQBox;
 constexpr int kOffStage = kOffQ;  // output staging [64][512] fp32 over Q and the gather stages
 constexpr int kOffP = kOffKV + kStages * kKVStage;     // [P stage][hi, lo]
 constexpr int kOffBar = kOffP + 2 * kPStages * kPBuf;
-constexpr int kNumBars = 3 + 4 * kStages + 2 * kPStages;
+constexpr int kNumBars = 4 + 2 * kStages + 2 * kSBufs + 2 * kPStages;
 constexpr int kOffTmem = kOffBar + 8 * kNumBars;
 constexpr int kOffIdx = kOffTmem + 16;                  // [kStages][kT] int
 constexpr int kOffAlpha = kOffIdx + kStages * kT * 4;   // [64] float
@@ -85,14 +93,18 @@ static_assert(kOffStage + kHB * kValue * 4 <= kOffP, "output staging overlaps th
 static_assert(kSmemTc <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // S buffers at columns 0, 32, 64 (M = 64 layout)
-constexpr uint32_t kColO = 128;   // O^T blocks at 128, 192, 256, 320
+constexpr uint32_t kColS = 0;     // the S buffer, columns 0..47 (M = 64 layout)
+constexpr uint32_t kColQ = 64;    // Q dims 0..383, two bf16 per column (M = 64 layout)
+constexpr uint32_t kColO = 256;   // O^T blocks at 256, 320, 384, 448
+static_assert(kColS + kT * kSBufs <= kColQ && kColQ + 32 * kQTmemBoxes <= kColO &&
+                  kColO + 4 * 64 <= kTmemCols,
+              "TMEM columns");
 
 // kind::f16 instruction descriptors (bf16 in, fp32 accumulate).
 constexpr uint32_t kIdescS = idesc_bf16_f32(64, kT);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, kHB) | (1u << 15);  // A MN-major
-constexpr int kSplitCols = kT / 2;  // logits per half warp
-static_assert(kSplitCols == 16, "one 16-column load per half warp covers its logits");
+constexpr int kSplitCols = kT / 2;  // logits per half warp (16 + 8 columns)
+static_assert(kSplitCols == 24, "the logit loads cover 16 + 8 columns per half warp");
 
 template <bool kMasked>
 __global__ void __launch_bounds__(kThreadsTc, 1)
@@ -108,11 +120,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   auto b_kvfull = [&](int s) { return bars + 8u * (1 + s); };
   auto b_kvempty = [&](int s) { return bars + 8u * (1 + kStages + s); };
   auto b_sfull = [&](int s) { return bars + 8u * (1 + 2 * kStages + s); };
-  auto b_sempty = [&](int s) { return bars + 8u * (1 + 3 * kStages + s); };
-  auto b_pfull = [&](int s) { return bars + 8u * (1 + 4 * kStages + s); };
-  auto b_pempty = [&](int s) { return bars + 8u * (1 + 4 * kStages + kPStages + s); };
-  const uint32_t b_odone = bars + 8u * (1 + 4 * kStages + 2 * kPStages);
+  auto b_sempty = [&](int s) { return bars + 8u * (1 + 2 * kStages + kSBufs + s); };
+  auto b_pfull = [&](int s) { return bars + 8u * (1 + 2 * kStages + 2 * kSBufs + s); };
+  auto b_pempty = [&](int s) { return bars + 8u * (1 + 2 * kStages + 2 * kSBufs + kPStages + s); };
+  const uint32_t b_odone = bars + 8u * (1 + 2 * kStages + 2 * kSBufs + 2 * kPStages);
   const uint32_t b_drain = b_odone + 8u;
+  const uint32_t b_qtmem = b_odone + 16u;  // Q's TMEM part stored
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(bp + kOffTmem);
   int* const tidx = reinterpret_cast<int*>(bp + kOffIdx);
   float* const alpha_s = reinterpret_cast<float*>(bp + kOffAlpha);
@@ -130,6 +143,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(b_kvfull(s), kMasked ? 1 : kGroupThreads);
       mbar_init(b_kvempty(s), 1);
+    }
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(b_sfull(s), 1);
       mbar_init(b_sempty(s), kSoftThreads);
     }
@@ -139,6 +154,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     mbar_init(b_odone, 1);
     mbar_init(b_drain, 1);
+    mbar_init(b_qtmem, kSoftThreads);
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -295,10 +311,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // warp-uniform); one elected lane issues each MMA and commit.
     if (lane == 0) {
       tma_prefetch_map(&qmap);
-      mbar_arrive_expect_tx(b_qfull, kBoxes * kQBox);
+      // Only Q's shared-memory part; the softmax warps store the rest in TMEM.
+      mbar_arrive_expect_tx(b_qfull, kQSmemBoxes * kQBox);
       const uint64_t pol = l2_policy_evict_first();
-      for (int j = 0; j < kBoxes; ++j) {
-        tma_load_2d(sQ + j * kQBox, &qmap, b_qfull, 64 * j, r * P.H + h0, pol);
+      for (int j = kQTmemBoxes; j < kBoxes; ++j) {
+        tma_load_2d(sQ + (j - kQTmemBoxes) * kQBox, &qmap, b_qfull, 64 * j, r * P.H + h0, pol);
       }
     }
     __syncwarp();
@@ -311,7 +328,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     auto wait_all = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, P.err));
     };
-    bool ok = wait_all(b_qfull, 0);
+    bool ok = wait_all(b_qfull, 0) && wait_all(b_qtmem, 0);
+    tc_fence_after();
     auto issue_pv = [&](int u) {
       const int st = u % kStages;
       const int pb = u % kPStages;
@@ -339,6 +357,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int st = t % kStages;
       const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
+      const int sb = t % kSBufs;
+      const uint32_t sph = static_cast<uint32_t>((t / kSBufs) & 1);
       // S(t) goes first: the softmax waits on it.  While tile t's rows are
       // still arriving, the previous tile's P.V is issued as soon as its P is
       // ready, which frees its gather stage early.  The polls do not block
@@ -347,7 +367,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const long long w0 = clock64();
       for (unsigned it = 1;; ++it) {
         if (__all_sync(0xffffffffu, mbar_test_wait(b_kvfull(st), ph) &&
-                                        mbar_test_wait(b_sempty(st), ph ^ 1u))) {
+                                        mbar_test_wait(b_sempty(sb), sph ^ 1u))) {
           break;
         }
         if (pv_pending && __all_sync(0xffffffffu, p_ready(t - 1))) {
@@ -367,15 +387,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (!ok) break;
       tc_fence_after();
       const uint64_t dk = dkv0 + static_cast<uint64_t>((st * kKVStage) >> 4);
-      const uint32_t d = tmem + kColS + 32u * st;
+      const uint32_t d = tmem + kColS + static_cast<uint32_t>(kT) * sb;
 #pragma unroll
       for (int ks = 0; ks < kLatent / 16; ++ks) {
+        const int box = ks >> 2;
         const uint32_t off = (ks & 3) * 32;
-        tc_mma_bf16_warp(d, dq + static_cast<uint64_t>(((ks >> 2) * kQBox + off) >> 4),
-                         dk + static_cast<uint64_t>(((ks >> 2) * kKVBox + off) >> 4), kIdescS,
-                         ks > 0 ? 1u : 0u);
+        const uint64_t b = dk + static_cast<uint64_t>((box * kKVBox + off) >> 4);
+        if (box < kQTmemBoxes) {  // 16 dims = 8 TMEM columns of Q per K step
+          tc_mma_bf16_ts_warp(d, tmem + kColQ + 8u * ks, b, kIdescS, ks > 0 ? 1u : 0u);
+        } else {
+          tc_mma_bf16_warp(d, dq + static_cast<uint64_t>(((box - kQTmemBoxes) * kQBox + off) >> 4),
+                           b, kIdescS, 1u);
+        }
       }
-      tc_commit_warp(b_sfull(st));
+      tc_commit_warp(b_sfull(sb));
       if (pv_pending) {
         ok = wait_all(b_pfull((t - 1) % kPStages), static_cast<uint32_t>(((t - 1) / kPStages) & 1));
         if (!ok) break;
@@ -407,32 +432,63 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // the product used (the same with the lo part; the rounded hi parts
     // without it), which normalises the output.
     float m_run = -INFINITY, l_run = 0.f, lh_run = 0.f;
+    {
+      // Q's dims 0..383 of head row hl into TMEM, in the M = 64 operand
+      // layout (head 16q + i at lane 32q + i, dims 2c and 2c + 1 in column
+      // kColQ + c): each half warp writes 32 dims of the row per store.
+      const int half = lane >> 4;
+      const bool have = h0 + hl < P.H;
+      const uint4* const src = reinterpret_cast<const uint4*>(
+          P.q + (static_cast<size_t>(r) * P.H + h0 + hl) * kLatent);
+#pragma unroll 1
+      for (int m = 0; m < kQTmemBoxes; ++m) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 x = have ? __ldg(src + (64 * m + 32 * half) / 8 + j) : make_uint4(0, 0, 0, 0);
+          v[4 * j] = x.x;
+          v[4 * j + 1] = x.y;
+          v[4 * j + 2] = x.z;
+          v[4 * j + 3] = x.w;
+        }
+        tmem_st_16x32bx2_x16<16>(tmem + lane_base + kColQ + 32u * m, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(b_qtmem);
+    }
     bool ok = true;
     for (int t = 0; t < n_tiles && ok; ++t) {
       const int st = t % kStages;
       const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
-      ok = mbar_wait(b_sfull(st), ph, P.err);
+      const int sb = t % kSBufs;
+      ok = mbar_wait(b_sfull(sb), static_cast<uint32_t>((t / kSBufs) & 1), P.err);
       if (!ok) break;
       tc_fence_after();
-      // This thread's half of its head row: keys k0 .. k0 + 15 of the tile.
-      uint32_t va[kSplitCols];
-      tmem_ld_16x32bx2_x16<kSplitCols>(tmem + lane_base + kColS + 32u * st, va);
+      // This thread's half of its head row: keys k0 .. k0 + 23 of the tile.
+      uint32_t va[16], vb[8];
+      const uint32_t sa = tmem + lane_base + kColS + static_cast<uint32_t>(kT) * sb;
+      tmem_ld_16x32bx2_x16<kSplitCols>(sa, va);
+      tmem_ld_16x32bx2_x8<kSplitCols>(sa + 16u, vb);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(b_sempty(st));
+      mbar_arrive(b_sempty(sb));
       // The tile's slot list was written by its gather group before kv_full.
       ok = mbar_wait(b_kvfull(st), ph, P.err);
       if (!ok) break;
       // Logits in base 2; unused slots masked.
       const int* const ti = tidx + st * kT;
+      const unsigned v_lo = __ballot_sync(0xffffffffu, ti[lane] >= 0);
+      const unsigned v_hi = __ballot_sync(0xffffffffu, lane < kT - 32 && ti[32 + lane] >= 0);
       const int k0 = (lane >> 4) * kSplitCols;
-      const unsigned valid = __ballot_sync(0xffffffffu, ti[lane] >= 0) >> k0;
+      const unsigned long long valid =
+          ((static_cast<unsigned long long>(v_hi) << 32) | v_lo) >> k0;
       float s[kSplitCols];
       float tmax = -INFINITY;
 #pragma unroll
       for (int k = 0; k < kSplitCols; ++k) {
-        const float raw_s = __uint_as_float(va[k]);
-        s[k] = ((valid >> k) & 1u) ? raw_s * P.scale_log2 : -INFINITY;
+        const float raw_s = __uint_as_float(k < 16 ? va[k] : vb[k - 16]);
+        s[k] = ((valid >> k) & 1ull) ? raw_s * P.scale_log2 : -INFINITY;
         tmax = fmaxf(tmax, s[k]);
       }
       tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
@@ -642,6 +698,7 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   P.H = a.H;
   P.top_k = a.top_k;
   P.scale_log2 = a.scale * kLog2e;
+  P.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   const int head_blocks = (a.H + kHB - 1) / kHB;
   e = launch_pdl(sparse_attn_tc_kernel<kMasked>, dim3(a.Nq, head_blocks, a.plan.n_split),
                  dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, kvmap, P);
