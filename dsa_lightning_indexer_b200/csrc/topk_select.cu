@@ -309,12 +309,69 @@ __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, i
   need = remaining;
 }
 
+// Finds, among the `n` keys key_at(0 .. n-1), the `want`-th largest key theta
+// and how many keys equal to theta are needed, with a block of kThr threads.
+// Every key has the bits `known_mask` equal to `known`; radix passes of up to
+// 11 bits cover the bits in [lo_bit, hi_bit].
+template <int kThr, class KeyAt>
+__device__ void radix_select(KeyAt key_at, int n, int want, int lo_bit, int hi_bit,
+                             uint32_t known, uint32_t known_mask, int* hist /*[2048]*/, int* buf,
+                             uint32_t& theta, int& need) {
+  constexpr int kD = 2048 / kThr;  // digits per thread in the scan
+  __shared__ int pd, pa;
+  uint32_t prefix = known, pmask = known_mask;
+  int remaining = want;
+  for (int top = hi_bit; top >= lo_bit;) {
+    const int nbits = min(11, top - lo_bit + 1);
+    const int shift = top - nbits + 1;
+    const uint32_t dmask = (1u << nbits) - 1u;
+    for (int i = threadIdx.x; i < 2048; i += kThr) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kThr) {
+      const uint32_t key = key_at(i);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
+    }
+    __syncthreads();
+    // Thread t scans digits kD*u .. kD*u + kD-1 with u = kThr-1-t, so the
+    // exclusive prefix in thread order counts the keys in higher digits.
+    const int u = kThr - 1 - static_cast<int>(threadIdx.x);
+    int c[kD];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < kD; ++j) {
+      c[j] = hist[kD * u + j];
+      tot += c[j];
+    }
+    int total;
+    int above = block_excl_sum_nw<kThr / 32>(tot, buf, total);
+    if (above < remaining && remaining <= above + tot) {
+#pragma unroll
+      for (int j = kD - 1; j >= 0; --j) {
+        if (above + c[j] >= remaining) {
+          pd = kD * u + j;
+          pa = above;
+          break;
+        }
+        above += c[j];
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(pd) << shift;
+    pmask |= dmask << shift;
+    remaining -= pa;
+    __syncthreads();
+    top = shift - 1;
+  }
+  theta = prefix;
+  need = remaining;
+}
+
 // ------------------------------------------------------- one CTA per row --
-// Many rows that each fit one CTA's shared memory (prefill).  Three sweeps
-// over the row's keys instead of one per radix digit:
-//   1. load the scores as keys (16-byte loads) and count them by their top
-//      12 bits; one scan of the 4096 counts gives the bin holding the k-th
-//      largest key and how many keys lie above it;
+// Many rows (prefill): one 256-thread CTA per row and three sweeps over the
+// row's scores instead of one per radix digit:
+//   1. count the keys by their top 12 bits (16-byte loads); one scan of the
+//      4096 counts gives the bin holding the k-th largest key and how many
+//      keys lie above it;
 //   2. copy the keys of that bin (typically a few hundred) with their
 //      positions to a candidate list, and count per warp chunk the keys
 //      above the bin;
@@ -322,21 +379,25 @@ __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, i
 //      come from radix passes over the candidates alone (over the whole row
 //      when the bin holds more than kRowCandMax keys, i.e. heavy ties);
 //   3. emit in position order as the cluster kernel does.
+// Sweeps 2 and 3 re-read the row (from L2: it was just read), so a CTA needs
+// only the histogram and the candidates in shared memory (32 KB) and several
+// rows share an SM, hiding one another's barrier waits.
 constexpr int kRowCandMax = 2048;
+constexpr int kRThreads = 256;
+constexpr int kRWarps = kRThreads / 32;
 
 __device__ __forceinline__ void row_hist_add(int* hist, uint32_t key) {
   atomicAdd(&hist[key >> kHistShift], 1);
 }
 
-__global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkParams P) {
+__global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   int* const hist = reinterpret_cast<int*>(smem);                          // [kHistBins]
   uint32_t* const ckey = reinterpret_cast<uint32_t*>(hist + kHistBins);    // [kRowCandMax]
   int* const cpos = reinterpret_cast<int*>(ckey + kRowCandMax);            // [kRowCandMax]
-  uint32_t* const keys = reinterpret_cast<uint32_t*>(cpos + kRowCandMax);  // [slice]
-  __shared__ int buf[kHWarps + 1];
+  __shared__ int buf[kRWarps + 1];
   __shared__ int s_bin, s_above, s_cnt, s_ncand;
-  __shared__ int warp_gt[kHWarps], warp_eq[kHWarps];
+  __shared__ int warp_gt[kRWarps], warp_eq[kRWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
@@ -346,56 +407,58 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
   const int b = owner_seq(P.q_offsets, P.B, r);
   const int q0 = P.q_offsets[b];
   const int nq = P.q_offsets[b + 1] - q0;
-  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;  // positions 0..p; n <= slice
+  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;  // positions 0..p
   const int k = P.top_k;
   int32_t* const out = P.idx + static_cast<size_t>(r) * k;
   if (n <= k) {  // every causal position is kept
-    for (int i = tid; i < k; i += kHThreads) out[i] = i < n ? i : -1;
+    for (int i = tid; i < k; i += kRThreads) out[i] = i < n ? i : -1;
     return;
   }
+  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
+  auto key_at = [&](int i) { return score_key(sc[i]); };
 
-  // ---- sweep 1: keys into shared memory, coarse histogram
-  for (int i = tid; i < kHistBins; i += kHThreads) hist[i] = 0;
+  // ---- sweep 1: coarse histogram
+  for (int i = tid; i < kHistBins; i += kRThreads) hist[i] = 0;
   if (tid == 0) s_ncand = 0;
-  if (tid < kHWarps) {
+  if (tid < kRWarps) {
     warp_gt[tid] = 0;
     warp_eq[tid] = 0;
   }
   __syncthreads();
-  const float* const sc = P.scores + static_cast<size_t>(r) * P.ld;
   const int n4 = (reinterpret_cast<uintptr_t>(sc) & 15u) == 0 ? (n & ~3) : 0;
-  for (int i = 4 * tid; i < n4; i += 4 * kHThreads) {
+  for (int i = 4 * tid; i < n4; i += 4 * kRThreads) {
     const float4 v = *reinterpret_cast<const float4*>(sc + i);
-    const uint4 kk = make_uint4(score_key(v.x), score_key(v.y), score_key(v.z), score_key(v.w));
-    *reinterpret_cast<uint4*>(keys + i) = kk;
-    row_hist_add(hist, kk.x);
-    row_hist_add(hist, kk.y);
-    row_hist_add(hist, kk.z);
-    row_hist_add(hist, kk.w);
+    row_hist_add(hist, score_key(v.x));
+    row_hist_add(hist, score_key(v.y));
+    row_hist_add(hist, score_key(v.z));
+    row_hist_add(hist, score_key(v.w));
   }
-  for (int i = n4 + tid; i < n; i += kHThreads) {
-    const uint32_t key = score_key(sc[i]);
-    keys[i] = key;
-    row_hist_add(hist, key);
-  }
+  for (int i = n4 + tid; i < n; i += kRThreads) row_hist_add(hist, key_at(i));
   __syncthreads();
   {
-    // Thread t holds bins 8u .. 8u+7 with u = 511 - t, so the exclusive
+    // Thread t holds bins 16u .. 16u+15 with u = 255 - t, so the exclusive
     // prefix in thread order counts the keys in higher bins.
-    const int u = kHThreads - 1 - tid;
-    const int4 ha = reinterpret_cast<const int4*>(hist)[2 * u];
-    const int4 hb = reinterpret_cast<const int4*>(hist)[2 * u + 1];
-    const int c[8] = {ha.x, ha.y, ha.z, ha.w, hb.x, hb.y, hb.z, hb.w};
+    constexpr int kPer = kHistBins / kRThreads;
+    const int u = kRThreads - 1 - tid;
+    int c[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; j += 4) {
+      const int4 h = reinterpret_cast<const int4*>(hist)[(kPer * u + j) / 4];
+      c[j] = h.x;
+      c[j + 1] = h.y;
+      c[j + 2] = h.z;
+      c[j + 3] = h.w;
+    }
     int tot = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) tot += c[j];
+    for (int j = 0; j < kPer; ++j) tot += c[j];
     int total;
-    int above = block_excl_sum_nw<kHWarps>(tot, buf, total);
+    int above = block_excl_sum_nw<kRWarps>(tot, buf, total);
     if (above < k && k <= above + tot) {
 #pragma unroll
-      for (int j = 7; j >= 0; --j) {
+      for (int j = kPer - 1; j >= 0; --j) {
         if (above + c[j] >= k) {
-          s_bin = 8 * u + j;
+          s_bin = kPer * u + j;
           s_above = above;
           s_cnt = c[j];
           break;
@@ -410,7 +473,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
   const bool compact = s_cnt <= kRowCandMax;
 
   // ---- sweep 2: candidates of the bin; keys above the bin per warp chunk
-  const int per_warp = ((n + kHWarps - 1) / kHWarps + 31) & ~31;
+  const int per_warp = ((n + kRWarps - 1) / kRWarps + 31) & ~31;
   const int w0 = warp * per_warp;
   const int w1 = min(n, w0 + per_warp);
   const unsigned lt = (1u << lane) - 1u;
@@ -418,7 +481,8 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
     int g = 0;
     for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
       const bool in = i < w1;
-      const int d = in ? static_cast<int>(keys[i] >> kHistShift) : -1;
+      const uint32_t key = in ? key_at(i) : 0u;
+      const int d = in ? static_cast<int>(key >> kHistShift) : -1;
       g += __popc(__ballot_sync(0xffffffffu, d > bin));
       const unsigned m = __ballot_sync(0xffffffffu, d == bin);
       if (m != 0u) {
@@ -427,7 +491,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
         base = __shfl_sync(0xffffffffu, base, 0);
         if ((m >> lane) & 1u) {
           const int j = base + __popc(m & lt);
-          ckey[j] = keys[i];
+          ckey[j] = key;
           cpos[j] = i;
         }
       }
@@ -440,10 +504,11 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
   const uint32_t known = static_cast<uint32_t>(bin) << kHistShift;
   const uint32_t known_mask = ~((1u << kHistShift) - 1u);
   if (compact) {
-    smem_select(ckey, s_ncand, want, 0, kHistShift - 1, known, known_mask, hist, buf, theta, need);
+    radix_select<kRThreads>([&](int j) { return ckey[j]; }, s_ncand, want, 0, kHistShift - 1,
+                            known, known_mask, hist, buf, theta, need);
     // Candidates above theta and equal to it, by the warp chunk holding them.
     const int nc = s_ncand;
-    for (int j = tid; j < nc; j += kHThreads) {
+    for (int j = tid; j < nc; j += kRThreads) {
       const uint32_t key = ckey[j];
       const int w = cpos[j] / per_warp;
       if (key > theta) {
@@ -453,11 +518,12 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
       }
     }
   } else {
-    smem_select(keys, n, want, 0, kHistShift - 1, known, known_mask, hist, buf, theta, need);
+    radix_select<kRThreads>(key_at, n, want, 0, kHistShift - 1, known, known_mask, hist, buf,
+                            theta, need);
     int g = 0, e = 0;
     for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
       const bool in = i < w1;
-      const uint32_t key = in ? keys[i] : 0u;
+      const uint32_t key = in ? key_at(i) : 0u;
       g += __popc(__ballot_sync(0xffffffffu, in && key > theta));
       e += __popc(__ballot_sync(0xffffffffu, in && key == theta));
     }
@@ -476,7 +542,7 @@ __global__ void __launch_bounds__(kHThreads, 2) topk_row_cta_kernel(const TopkPa
   }
   for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
     const bool in = i < w1;
-    const uint32_t key = in ? keys[i] : 0u;
+    const uint32_t key = in ? key_at(i) : 0u;
     const unsigned gm = __ballot_sync(0xffffffffu, in && key > theta);
     const unsigned em = __ballot_sync(0xffffffffu, in && key == theta);
     const bool take_eq = ((em >> lane) & 1u) && eq_acc + __popc(em & lt) < need;
@@ -957,14 +1023,13 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
     return launch_pdl(topk_rows_kernel, dim3(a.Nq), dim3(kThreads), 0, stream, 0, P);
   }
   P.slice = static_cast<int>(slice_of(cs));
-  if (cs == 1) {  // many rows, each within one CTA
-    const size_t head = static_cast<size_t>(kHistBins) * sizeof(int) +
+  if (cs == 1) {  // many rows, one CTA each
+    const size_t smem = static_cast<size_t>(kHistBins) * sizeof(int) +
                         static_cast<size_t>(kRowCandMax) * (sizeof(uint32_t) + sizeof(int));
-    cudaError_t e = ensure_smem_limit<topk_row_cta_kernel>(
-        static_cast<int>(head + static_cast<size_t>(kMaxSlice) * sizeof(uint32_t)));
+    cudaError_t e = ensure_smem_limit<topk_row_cta_kernel>(static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    return launch_pdl(topk_row_cta_kernel, dim3(static_cast<unsigned>(a.Nq)), dim3(kHThreads),
-                      head + static_cast<size_t>(P.slice) * sizeof(uint32_t), stream, 0, P);
+    return launch_pdl(topk_row_cta_kernel, dim3(static_cast<unsigned>(a.Nq)), dim3(kRThreads),
+                      smem, stream, 0, P);
   }
   const size_t smem = 2 * kBins * sizeof(int) + static_cast<size_t>(P.slice) * sizeof(uint32_t);
   // The limit is raised once, to the largest slice any launch may use.
