@@ -70,6 +70,19 @@ __device__ __forceinline__ long long seq_row(const SeqRows& s, int pos) {
          static_cast<long long>(pos & ((1 << s.page_shift) - 1));
 }
 
+// (a, b) = (wa, wb) * (xa, xb) + (a, b) as one paired fp32 FMA; each lane is
+// an fma rounded to nearest, the same result as fmaf.
+__device__ __forceinline__ void ffma2(float& a, float& b, float wa, float wb, float xa, float xb) {
+  asm("{\n\t.reg .b64 acc, w, x;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 w, {%2, %3};\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "fma.rn.f32x2 acc, w, x, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(wa), "f"(wb), "f"(xa), "f"(xb));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -376,14 +376,16 @@ __global__ void __launch_bounds__(Cfg<QT>::kThreads, 1)
           tmem_ld_wait();
           const float4* wp =
               reinterpret_cast<const float4*>(P.w + static_cast<size_t>(v.row0 + jq) * kIdxHeads);
+          // Four partial sums (heads h = j mod 4), updated two at a time by
+          // paired fp32 FMAs: each lane rounds as fmaf does, in the same order.
           float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
           for (int h4 = 0; h4 < kIdxHeads / 4; ++h4) {
             const float4 ww = __ldg(wp + h4);
-            s0 = fmaf(ww.x, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f), s0);
-            s1 = fmaf(ww.y, fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f), s1);
-            s2 = fmaf(ww.z, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f), s2);
-            s3 = fmaf(ww.w, fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f), s3);
+            ffma2(s0, s1, ww.x, ww.y, fmaxf(__uint_as_float(r[4 * h4 + 0]), 0.f),
+                  fmaxf(__uint_as_float(r[4 * h4 + 1]), 0.f));
+            ffma2(s2, s3, ww.z, ww.w, fmaxf(__uint_as_float(r[4 * h4 + 2]), 0.f),
+                  fmaxf(__uint_as_float(r[4 * h4 + 3]), 0.f));
           }
           float s = (s0 + s1) + (s2 + s3);
           if (s == 0.f) s = 0.f;  // one zero: -0 and +0 are the same score
