@@ -161,6 +161,11 @@ ATTN = {
     # 48 query rows of 2048 selected each: P without its lo part, split over
     # CTAs and merged
     "long_rows_hi_only": lambda: synth.custom([3000], [48], 64, 2048, seed=117),
+    # 80 heads: a full 64-head block and one of 16, whose query rows past H
+    # are zero in tensor memory; short rows (P with its lo part), then rows
+    # of 1024 selected (P alone)
+    "prefill_h80": lambda: synth.prefill(256, 80, 96, seed=118),
+    "long_rows_h80_hi_only": lambda: synth.custom([1500], [40], 80, 1024, seed=119),
 }
 
 
