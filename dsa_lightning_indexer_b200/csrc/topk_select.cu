@@ -367,21 +367,22 @@ __device__ void radix_select(KeyAt key_at, int n, int want, int lo_bit, int hi_b
 }
 
 // ------------------------------------------------------- one CTA per row --
-// Many rows (prefill): one 256-thread CTA per row and three sweeps over the
-// row's scores instead of one per radix digit:
+// Many rows (prefill): one 256-thread CTA per row.
 //   1. count the keys by their top 12 bits (16-byte loads); one scan of the
 //      4096 counts gives the bin holding the k-th largest key and how many
 //      keys lie above it;
-//   2. copy the keys of that bin (typically a few hundred) with their
-//      positions to a candidate list, and count per warp chunk the keys
-//      above the bin;
-//      the k-th key theta and the number of keys equal to theta to keep then
-//      come from radix passes over the candidates alone (over the whole row
-//      when the bin holds more than kRowCandMax keys, i.e. heavy ties);
-//   3. emit in position order as the cluster kernel does.
-// Sweeps 2 and 3 re-read the row (from L2: it was just read), so a CTA needs
-// only the histogram and the candidates in shared memory (32 KB) and several
-// rows share an SM, hiding one another's barrier waits.
+//   2. a second read of the row (from L2: it was just read) gives a bitmask
+//      of the positions above that bin and a list of the keys inside it
+//      (typically a few hundred) with their positions;
+//   3. radix passes (11 + 9 bits) over the candidates alone give the k-th
+//      key theta and how many keys equal to theta to keep; the selected
+//      candidates are added to the bitmask (ties at theta: the lowest
+//      positions, by a radix select on the complemented positions);
+//   4. the positions are emitted in ascending order from the bitmask words,
+//      placed by one block prefix sum of their bit counts.
+// A bin holding more than kRowCandMax keys (heavy ties) takes the whole-row
+// path instead: radix passes over every key of the row and an ordered
+// emission, both re-reading the scores.
 constexpr int kRowCandMax = 2048;
 constexpr int kRThreads = 256;
 constexpr int kRWarps = kRThreads / 32;
@@ -390,13 +391,23 @@ __device__ __forceinline__ void row_hist_add(int* hist, uint32_t key) {
   atomicAdd(&hist[key >> kHistShift], 1);
 }
 
+// Dynamic shared memory of the row kernel for rows of up to `slice` keys
+// (a multiple of 128): histogram, candidates, bitmask.  Small enough that
+// six rows share an SM, whose loads hide one another's latency.
+__host__ __device__ constexpr size_t row_cta_smem(int slice) {
+  return static_cast<size_t>(kHistBins) * sizeof(int) +
+         static_cast<size_t>(kRowCandMax) * (sizeof(uint32_t) + sizeof(int)) +
+         static_cast<size_t>(slice / 32) * sizeof(uint32_t);
+}
+
 __global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   int* const hist = reinterpret_cast<int*>(smem);                          // [kHistBins]
   uint32_t* const ckey = reinterpret_cast<uint32_t*>(hist + kHistBins);    // [kRowCandMax]
   int* const cpos = reinterpret_cast<int*>(ckey + kRowCandMax);            // [kRowCandMax]
+  uint32_t* const mask = reinterpret_cast<uint32_t*>(cpos + kRowCandMax);  // [slice / 32]
   __shared__ int buf[kRWarps + 1];
-  __shared__ int s_bin, s_above, s_cnt, s_ncand;
+  __shared__ int s_bin, s_above, s_cnt, s_ncand, s_neq;
   __shared__ int warp_gt[kRWarps], warp_eq[kRWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -407,7 +418,7 @@ __global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkPa
   const int b = owner_seq(P.q_offsets, P.B, r);
   const int q0 = P.q_offsets[b];
   const int nq = P.q_offsets[b + 1] - q0;
-  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;  // positions 0..p
+  const int n = P.ctx_lens[b] - nq + (r - q0) + 1;  // positions 0..p; n <= slice
   const int k = P.top_k;
   int32_t* const out = P.idx + static_cast<size_t>(r) * k;
   if (n <= k) {  // every causal position is kept
@@ -419,7 +430,10 @@ __global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkPa
 
   // ---- sweep 1: coarse histogram
   for (int i = tid; i < kHistBins; i += kRThreads) hist[i] = 0;
-  if (tid == 0) s_ncand = 0;
+  if (tid == 0) {
+    s_ncand = 0;
+    s_neq = 0;
+  }
   if (tid < kRWarps) {
     warp_gt[tid] = 0;
     warp_eq[tid] = 0;
@@ -470,56 +484,82 @@ __global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkPa
   __syncthreads();
   const int bin = s_bin;
   const int want = k - s_above;  // keys to keep from the bin, 1 .. s_cnt
-  const bool compact = s_cnt <= kRowCandMax;
-
-  // ---- sweep 2: candidates of the bin; keys above the bin per warp chunk
-  const int per_warp = ((n + kRWarps - 1) / kRWarps + 31) & ~31;
-  const int w0 = warp * per_warp;
-  const int w1 = min(n, w0 + per_warp);
+  const uint32_t known = static_cast<uint32_t>(bin) << kHistShift;
+  const uint32_t known_mask = ~((1u << kHistShift) - 1u);
   const unsigned lt = (1u << lane) - 1u;
-  if (compact) {
-    int g = 0;
-    for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
-      const bool in = i < w1;
-      const uint32_t key = in ? key_at(i) : 0u;
-      const int d = in ? static_cast<int>(key >> kHistShift) : -1;
-      g += __popc(__ballot_sync(0xffffffffu, d > bin));
-      const unsigned m = __ballot_sync(0xffffffffu, d == bin);
-      if (m != 0u) {
+  uint32_t theta;
+  int need;
+
+  if (s_cnt <= kRowCandMax) {
+    // ---- sweep 2: bitmask above the bin, candidates
+    const int W = (n + 31) >> 5;
+    for (int w = warp; w < W; w += kRWarps) {
+      const int i = 32 * w + lane;
+      const uint32_t key = i < n ? key_at(i) : 0u;
+      const int d = i < n ? static_cast<int>(key >> kHistShift) : -1;
+      const unsigned gm = __ballot_sync(0xffffffffu, d > bin);
+      const unsigned em = __ballot_sync(0xffffffffu, d == bin);
+      if (lane == 0) mask[w] = gm;
+      if (em != 0u) {
         int base = 0;
-        if (lane == 0) base = atomicAdd(&s_ncand, __popc(m));
+        if (lane == 0) base = atomicAdd(&s_ncand, __popc(em));
         base = __shfl_sync(0xffffffffu, base, 0);
-        if ((m >> lane) & 1u) {
-          const int j = base + __popc(m & lt);
+        if (d == bin) {
+          const int j = base + __popc(em & lt);
           ckey[j] = key;
           cpos[j] = i;
         }
       }
     }
-    if (lane == 0) atomicAdd(&warp_gt[warp], g);
-  }
-  __syncthreads();
-  uint32_t theta;
-  int need;
-  const uint32_t known = static_cast<uint32_t>(bin) << kHistShift;
-  const uint32_t known_mask = ~((1u << kHistShift) - 1u);
-  if (compact) {
-    radix_select<kRThreads>([&](int j) { return ckey[j]; }, s_ncand, want, 0, kHistShift - 1,
-                            known, known_mask, hist, buf, theta, need);
-    // Candidates above theta and equal to it, by the warp chunk holding them.
+    __syncthreads();
     const int nc = s_ncand;
+    radix_select<kRThreads>([&](int j) { return ckey[j]; }, nc, want, 0, kHistShift - 1, known,
+                            known_mask, hist, buf, theta, need);
+    // Keys equal to theta: keep the `need` lowest positions.
+    for (int j = tid; j < nc; j += kRThreads) {
+      if (ckey[j] == theta) atomicAdd(&s_neq, 1);
+    }
+    __syncthreads();
+    uint32_t pos_cut = 0u;  // equal keys kept: ~position >= pos_cut
+    if (need < s_neq) {
+      int unused;
+      radix_select<kRThreads>(
+          [&](int j) { return ckey[j] == theta ? ~static_cast<uint32_t>(cpos[j]) : 0u; }, nc,
+          need, 0, 31, 0u, 0u, hist, buf, pos_cut, unused);
+    }
     for (int j = tid; j < nc; j += kRThreads) {
       const uint32_t key = ckey[j];
-      const int w = cpos[j] / per_warp;
-      if (key > theta) {
-        atomicAdd(&warp_gt[w], 1);
-      } else if (key == theta) {
-        atomicAdd(&warp_eq[w], 1);
+      const int pos = cpos[j];
+      if (key > theta || (key == theta && ~static_cast<uint32_t>(pos) >= pos_cut)) {
+        atomicOr(&mask[pos >> 5], 1u << (pos & 31));
       }
     }
-  } else {
-    radix_select<kRThreads>(key_at, n, want, 0, kHistShift - 1, known, known_mask, hist, buf,
-                            theta, need);
+    __syncthreads();
+    // ---- emit from the bitmask: each thread a run of words, in order
+    const int wpt = (W + kRThreads - 1) / kRThreads;
+    const int wa = min(W, tid * wpt), wb = min(W, wa + wpt);
+    int cnt = 0;
+    for (int w = wa; w < wb; ++w) cnt += __popc(mask[w]);
+    int total;
+    int at = block_excl_sum_nw<kRWarps>(cnt, buf, total);
+    for (int w = wa; w < wb; ++w) {
+      uint32_t m = mask[w];
+      while (m != 0u && at < k) {
+        out[at++] = 32 * w + __ffs(m) - 1;
+        m &= m - 1u;
+      }
+    }
+    for (int i = total + tid; i < k; i += kRThreads) out[i] = -1;  // never with exact counts
+    return;
+  }
+
+  // ---- heavy ties: radix passes over the whole row, then ordered emission
+  const int per_warp = ((n + kRWarps - 1) / kRWarps + 31) & ~31;
+  const int w0 = warp * per_warp;
+  const int w1 = min(n, w0 + per_warp);
+  radix_select<kRThreads>(key_at, n, want, 0, kHistShift - 1, known, known_mask, hist, buf, theta,
+                          need);
+  {
     int g = 0, e = 0;
     for (int i = w0 + lane; i < w0 + per_warp; i += 32) {
       const bool in = i < w1;
@@ -533,8 +573,6 @@ __global__ void __launch_bounds__(kRThreads, 6) topk_row_cta_kernel(const TopkPa
     }
   }
   __syncthreads();
-
-  // ---- sweep 3: emit keys > theta and the first `need` keys == theta
   int eq_acc = 0, sel_acc = 0;
   for (int w = 0; w < warp; ++w) {
     sel_acc += warp_gt[w] + min(max(need - eq_acc, 0), warp_eq[w]);
@@ -1024,12 +1062,11 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
   }
   P.slice = static_cast<int>(slice_of(cs));
   if (cs == 1) {  // many rows, one CTA each
-    const size_t smem = static_cast<size_t>(kHistBins) * sizeof(int) +
-                        static_cast<size_t>(kRowCandMax) * (sizeof(uint32_t) + sizeof(int));
-    cudaError_t e = ensure_smem_limit<topk_row_cta_kernel>(static_cast<int>(smem));
+    // The limit is raised once, to the largest slice any launch may use.
+    cudaError_t e = ensure_smem_limit<topk_row_cta_kernel>(static_cast<int>(row_cta_smem(kMaxSlice)));
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_row_cta_kernel, dim3(static_cast<unsigned>(a.Nq)), dim3(kRThreads),
-                      smem, stream, 0, P);
+                      row_cta_smem(P.slice), stream, 0, P);
   }
   const size_t smem = 2 * kBins * sizeof(int) + static_cast<size_t>(P.slice) * sizeof(uint32_t);
   // The limit is raised once, to the largest slice any launch may use.
