@@ -30,6 +30,8 @@ struct TcParams {
   int batch_ready;      // the batch arrays may be read before the dependent-launch wait
   float scale_log2;
   const __nv_bfloat16* q;  // [Nq][H][576] queries (the kernels that read them directly)
+  int wave;                // CTAs resident at once (one per SM): the many-row kernel
+                           // prefetches for row r + wave
 };
 
 // MN-major operand in the 128-byte swizzle layout: 64-element chunks along

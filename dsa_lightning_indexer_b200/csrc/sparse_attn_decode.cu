@@ -387,6 +387,7 @@ cudaError_t launch_sparse_attn_decode(const AttnArgs& a, cudaStream_t stream) {
   P.top_k = a.top_k;
   P.scale_log2 = a.scale * kLog2e;
   P.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  P.wave = 0;
   const int head_blocks = (a.H + kHB - 1) / kHB;
   e = launch_pdl(sparse_attn_decode_kernel, dim3(a.Nq, head_blocks, a.plan.n_split),
                  dim3(kThreads), static_cast<size_t>(kSmemBytes), stream, 0, qmap, P);

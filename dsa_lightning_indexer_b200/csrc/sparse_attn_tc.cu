@@ -168,6 +168,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   pdl_wait();
   pdl_launch_dependents();
+  // The CTA of row r + P.wave starts about when this one ends (one CTA per
+  // SM, rows dealt in order): its index row and query block go to L2 now,
+  // so that its first loads do not wait on DRAM.
+  // (Bulk prefetches need 16-byte aligned addresses and sizes.)
+  if (threadIdx.x == 0 && P.wave > 0 && gridDim.y == 1 && gridDim.z == 1 &&
+      r + P.wave < P.Nq) {
+    const int rn = r + P.wave;
+    const int32_t* const ip = P.idx + static_cast<size_t>(rn) * P.top_k;
+    if ((P.top_k & 3) == 0 && (reinterpret_cast<uintptr_t>(ip) & 15u) == 0) {
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ip),
+                   "r"(static_cast<uint32_t>(P.top_k) * 4u)
+                   : "memory");
+    }
+    const __nv_bfloat16* const qp = P.q + static_cast<size_t>(rn) * P.H * kLatent;
+    if ((reinterpret_cast<uintptr_t>(qp) & 15u) == 0) {
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qp),
+                   "r"(static_cast<uint32_t>(P.H) * kLatent * 2u)
+                   : "memory");
+    }
+  }
 
   const RowSeq rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
   const long long kv0 = rs.rows.kv0;  // the masked route's contiguous rows
@@ -441,16 +461,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const bool have = h0 + hl < P.H;
       const uint4* const src = reinterpret_cast<const uint4*>(
           P.q + (static_cast<size_t>(r) * P.H + h0 + hl) * kLatent);
-#pragma unroll 1
+      // All of the thread's loads are in flight before the first store.
+      uint4 x[kQTmemBoxes][4];
+#pragma unroll
+      for (int m = 0; m < kQTmemBoxes; ++m) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          x[m][j] = have ? __ldg(src + (64 * m + 32 * half) / 8 + j) : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
       for (int m = 0; m < kQTmemBoxes; ++m) {
         uint32_t v[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const uint4 x = have ? __ldg(src + (64 * m + 32 * half) / 8 + j) : make_uint4(0, 0, 0, 0);
-          v[4 * j] = x.x;
-          v[4 * j + 1] = x.y;
-          v[4 * j + 2] = x.z;
-          v[4 * j + 3] = x.w;
+          v[4 * j] = x[m][j].x;
+          v[4 * j + 1] = x[m][j].y;
+          v[4 * j + 2] = x[m][j].z;
+          v[4 * j + 3] = x[m][j].w;
         }
         tmem_st_16x32bx2_x16<16>(tmem + lane_base + kColQ + 32u * m, v);
       }
@@ -579,21 +607,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // may still be running when the last tile's softmax ends).
     if (ok && n_tiles > 0) ok = mbar_wait(b_drain, 0, P.err);
     tc_fence_after();
-    // The Q block and the gather stages are free once the last product has
-    // completed (or, with no tile, once Q has landed): the 64 heads' rows of
-    // the result are staged there, [head][512] fp32, and leave in one bulk
-    // copy, contiguous in out (and in the slice partials) for the block.
+    // With no tile, nothing is read from TMEM: the result is zero.
     if (ok && n_tiles == 0) ok = mbar_wait(b_qfull, 0, P.err);
     const bool good = !named_bar_or(1, kSoftThreads, !ok);
     if (good) {
       const bool split = P.n_split > 1;
-      float* const stg = reinterpret_cast<float*>(bp + kOffStage);
-      const int nh = min(kHB, P.H - h0);
       const size_t rec = split ? (static_cast<size_t>(sp) * P.Nq + r) * P.H
                                : static_cast<size_t>(r) * P.H;
       float* const dst = (split ? P.part_o : P.out) + (rec + h0) * kValue;
-      // Heads 0-31, then 32-63: each half leaves in its own bulk copy while
-      // the next half is staged.
+      // Straight from TMEM to global memory: for each head a warp writes 32
+      // consecutive value dims (one 128-byte line) per store; streaming
+      // stores, as nothing in this launch reads the result again.
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
 #pragma unroll 1
@@ -612,21 +636,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             const int hh = 32 * half + j;
             float v = __uint_as_float(o[j]);
             if (!split || !use_lo) v *= rl_s[hh];
-            stg[hh * kValue + dv] = v;
+            if (h0 + hh < P.H) __stcs(dst + static_cast<size_t>(hh) * kValue + dv, v);
           }
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1, kSoftThreads);
-        const int n_half = min(32, nh - 32 * half);
-        if (threadIdx.x == 0 && n_half > 0) {
-          bulk_store_issue(dst + static_cast<size_t>(32 * half) * kValue,
-                           smem_u32(stg + 32 * half * kValue),
-                           static_cast<uint32_t>(n_half * kValue * 4));
-        }
       }
-      // Shared memory must outlive the copies' reads; their writes finish
-      // on their own before the grid completes.
-      if (threadIdx.x == 0) bulk_wait_all_read();
       if (owner && h0 + hl < P.H) {
         if (split) {
           P.part_ml[rec + h0 + hl] = make_float2(m_run, l_run);
@@ -700,6 +713,12 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t stream) {
   P.top_k = a.top_k;
   P.scale_log2 = a.scale * kLog2e;
   P.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    sms = 0;
+  }
+  P.wave = sms;  // 0: no prefetch
   const int head_blocks = (a.H + kHB - 1) / kHB;
   e = launch_pdl(sparse_attn_tc_kernel<kMasked>, dim3(a.Nq, head_blocks, a.plan.n_split),
                  dim3(kThreadsTc), static_cast<size_t>(kSmemTc), stream, 0, qmap, kvmap, P);
