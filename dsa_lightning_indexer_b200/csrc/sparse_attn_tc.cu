@@ -168,27 +168,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   pdl_wait();
   pdl_launch_dependents();
-  // The CTA of row r + P.wave starts about when this one ends (one CTA per
-  // SM, rows dealt in order): its index row and query block go to L2 now,
-  // so that its first loads do not wait on DRAM.
-  // (Bulk prefetches need 16-byte aligned addresses and sizes.)
-  if (threadIdx.x == 0 && P.wave > 0 && gridDim.y == 1 && gridDim.z == 1 &&
-      r + P.wave < P.Nq) {
-    const int rn = r + P.wave;
-    const int32_t* const ip = P.idx + static_cast<size_t>(rn) * P.top_k;
-    if ((P.top_k & 3) == 0 && (reinterpret_cast<uintptr_t>(ip) & 15u) == 0) {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ip),
-                   "r"(static_cast<uint32_t>(P.top_k) * 4u)
-                   : "memory");
-    }
-    const __nv_bfloat16* const qp = P.q + static_cast<size_t>(rn) * P.H * kLatent;
-    if ((reinterpret_cast<uintptr_t>(qp) & 15u) == 0) {
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qp),
-                   "r"(static_cast<uint32_t>(P.H) * kLatent * 2u)
-                   : "memory");
-    }
-  }
-
   const RowSeq rs = row_seq_warp(P.q_offsets, P.cache, P.ctx_lens, P.B, r);
   const long long kv0 = rs.rows.kv0;  // the masked route's contiguous rows
   const int32_t* const idx_row = P.idx + static_cast<size_t>(r) * P.top_k;
@@ -282,9 +261,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                      : "memory");
       }
     };
+    // The first tile's rows are copied at once (no prefetch); later tiles'
+    // rows are prefetched one of the group's tiles ahead.
     int row_cur = load_row(grp);
     int row_nxt = load_row(grp + kStages);
-    prefetch_row(row_cur);
     bool ok = true;
     for (int t = grp; t < n_tiles && ok; t += kStages) {
       prefetch_row(row_nxt);
@@ -325,6 +305,27 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       fence_proxy_async_smem();
       mbar_arrive(b_kvfull(grp));
+    }
+    // The CTA of row r + P.wave starts about when this one ends (one CTA per
+    // SM, rows dealt in order): once this CTA's rows are all requested, its
+    // index row and query block go to L2, so that its first loads do not
+    // wait on DRAM.  Bulk prefetches need 16-byte aligned addresses and
+    // sizes.
+    if (gt == 0 && grp == 0 && ok && P.wave > 0 && gridDim.y == 1 && gridDim.z == 1 &&
+        r + P.wave < P.Nq) {
+      const int rn = r + P.wave;
+      const int32_t* const ip = P.idx + static_cast<size_t>(rn) * P.top_k;
+      if ((P.top_k & 3) == 0 && (reinterpret_cast<uintptr_t>(ip) & 15u) == 0) {
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ip),
+                     "r"(static_cast<uint32_t>(P.top_k) * 4u)
+                     : "memory");
+      }
+      const __nv_bfloat16* const qp = P.q + static_cast<size_t>(rn) * P.H * kLatent;
+      if ((reinterpret_cast<uintptr_t>(qp) & 15u) == 0) {
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(qp),
+                     "r"(static_cast<uint32_t>(P.H) * kLatent * 2u)
+                     : "memory");
+      }
     }
   } else if (warp == 4) {
     // ------------------------------------------------ Q load + MMA issue --
