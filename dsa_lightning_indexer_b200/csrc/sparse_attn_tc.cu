@@ -267,7 +267,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     int row_nxt = load_row(grp + kStages);
     bool ok = true;
     for (int t = grp; t < n_tiles && ok; t += kStages) {
-      prefetch_row(row_nxt);
+      // Later tiles prefetch while they wait for their stage; the first
+      // does so after its copies have landed (it waits on nothing before).
+      if (t != grp) prefetch_row(row_nxt);
       const uint32_t ph = static_cast<uint32_t>((t / kStages) & 1);
       ok = mbar_wait(b_kvempty(grp), ph ^ 1u, P.err);
       if (!ok) break;
@@ -305,6 +307,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       fence_proxy_async_smem();
       mbar_arrive(b_kvfull(grp));
+      if (t == grp) prefetch_row(row_cur);  // the group's next tile (row_cur moved on)
     }
     // The CTA of row r + P.wave starts about when this one ends (one CTA per
     // SM, rows dealt in order): once this CTA's rows are all requested, its
