@@ -102,3 +102,32 @@ def test_prefill_oracle_sample_and_extrapolation():
     part = bench.prefill_oracle(wl, total=40)
     assert part["kind"] == "oracle" and "EXTRAPOLATED" in part["sample"]
     assert part["value"] > 0
+
+
+def test_profiled_traffic_follows_the_source_hashes(tmp_path):
+    """The roofline's DRAM traffic comes from the committed ncu record only
+    while the kernel's sources still hash to the prefixes recorded with it."""
+    import hashlib
+    import json
+    import os
+    rec = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles",
+                                      "indexer_score_b4_128k_traffic.json")))
+    assert rec["traffic_bytes"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    # the record is close to the launch's algorithmic bytes (no re-reads)
+    assert 1.0 <= rec["traffic_bytes"] / rec["algorithmic_bytes"] < 1.01
+    csrc = os.path.join(os.path.dirname(bench.__file__), "dsa_lightning_indexer_b200", "csrc")
+    for name in rec["source_sha256_prefix"]:
+        assert os.path.exists(os.path.join(csrc, name)), name
+    good = dict(rec)
+    good["source_sha256_prefix"] = {
+        n: hashlib.sha256(open(os.path.join(csrc, n), "rb").read()).hexdigest()[:16]
+        for n in rec["source_sha256_prefix"]}
+    p = tmp_path / "good.json"
+    p.write_text(json.dumps(good))
+    assert bench.profiled_traffic(str(p)) == rec["traffic_bytes"]
+    stale = dict(good)
+    stale["source_sha256_prefix"] = {n: "0" * 16 for n in good["source_sha256_prefix"]}
+    p2 = tmp_path / "stale.json"
+    p2.write_text(json.dumps(stale))
+    assert bench.profiled_traffic(str(p2)) is None
+    assert bench.profiled_traffic(str(tmp_path / "missing.json")) is None
