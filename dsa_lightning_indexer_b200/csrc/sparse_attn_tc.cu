@@ -13,10 +13,9 @@
 //   O^T += V_tile^T[512, 48] . P^T[48, 64 heads]     M = 128 (x4), N = 64, K = 48
 // Q's first 384 dims sit in TMEM for the whole row, so the S products read
 // that part of their A operand from tensor memory and only the last 192 dims
-// from shared memory: the tensor core's operand reads from shared memory set
-// the tile rate, and Q is the largest of them.  S lands in TMEM with one head
-// per lane, so each softmax thread owns one head row: max, exp2 and row sum
-// stay in registers.  P is written to shared
+// from shared memory; the shared memory this frees holds a third gather
+// stage.  S lands in TMEM with one head per lane, so each softmax thread
+// owns one head row: max, exp2 and row sum stay in registers.  P is written to shared
 // memory as bf16 hi + lo parts (two MMAs), keeping its rounding error near
 // 2^-16, on rows with fewer than kHiOnlyRows selected; longer rows take the
 // hi part alone.  The gathered tile is stored once, in the 128-byte swizzled layout,
