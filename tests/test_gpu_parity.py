@@ -119,6 +119,12 @@ def _score_rows(lens, seed, kind):
         elif kind == "heavy":             # wide dynamic range, negatives
             sc[r, :L] = (g.standard_normal(L) * np.exp(g.standard_normal(L) * 8)).astype(
                 np.float32)
+        elif kind == "tied_cut":          # the k-th largest inside a group of 300 equal
+            v = g.standard_normal(L).astype(np.float32)  # scores spread over the row
+            if L > 2048:
+                t = np.sort(v)[::-1][1950]
+                v[np.arange(0, L, L // 300)[:300]] = t
+            sc[r, :L] = v
     return sc
 
 
@@ -136,7 +142,7 @@ ROW_SETS = {
 
 
 @pytest.mark.parametrize("rows", sorted(ROW_SETS))
-@pytest.mark.parametrize("kind", ["normal", "coarse", "zeros", "heavy"])
+@pytest.mark.parametrize("kind", ["normal", "coarse", "zeros", "heavy", "tied_cut"])
 def test_topk_long_rows(kind, rows):
     lens = ROW_SETS[rows]
     wl = synth.Workload("rows", np.arange(len(lens) + 1, dtype=np.int32),
