@@ -172,6 +172,10 @@ ATTN = {
     # of 1024 selected (P alone)
     "prefill_h80": lambda: synth.prefill(256, 80, 96, seed=118),
     "long_rows_h80_hi_only": lambda: synth.custom([1500], [40], 80, 1024, seed=119),
+    # three sequences, 600 query rows through the many-row kernel: its L2
+    # prefetch for the row one wave later crosses sequence boundaries
+    "ragged_prefill_3seq": lambda: synth.custom([600, 900, 300], [200, 300, 100], 64, 256,
+                                                seed=120),
 }
 
 
