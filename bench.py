@@ -270,6 +270,16 @@ def indexer_causal_flops(wl):
     return float(2 * synth.HI * synth.DI) * float((pos + 1).sum())
 
 
+def attention_useful_flops(wl):
+    """2 * H * (576 + 512) flops per selected key of each query row (S over
+    the 576-wide rows, P.V over their first 512 dims); a row selects
+    min(top_k, p + 1) keys."""
+    pos = wl.positions()
+    n_sel = np.minimum(wl.top_k, pos + 1).astype(np.float64)
+    H = int(wl.q.shape[1])
+    return float(2 * H * (synth.D + synth.DV)) * float(n_sel.sum())
+
+
 def launches_per_layer(wl, sms=148):
     """Kernels one dsa_layer_forward launches: when the indexer builds score
     histograms, first the kernel that zeroes their region; the indexer (one
@@ -718,6 +728,8 @@ def prefill_bench(bd, dev, peaks, args):
     fl = indexer_causal_flops(wl)
     k1s = float(np.mean(k1)) * 1e-3
     tf = fl / k1s / 1e12
+    afl = attention_useful_flops(wl)
+    atf = afl / (float(np.mean(k3)) * 1e-3) / 1e12
     extra = {}
     if getattr(args, "with_oracle", False):
         extra["cpu_baseline"] = _safe(lambda: prefill_oracle(wl))
@@ -726,7 +738,11 @@ def prefill_bench(bd, dev, peaks, args):
             "sparse_attn_ms": float(np.mean(k3)),
             "indexer_roofline": {"bound": "tensor", "achieved": tf,
                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                 "frac": tf / peaks["bf16_tflops"], "causal_flops": fl}},
+                                 "frac": tf / peaks["bf16_tflops"], "causal_flops": fl},
+            "attention_roofline": {"bound": "tensor", "achieved": atf,
+                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": atf / peaks["bf16_tflops"], "useful_flops": afl,
+                                   "note": "S and P.V over the selected keys only"}},
             **extra}
 
 

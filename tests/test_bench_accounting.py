@@ -131,3 +131,12 @@ def test_profiled_traffic_follows_the_source_hashes(tmp_path):
     p2.write_text(json.dumps(stale))
     assert bench.profiled_traffic(str(p2)) is None
     assert bench.profiled_traffic(str(tmp_path / "missing.json")) is None
+
+
+def test_prefill_16k_attention_useful_flops():
+    wl = _layout([16384], [16384], 64, 2048)
+    # rows p < 2048 select p + 1 keys, the rest 2048
+    keys = 2048 * 2049 // 2 + (16384 - 2048) * 2048
+    assert keys == 31458304
+    assert bench.attention_useful_flops(wl) == 2 * 64 * (576 + 512) * keys
+    assert bench.attention_useful_flops(wl) / 1e12 == pytest.approx(4.381, abs=1e-3)
