@@ -264,7 +264,9 @@ struct HistParams {
 
 // Finds, among `n` shared-memory keys, the `want`-th largest key theta and how
 // many keys equal to theta are needed.  Every key has the bits `known_mask`
-// equal to `known`; radix passes cover the bits in [lo_bit, hi_bit].
+// equal to `known`; radix passes cover the bits in [lo_bit, hi_bit].  (The
+// emit kernel's form, for 512 threads; the generic radix_select below,
+// inlined there instead, made that kernel spill registers.)
 __device__ void smem_select(const uint32_t* keys, int n, int want, int lo_bit, int hi_bit,
                             uint32_t known, uint32_t known_mask, int* hist /*[2048]*/, int* buf,
                             uint32_t& theta, int& need) {
